@@ -1,0 +1,626 @@
+// gemm_tc.cu -- error-compensated GEMM on sm_100a tensor cores (tcgen05 + TMA + TMEM).
+//
+// Method (authors' v2 abstract; gist.science technical summary, section 2.B): each FP32
+// operand x is split into a 16-bit primary value and a 16-bit residual,
+//     hi = r16(x),  lo = r16((x - hi) * 2^L)          (L = 11 for FP16, 0 for BF16)
+// and C = A.B is synthesised from three 16-bit products with FP32 accumulation,
+//     C ~= Ah.Bh + 2^-L (Ah.Bl + Al.Bh).
+//
+// Kernel structure (one persistent CTA per SM, 12 warps):
+//   warp 0      TMA producer: FP32 tiles of both operands, 128-byte swizzled, into a
+//               ring of shared-memory stages (one stage = 64 values of K).
+//   warp 1      MMA issuer (one thread): per stage, the two correction products into a
+//               fresh TMEM accumulator, then Ah.Bh with scale-input-d = L, which scales
+//               the corrections by 2^-L as it adds the main product, then the rest of
+//               Ah.Bh.  The accumulator is double-buffered in TMEM.
+//   warps 2-7   split warps: read the FP32 stage, write hi and lo back into the same
+//               shared memory in the UMMA 128-byte-swizzle canonical layout, fence the
+//               async proxy and release the stage to the MMA issuer.  (No split pass
+//               goes through HBM.)
+//   warps 8-11  epilogue: drain each 64-wide K chunk from TMEM and add it to the running
+//               FP32 sum in registers (round-to-nearest, ascending chunk order), then
+//               store C.  In split-K mode every chunk value goes to a workspace instead,
+//               and heal_chunk_reduce adds them in the same order.
+// Because every chunk value comes from the same sequence of tensor-core instructions and
+// chunk values are added in a fixed order, C is identical bit for bit across runs, tile
+// shapes, operand swapping and split-K.
+//
+// Operand roles inside the kernel: "kernel-A" supplies the 128 MMA rows (TMEM lanes),
+// "kernel-B" the BN MMA columns.  Normal mode: kernel-A = A, kernel-B = B^T.  Swapped mode
+// (skinny M): kernel-A = B^T (weights), kernel-B = A, and C is written transposed.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "heal_internal.h"
+#include "heal_ptx.cuh"
+#include "heal_split.cuh"
+
+namespace heal {
+
+constexpr int kBM = 128;   // MMA M: rows of kernel-A per tile (= TMEM lanes)
+constexpr int kBK = 64;    // K per stage = one accumulation chunk
+constexpr int kThreads = 384;
+constexpr int kSplitWarp0 = 2, kNumSplitWarps = 6;
+constexpr int kEpiWarp0 = 8, kNumEpiWarps = 4;
+
+struct GemmArgs {
+  int Mk, Nk, K;            // kernel-space rows of kernel-A, rows of kernel-B, reduction
+  int tiles_m, tiles_n, num_chunks;
+  int splitk;               // 1: write chunk partials to ws
+  float* out;
+  long long out_si, out_sj; // element (i, j) -> out[i*si + j*sj]
+  float* ws;                // [num_chunks][Nk][Mk] chunk values (split-K mode)
+  const int8_t* chan_exp;   // nullable, [K]
+  int expA_sign, expB_sign; // +1 / -1: which operand gets 2^+e and which 2^-e
+  unsigned int* status;     // device status word
+};
+
+template <int BN>
+struct Cfg {
+  static constexpr int kABytes = kBM * kBK * 4;             // 32 KB of FP32
+  static constexpr int kBBytes = BN * kBK * 4;
+  static constexpr int kStageBytes = kABytes + kBBytes;
+  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kTmemCols = (2 * BN) <= 32 ? 32 : (2 * BN) <= 64 ? 64 : (2 * BN) <= 128 ? 128 : (2 * BN) <= 256 ? 256 : 512;
+  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
+  static_assert(kStages >= 2, "at least two stages");
+};
+
+// ---------------------------------------------------------------------------------
+// Work iteration shared by every role: (tile, chunk) pairs in a fixed order.
+//   full-K mode : tiles blockIdx.x, +gridDim.x, ...; chunks 0..num_chunks-1 per tile
+//   split-K mode: a contiguous slice of the flattened (tile, chunk) sequence
+// ---------------------------------------------------------------------------------
+struct WorkIter {
+  int tile, chunk, u, u_end, ntiles, nc, splitk;
+  __device__ WorkIter(const GemmArgs& a) {
+    ntiles = a.tiles_m * a.tiles_n;
+    nc = a.num_chunks;
+    splitk = a.splitk;
+    if (splitk) {
+      const long long total = (long long)ntiles * nc;
+      u = (int)((total * blockIdx.x) / gridDim.x);
+      u_end = (int)((total * (blockIdx.x + 1)) / gridDim.x);
+      tile = u / nc;
+      chunk = u % nc;
+    } else {
+      tile = blockIdx.x;
+      chunk = 0;
+      u = 0;
+      u_end = 0;
+    }
+  }
+  __device__ bool valid() const { return splitk ? (u < u_end) : (tile < ntiles); }
+  __device__ void advance() {
+    if (splitk) {
+      ++u;
+      tile = u / nc;
+      chunk = u % nc;
+    } else if (++chunk == nc) {
+      chunk = 0;
+      tile += gridDim.x;
+    }
+  }
+};
+
+// Tile raster: groups of 8 kernel-A row tiles, column tiles inside a group.
+__device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int& tm, int& tn) {
+  constexpr int GM = 8;
+  const int group = GM * tiles_n;
+  const int g = tile / group;
+  const int first_m = g * GM;
+  const int gm = min(tiles_m - first_m, GM);
+  const int local = tile - g * group;
+  tm = first_m + local % gm;
+  tn = local / gm;
+}
+
+// ---------------------------------------------------------------------------------
+// TMA of one operand tile (R rows x 64 K) into a stage.
+//   K-major  (K contiguous) : two boxes {32 K, R rows} -> [0, R*128) and [R*128, R*256)
+//   MN-major (rows contiguous): R/32 boxes {32 rows, 64 K} -> b*8192
+//   16-bit pre-split input   : hi/lo boxes of 64 values that land exactly where the
+//                              in-place split would have written them.
+// ---------------------------------------------------------------------------------
+template <int R, bool MN, bool PRESPLIT>
+__device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, const CUtensorMap* map_lo,
+                                             uint64_t* bar, int row0, int k0) {
+  if constexpr (!PRESPLIT) {
+    if constexpr (!MN) {
+      tma_load_2d(dst, map, bar, k0, row0);
+      tma_load_2d(dst + R * 128, map, bar, k0 + 32, row0);
+    } else {
+#pragma unroll
+      for (int b = 0; b < R / 32; ++b) tma_load_2d(dst + b * 8192, map, bar, row0 + 32 * b, k0);
+    }
+  } else {
+    if constexpr (!MN) {
+      tma_load_2d(dst, map, bar, k0, row0);              // hi: R rows x 64 values
+      tma_load_2d(dst + R * 128, map_lo, bar, k0, row0);  // lo
+    } else {
+#pragma unroll
+      for (int p = 0; p < R / 64; ++p) {
+        tma_load_2d(dst + (2 * p) * 8192, map, bar, row0 + 64 * p, k0);
+        tma_load_2d(dst + (2 * p + 1) * 8192, map_lo, bar, row0 + 64 * p, k0);
+      }
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// In-place split of one 2 KB region pair by one warp.
+// src0/src1 each hold one 128-byte-swizzled atom of 8 rows x 32 FP32 values; together
+// they are 8 rows x 64 values.  Afterwards src0 holds the 16-bit hi atom (8 rows x 64)
+// and src1 the lo atom, both in the 128-byte-swizzle canonical layout.
+// Lane -> (atom row = lane & 7, quarter = lane >> 3): conflict-free 16-byte accesses.
+// kb: K index of the region's first value (K-major) or first row (MN-major), used for
+// the optional channel exponents; values at K >= K are TMA zero fill and stay zero.
+// ---------------------------------------------------------------------------------
+__device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
+
+template <int FMT, bool MN>
+__device__ __forceinline__ void split_pair(uint8_t* src0, uint8_t* src1, int lane, const int8_t* chan_exp,
+                                           int exp_sign, int kb, int K) {
+  const int row = lane & 7, q = lane >> 3;
+  uint8_t* r0 = src0 + row * 128;
+  uint8_t* r1 = src1 + row * 128;
+  float v[16];
+  *reinterpret_cast<float4*>(&v[0]) = *reinterpret_cast<const float4*>(r0 + (((2 * q) ^ row) << 4));
+  *reinterpret_cast<float4*>(&v[4]) = *reinterpret_cast<const float4*>(r0 + (((2 * q + 1) ^ row) << 4));
+  *reinterpret_cast<float4*>(&v[8]) = *reinterpret_cast<const float4*>(r1 + (((2 * q) ^ row) << 4));
+  *reinterpret_cast<float4*>(&v[12]) = *reinterpret_cast<const float4*>(r1 + (((2 * q + 1) ^ row) << 4));
+  if (chan_exp != nullptr) {
+    if constexpr (MN) {
+      // every value of this lane has K index kb + row
+      const int k = kb + row;
+      const float s = k < K ? pow2f(exp_sign * (int)__ldg(chan_exp + k)) : 0.0f;   // beyond K: TMA zero fill
+#pragma unroll
+      for (int t = 0; t < 16; ++t) v[t] = __fmul_rn(v[t], s);
+    } else {
+      // K index of value t: kb + 8q + t (t < 8), kb + 32 + 8q + (t - 8)
+#pragma unroll
+      for (int t = 0; t < 16; ++t) {
+        const int k = kb + (t < 8 ? 8 * q + t : 32 + 8 * q + (t - 8));
+        if (k < K) v[t] = __fmul_rn(v[t], pow2f(exp_sign * (int)__ldg(chan_exp + k)));
+      }
+    }
+  }
+  __syncwarp();
+  uint4 h0, h1, l0, l1;
+  h0.x = split2<FMT>(v[0], v[1], l0.x);
+  h0.y = split2<FMT>(v[2], v[3], l0.y);
+  h0.z = split2<FMT>(v[4], v[5], l0.z);
+  h0.w = split2<FMT>(v[6], v[7], l0.w);
+  h1.x = split2<FMT>(v[8], v[9], l1.x);
+  h1.y = split2<FMT>(v[10], v[11], l1.y);
+  h1.z = split2<FMT>(v[12], v[13], l1.z);
+  h1.w = split2<FMT>(v[14], v[15], l1.w);
+  *reinterpret_cast<uint4*>(r0 + ((q ^ row) << 4)) = h0;
+  *reinterpret_cast<uint4*>(r0 + (((4 + q) ^ row) << 4)) = h1;
+  *reinterpret_cast<uint4*>(r1 + ((q ^ row) << 4)) = l0;
+  *reinterpret_cast<uint4*>(r1 + (((4 + q) ^ row) << 4)) = l1;
+}
+
+// Region pair t of an operand tile with R rows (t in [0, R/8)).
+template <int R, bool MN>
+__device__ __forceinline__ void pair_addr(uint8_t* base, int t, uint8_t*& s0, uint8_t*& s1, int& kb_off) {
+  if constexpr (!MN) {
+    s0 = base + t * 1024;
+    s1 = base + R * 128 + t * 1024;
+    kb_off = 0;
+  } else {
+    const int p = t >> 3, j = t & 7;
+    s0 = base + (2 * p) * 8192 + j * 1024;
+    s1 = base + (2 * p + 1) * 8192 + j * 1024;
+    kb_off = 8 * j;
+  }
+}
+
+// Shared-memory descriptors of the hi / lo tiles of an operand with R rows.
+template <int R, bool MN>
+struct OperandDesc {
+  static __device__ __forceinline__ uint64_t hi(uint32_t base) {
+    return MN ? smem_desc_sw128(base, 16384, 1024) : smem_desc_sw128(base, 16, 1024);
+  }
+  static __device__ __forceinline__ uint64_t lo(uint32_t base) {
+    return MN ? smem_desc_sw128(base + 8192, 16384, 1024) : smem_desc_sw128(base + R * 128, 16, 1024);
+  }
+  // advance by one K=16 step (descriptor address field counts 16-byte units)
+  static constexpr uint64_t kStep = MN ? (2048 >> 4) : (32 >> 4);
+};
+
+// ---------------------------------------------------------------------------------
+// The kernel
+// ---------------------------------------------------------------------------------
+template <int BN, bool A_MN, bool B_MN, int FMT, bool CORR_SWAP, bool A_PRE, bool B_PRE>
+__global__ void __launch_bounds__(kThreads, 1)
+    heal_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA_lo,
+                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB_lo,
+                     const GemmArgs args) {
+  using C = Cfg<BN>;
+  constexpr int S = C::kStages;
+  constexpr int kLoShift = FMT == 0 ? 11 : 0;
+  constexpr uint32_t kIdesc = idesc_f16(kBM, BN, FMT, A_MN ? 1 : 0, B_MN ? 1 : 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment of the shared-window address (128-byte swizzle atoms)
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  uint64_t* full = bars;                 // TMA -> split       (tx bytes)
+  uint64_t* split_done = bars + S;       // split -> MMA       (all split threads arrive)
+  uint64_t* empty = bars + 2 * S;        // MMA -> TMA         (tcgen05.commit)
+  uint64_t* acc_full = bars + 3 * S;     // MMA -> epilogue    (tcgen05.commit)
+  uint64_t* acc_empty = bars + 3 * S + 2;// epilogue -> MMA    (128 arrivals)
+  uint64_t* mma_done = bars + 3 * S + 4; // MMA drain on exit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&split_done[s], kNumSplitWarps * 32);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kNumEpiWarps * 32);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  if (warp == 1 && lane == 0) {
+    tma_prefetch_desc(&tmA);
+    tma_prefetch_desc(&tmB);
+    if (A_PRE) tma_prefetch_desc(&tmA_lo);
+    if (B_PRE) tma_prefetch_desc(&tmB_lo);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    if (lane == 0) {
+      int it = 0;
+      for (WorkIter w(args); w.valid(); w.advance(), ++it) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)(it / S) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, args.status, 100)) break;
+        int tm, tn;
+        tile_coords(w.tile, args.tiles_m, args.tiles_n, tm, tn);
+        const int k0 = w.chunk * kBK;
+        uint8_t* st = stages + s * C::kStageBytes;
+        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
+        load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, &full[s], tm * kBM, k0);
+        load_operand<BN, B_MN, B_PRE>(st + C::kABytes, &tmB, &tmB_lo, &full[s], tn * BN, k0);
+      }
+      // Do not leave the CTA with copies in flight: wait (bounded) for the last fill of
+      // every stage that was issued.
+      for (int j = 0; j < S && j < it; ++j) {
+        const int jt = it - 1 - j;
+        volatile int dummy = 0;
+        mbar_wait(&full[jt % S], (uint32_t)(jt / S) & 1u, &dummy, args.status, 101);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer ------------------------------
+    if (lane == 0) {
+      int it = 0;
+      for (WorkIter w(args); w.valid(); w.advance(), ++it) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)(it / S) & 1u;
+        const int b = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(&split_done[s], ph, abort_flag, args.status, 110)) break;
+        if (!mbar_wait(&acc_empty[b], aph ^ 1u, abort_flag, args.status, 111)) break;
+        tc_fence_after();
+        const uint32_t sa = smem_u32(stages + s * C::kStageBytes);
+        const uint32_t sb = sa + C::kABytes;
+        const uint64_t a_hi = OperandDesc<kBM, A_MN>::hi(sa), a_lo = OperandDesc<kBM, A_MN>::lo(sa);
+        const uint64_t b_hi = OperandDesc<BN, B_MN>::hi(sb), b_lo = OperandDesc<BN, B_MN>::lo(sb);
+        constexpr uint64_t dA = OperandDesc<kBM, A_MN>::kStep, dB = OperandDesc<BN, B_MN>::kStep;
+        const uint32_t d = tmem_base + (uint32_t)(b * BN);
+        // corrections first: Ah.Bl then Al.Bh in the caller's operand order
+#pragma unroll
+        for (int j = 0; j < kBK / 16; ++j) {
+          if constexpr (!CORR_SWAP) {
+            mma_f16(d, a_hi + j * dA, b_lo + j * dB, kIdesc, j > 0 ? 1u : 0u);
+            mma_f16(d, a_lo + j * dA, b_hi + j * dB, kIdesc, 1u);
+          } else {
+            mma_f16(d, a_lo + j * dA, b_hi + j * dB, kIdesc, j > 0 ? 1u : 0u);
+            mma_f16(d, a_hi + j * dA, b_lo + j * dB, kIdesc, 1u);
+          }
+        }
+        // main product; its first step scales the corrections by 2^-L
+        mma_f16_scale_d<kLoShift>(d, a_hi, b_hi, kIdesc);
+#pragma unroll
+        for (int j = 1; j < kBK / 16; ++j) mma_f16(d, a_hi + j * dA, b_hi + j * dB, kIdesc, 1u);
+        tc_commit(&empty[s]);
+        tc_commit(&acc_full[b]);
+      }
+      // drain: every MMA issued by this thread has completed before TMEM is released
+      tc_commit(mma_done);
+      volatile int dummy = 0;
+      mbar_wait(mma_done, 0, &dummy, args.status, 112);
+    }
+  } else if (warp < kEpiWarp0) {
+    // ------------------------------ split warps ------------------------------
+    const int sw = warp - kSplitWarp0;
+    constexpr int kPairsA = kBM / 8, kPairsB = BN / 8;
+    int it = 0;
+    for (WorkIter w(args); w.valid(); w.advance(), ++it) {
+      const int s = it % S;
+      const uint32_t ph = (uint32_t)(it / S) & 1u;
+      if (!mbar_wait(&full[s], ph, abort_flag, args.status, 120)) break;
+      uint8_t* st = stages + s * C::kStageBytes;
+      const int k0 = w.chunk * kBK;
+      constexpr int kFirst = A_PRE ? kPairsA : 0;
+      constexpr int kLast = B_PRE ? kPairsA : kPairsA + kPairsB;
+      for (int t = kFirst + sw; t < kLast; t += kNumSplitWarps) {
+        uint8_t *s0, *s1;
+        int kboff;
+        if (t < kPairsA) {
+          pair_addr<kBM, A_MN>(st, t, s0, s1, kboff);
+          split_pair<FMT, A_MN>(s0, s1, lane, args.chan_exp, args.expA_sign, k0 + kboff, args.K);
+        } else {
+          pair_addr<BN, B_MN>(st + C::kABytes, t - kPairsA, s0, s1, kboff);
+          split_pair<FMT, B_MN>(s0, s1, lane, args.chan_exp, args.expB_sign, k0 + kboff, args.K);
+        }
+      }
+      fence_proxy_async_smem();
+      mbar_arrive(&split_done[s]);
+    }
+  } else {
+    // ------------------------------ epilogue ------------------------------
+    const int quarter = warp & 3;            // TMEM lanes this warp may access
+    const int i_local = quarter * 32 + lane; // tile row
+    float acc[BN];
+#pragma unroll
+    for (int t = 0; t < BN; ++t) acc[t] = 0.0f;
+    int it = 0;
+    bool ok = true;
+    for (WorkIter w(args); w.valid(); w.advance(), ++it) {
+      const int b = it & 1;
+      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      if (!mbar_wait(&acc_full[b], aph, abort_flag, args.status, 130)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      int tm, tn;
+      tile_coords(w.tile, args.tiles_m, args.tiles_n, tm, tn);
+      const int gi = tm * kBM + i_local;
+      const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * BN);
+      if (!args.splitk) {
+        const bool first = (w.chunk == 0);
+#pragma unroll
+        for (int c = 0; c < BN / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c * 16, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float dv = __uint_as_float(r[t]);
+            acc[c * 16 + t] = first ? dv : __fadd_rn(acc[c * 16 + t], dv);
+          }
+        }
+      } else {
+        float* wsc = args.ws + (size_t)w.chunk * args.Nk * args.Mk;
+#pragma unroll
+        for (int c = 0; c < BN / 16; ++c) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c * 16, r);
+          tmem_ld_wait();
+          if (gi < args.Mk) {
+#pragma unroll
+            for (int t = 0; t < 16; ++t) {
+              const int gj = tn * BN + c * 16 + t;
+              if (gj < args.Nk) wsc[(size_t)gj * args.Mk + gi] = __uint_as_float(r[t]);
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&acc_empty[b]);
+      if (!args.splitk && w.chunk == w.nc - 1 && gi < args.Mk) {
+        // store the finished row slice of C
+        const int gj0 = tn * BN;
+        if (args.out_sj == 1) {
+          float* orow = args.out + (size_t)gi * args.out_si + gj0;
+          const bool vec = ((reinterpret_cast<uintptr_t>(orow) & 15) == 0) && (gj0 + BN <= args.Nk);
+          if (vec) {
+#pragma unroll
+            for (int t = 0; t < BN; t += 4)
+              *reinterpret_cast<float4*>(orow + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
+          } else {
+#pragma unroll
+            for (int t = 0; t < BN; ++t)
+              if (gj0 + t < args.Nk) orow[t] = acc[t];
+          }
+        } else {
+#pragma unroll
+          for (int t = 0; t < BN; ++t)
+            if (gj0 + t < args.Nk) args.out[(size_t)gi * args.out_si + (size_t)(gj0 + t) * args.out_sj] = acc[t];
+        }
+      }
+    }
+    (void)ok;
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem_base, C::kTmemCols);
+}
+
+// Ordered sum of chunk values: out(i, j) = ((ws[0] + ws[1]) + ws[2]) + ...
+__global__ void heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk, int Nk, float* out,
+                                         long long si, long long sj) {
+  const long long total = (long long)Mk * Nk;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const int i = (int)(e % Mk), j = (int)(e / Mk);
+    const float* p = ws + (size_t)j * Mk + i;
+    float acc = p[0];
+    for (int c = 1; c < num_chunks; ++c) acc = __fadd_rn(acc, p[(size_t)c * Mk * Nk]);
+    out[(size_t)i * si + (size_t)j * sj] = acc;
+  }
+}
+
+// ---------------------------------------------------------------------------------
+// Host side
+// ---------------------------------------------------------------------------------
+namespace {
+
+bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, int elem_bytes, const void* base, uint64_t inner,
+               uint64_t outer, uint64_t row_stride_elems, uint32_t box_inner, uint32_t box_outer) {
+  const cuuint64_t dims[2] = {inner, outer};
+  const cuuint64_t strides[1] = {row_stride_elems * (uint64_t)elem_bytes};
+  const cuuint32_t box[2] = {box_inner, box_outer};
+  const cuuint32_t estr[2] = {1, 1};
+  return encode_tensor_map(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// Operand tensor map: R rows of the tile, matrix with `rows` rows and K columns where
+// element (row, k) lives at base[row*ld + k] (K-major) or base[k*ld + row] (MN-major).
+bool operand_map(CUtensorMap* map, const void* base, bool mn, bool is16, int rows, int K, long long ld, int R) {
+  const CUtensorMapDataType dt = is16 ? CU_TENSOR_MAP_DATA_TYPE_UINT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32;
+  const int eb = is16 ? 2 : 4;
+  const uint32_t inner_box = is16 ? 64u : 32u;   // 128 bytes
+  if (!mn) return encode_2d(map, dt, eb, base, (uint64_t)K, (uint64_t)rows, (uint64_t)ld, inner_box, (uint32_t)R);
+  return encode_2d(map, dt, eb, base, (uint64_t)rows, (uint64_t)K, (uint64_t)ld, inner_box, 64u);
+}
+
+template <int BN, bool A_MN, bool B_MN, int FMT, bool CORR_SWAP, bool A_PRE, bool B_PRE>
+cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& alo, const CUtensorMap& b,
+                           const CUtensorMap& blo, const GemmArgs& args, int grid, cudaStream_t stream) {
+  auto kern = heal_gemm_kernel<BN, A_MN, B_MN, FMT, CORR_SWAP, A_PRE, B_PRE>;
+  const int smem = Cfg<BN>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kThreads, smem, stream>>>(a, alo, b, blo, args);
+  return cudaGetLastError();
+}
+
+template <int BN, bool A_MN, bool B_MN, bool CORR_SWAP, bool A_PRE, bool B_PRE>
+cudaError_t launch_fmt(int fmt, const CUtensorMap& a, const CUtensorMap& alo, const CUtensorMap& b,
+                       const CUtensorMap& blo, const GemmArgs& args, int grid, cudaStream_t stream) {
+  if (fmt == 0) return launch_variant<BN, A_MN, B_MN, 0, CORR_SWAP, A_PRE, B_PRE>(a, alo, b, blo, args, grid, stream);
+  return launch_variant<BN, A_MN, B_MN, 1, CORR_SWAP, A_PRE, B_PRE>(a, alo, b, blo, args, grid, stream);
+}
+
+}  // namespace
+
+size_t gemm_workspace_bytes(int M, int N, int K, int tile_config) {
+  if (tile_config != HEAL_TILE_SKINNY_SPLITK) return 0;
+  const size_t nc = (size_t)((K + kBK - 1) / kBK);
+  const size_t mpad = (size_t)(M <= 16 ? 16 : M <= 32 ? 32 : 64);
+  (void)mpad;
+  return nc * (size_t)M * (size_t)N * sizeof(float);
+}
+
+heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, const void* B, long long ldb,
+                          float* Cout, long long ldc, int fmt, const heal_gemm_opts_t& o, cudaStream_t stream) {
+  int cfg = o.tile_config;
+  if (cfg == HEAL_TILE_AUTO) {
+    cfg = (M <= 64 && o.workspace != nullptr && o.workspace_bytes >= gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK) &&
+           !o.b_presplit)
+              ? HEAL_TILE_SKINNY_SPLITK
+              : HEAL_TILE_128x128;
+  }
+  const int sms = device_sm_count();
+  if (sms <= 0) return HEAL_ERR_CUDA;
+  const bool b_mn = (o.b_layout == 0);   // B stored K x N: N contiguous
+  const int nc = (K + kBK - 1) / kBK;
+  CUtensorMap ta{}, talo{}, tb{}, tblo{};
+  GemmArgs args{};
+  args.K = K;
+  args.num_chunks = nc;
+  args.chan_exp = o.chan_exp;
+  args.status = device_status_ptr();
+  cudaError_t err = cudaSuccess;
+
+  if (cfg == HEAL_TILE_128x128 || cfg == HEAL_TILE_128x256) {
+    if (cfg == HEAL_TILE_128x256) return HEAL_ERR_UNSUPPORTED;   // not built in this version
+    constexpr int BN = 128;
+    args.Mk = M;
+    args.Nk = N;
+    args.tiles_m = (M + kBM - 1) / kBM;
+    args.tiles_n = (N + BN - 1) / BN;
+    args.splitk = 0;
+    args.out = Cout;
+    args.out_si = ldc;
+    args.out_sj = 1;
+    args.expA_sign = -1;
+    args.expB_sign = +1;
+    if (!operand_map(&ta, A, false, false, M, K, lda, kBM)) return HEAL_ERR_CUDA;
+    if (!o.b_presplit) {
+      if (!operand_map(&tb, B, b_mn, false, N, K, ldb, BN)) return HEAL_ERR_CUDA;
+    } else {
+      if (!operand_map(&tb, B, b_mn, true, N, K, ldb, BN)) return HEAL_ERR_CUDA;
+      if (!operand_map(&tblo, o.b_lo, b_mn, true, N, K, ldb, BN)) return HEAL_ERR_CUDA;
+    }
+    const int ntiles = args.tiles_m * args.tiles_n;
+    const int grid = ntiles < sms ? ntiles : sms;
+    if (!o.b_presplit) {
+      err = b_mn ? launch_fmt<BN, false, true, false, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
+                 : launch_fmt<BN, false, false, false, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
+    } else {
+      err = b_mn ? launch_fmt<BN, false, true, false, false, true>(fmt, ta, talo, tb, tblo, args, grid, stream)
+                 : launch_fmt<BN, false, false, false, false, true>(fmt, ta, talo, tb, tblo, args, grid, stream);
+    }
+    return err == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+  }
+
+  if (cfg == HEAL_TILE_SKINNY_SPLITK) {
+    if (o.b_presplit) return HEAL_ERR_UNSUPPORTED;
+    if (M > 64) return HEAL_ERR_UNSUPPORTED;
+    if (o.workspace == nullptr || o.workspace_bytes < gemm_workspace_bytes(M, N, K, cfg)) return HEAL_ERR_INVALID_ARGUMENT;
+    // swapped roles: kernel-A = B^T (N rows), kernel-B = A (M rows), C written transposed
+    args.Mk = N;
+    args.Nk = M;
+    args.tiles_m = (N + kBM - 1) / kBM;
+    args.tiles_n = 1;
+    args.splitk = 1;
+    args.ws = static_cast<float*>(o.workspace);
+    args.out = Cout;
+    args.out_si = 1;
+    args.out_sj = ldc;
+    args.expA_sign = +1;
+    args.expB_sign = -1;
+    const int BNk = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    if (!operand_map(&ta, B, b_mn, false, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
+    if (!operand_map(&tb, A, false, false, M, K, lda, BNk)) return HEAL_ERR_CUDA;
+    const long long units = (long long)args.tiles_m * nc;
+    const int grid = (int)(units < sms ? units : sms);
+    if (BNk == 16)
+      err = b_mn ? launch_fmt<16, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
+                 : launch_fmt<16, false, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
+    else if (BNk == 32)
+      err = b_mn ? launch_fmt<32, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
+                 : launch_fmt<32, false, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
+    else
+      err = b_mn ? launch_fmt<64, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
+                 : launch_fmt<64, false, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
+    if (err != cudaSuccess) return HEAL_ERR_CUDA;
+    const long long total = (long long)M * N;
+    int rgrid = (int)((total + 255) / 256);
+    if (rgrid > 4 * sms) rgrid = 4 * sms;
+    heal_chunk_reduce_kernel<<<rgrid, 256, 0, stream>>>(args.ws, nc, N, M, Cout, 1, ldc);
+    return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+  }
+  return HEAL_ERR_UNSUPPORTED;
+}
+
+}  // namespace heal

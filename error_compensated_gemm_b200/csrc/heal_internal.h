@@ -1,0 +1,38 @@
+// heal_internal.h -- declarations shared by the library's translation units.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "../../include/heal.h"
+
+namespace heal {
+
+// SM count of the current device (cached per device); <= 0 on error.
+int device_sm_count();
+
+// Device address of the status word on the current device (nullptr on error).
+unsigned int* device_status_ptr();
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point (no libcuda link).
+bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, cuuint32_t rank, void* base,
+                       const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
+                       const cuuint32_t* elem_strides, CUtensorMapSwizzle swizzle);
+
+heal_status_t split_launch(const float* x, void* hi, void* lo, long long n, int fmt, cudaStream_t s);
+
+size_t gemm_workspace_bytes(int M, int N, int K, int tile_config);
+heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, const void* B, long long ldb,
+                          float* C, long long ldc, int fmt, const heal_gemm_opts_t& o, cudaStream_t s);
+
+heal_status_t kv_quant_launch(const void* x, int is_bf16, int B, int T, int H, int D, long long sb,
+                              long long st, long long sh, int16_t* q, float* sc, int Tmax, int t_off,
+                              cudaStream_t s);
+
+size_t attention_workspace_bytes(int B, int Hq, int Tq, int Tmax);
+heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t* k, const float* ks,
+                               const int16_t* v, const float* vs, int B, int Hq, int Hkv, int D, int Tq,
+                               const int32_t* kv_len, int Tmax, float scale, int causal, float* out,
+                               void* ws, size_t ws_bytes, int64_t* qk_out, cudaStream_t s);
+
+}  // namespace heal

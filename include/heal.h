@@ -1,0 +1,177 @@
+/*
+ * heal.h -- C ABI of libheal.so, the B200 (sm_100a) hot path of HEAL.
+ *
+ * HEAL ("Demystifying Numerical Instability in LLM Inference: Achieving Reproducible
+ * Inference for Mission-Critical Tasks with HEAL", arXiv 2606.21023) keeps FP32-level
+ * numerics without an FP32 pipeline:
+ *   - GEMMs are synthesised on 16-bit tensor cores by algebraic error compensation
+ *     (authors' v2 abstract; gist.science technical summary, section 2.B);
+ *   - Q/K/V are stored as INT16 and unpacked into FP16 pairs for the attention
+ *     contractions (abstract; technical summary, section 2.A).
+ *
+ * Conventions for every call:
+ *   - All tensor pointers are DEVICE pointers owned by the caller.  The library never
+ *     allocates, frees or retains them; scratch comes from caller-provided workspaces.
+ *   - Every call is asynchronous and stream-ordered on `stream` (NULL = legacy default
+ *     stream).  Arguments are validated on the host before any launch; a rejected call
+ *     launches nothing and leaves every output untouched.
+ *   - Return codes: HEAL_OK, HEAL_ERR_INVALID_ARGUMENT (null pointer, bad size, stride
+ *     or alignment), HEAL_ERR_UNSUPPORTED (valid but outside what the kernels cover),
+ *     HEAL_ERR_CUDA (a CUDA runtime error at launch; the CUDA error is cleared).
+ *     Device-side failures (a bounded wait that ran out) are reported asynchronously by
+ *     heal_get_device_status().
+ *   - Matrices are row-major with explicit leading dimensions in elements.  No C++
+ *     exception crosses this boundary.
+ */
+#ifndef HEAL_H_
+#define HEAL_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream. */
+typedef struct CUstream_st* heal_stream_t;
+
+typedef enum {
+  HEAL_OK = 0,
+  HEAL_ERR_INVALID_ARGUMENT = 1,
+  HEAL_ERR_UNSUPPORTED = 2,
+  HEAL_ERR_CUDA = 3,
+  HEAL_ERR_TIMEOUT = 4
+} heal_status_t;
+
+/* 16-bit format of the hi/lo residual split (technical summary, section 2.B: "a primary
+ * 16-bit value and a residual error term"; the overflow remark there names FP16).
+ *   HEAL_SPLIT_FP16_S11: hi = fp16_rn(x), lo = fp16_rn((x - hi) * 2^11); the products
+ *                        that use lo are scaled by 2^-11.  Default; FP32-level accuracy.
+ *   HEAL_SPLIT_BF16:     hi = bf16_rn(x), lo = bf16_rn(x - hi).  Wider range, ~16 bits. */
+typedef enum { HEAL_SPLIT_FP16_S11 = 0, HEAL_SPLIT_BF16 = 1 } heal_split_fmt_t;
+
+/* Fixed tile configurations of heal_gemm_compensated.  All configurations produce
+ * bitwise-identical C (see heal_gemm_compensated).  HEAL_TILE_AUTO picks by shape. */
+enum {
+  HEAL_TILE_AUTO = -1,
+  HEAL_TILE_128x128 = 0,      /* 1 CTA per tile, full K per tile                        */
+  HEAL_TILE_128x256 = 1,      /* 1 CTA per tile, wider N                                */
+  HEAL_TILE_SKINNY_SPLITK = 2 /* operands swapped (weights on the MMA M side), K split
+                                 over CTAs; needs a workspace                           */
+};
+
+typedef struct {
+  int tile_config;          /* HEAL_TILE_* ; -1 = automatic                                  */
+  const int8_t* chan_exp;   /* nullable device pointer, int8 [K]: outlier-channel rescale.
+                               Column k of A is multiplied by 2^-e_k and row k of B by 2^e_k
+                               before the split.  Powers of two, so A.B is unchanged; it
+                               keeps FP16 hi parts finite for large channels (technical
+                               summary, section 2.B, "Overflow Handling").  |e_k| <= 64.   */
+  int b_layout;             /* 0: B is K x N row-major (ldb >= N); 1: B is N x K row-major
+                               (ldb >= K), the torch.nn.Linear weight layout                 */
+  int b_presplit;           /* 1: `B` holds the 16-bit hi part and `b_lo` the lo part, both
+                               written by heal_split in `fmt`, in b_layout.  The kernel then
+                               splits only A.                                               */
+  const void* b_lo;         /* lo part when b_presplit = 1                                   */
+  void* workspace;          /* device scratch for HEAL_TILE_SKINNY_SPLITK (nullable)        */
+  size_t workspace_bytes;
+  int reserved[4];          /* must be zero                                                  */
+} heal_gemm_opts_t;
+
+/* K1. Hi/lo split of n FP32 values (technical summary, section 2.B, "Mechanism").
+ *   x  : device, float32 [n]
+ *   hi : device, 16-bit [n] (fp16 or bf16 encodings per fmt), written
+ *   lo : device, 16-bit [n], written
+ * Elementwise, round-to-nearest-even; |x| >= 65520 gives an infinite FP16 hi.
+ * n == 0 is a no-op.  Pointers must be 4-byte aligned (16-byte for full speed).      */
+heal_status_t heal_split(const float* x, void* hi, void* lo, int64_t n,
+                         heal_split_fmt_t fmt, heal_stream_t stream);
+
+/* K2/K3. Error-compensated GEMM  C = A . B  on 16-bit tensor cores (authors' abstract;
+ * technical summary, section 2.B).
+ *   A : device float32, M x K row-major, leading dimension lda >= K
+ *   B : device float32 (or 16-bit hi when opts->b_presplit), layout per opts->b_layout
+ *   C : device float32, M x N row-major, ldc >= N; FP32 result, no 16-bit store.
+ * Both operands are split into hi/lo in shared memory by the kernel and
+ *   C = Ah.Bh + s.(Ah.Bl + Al.Bh),  s = 2^-11 (FP16_S11) or 1 (BF16),
+ * with FP32 accumulation.  K is processed in chunks of 64: each chunk's value comes
+ * from the tensor cores, and chunk values are added in ascending order in FP32 round-
+ * to-nearest.  The result is therefore identical bit for bit across runs and across
+ * tile configurations.
+ * Alignment: A, B, C (and b_lo) 16-byte aligned; lda, ldb multiples of 4 (8 for a
+ * pre-split B).  M, N, K >= 1 and < 2^31.  HEAL_TILE_SKINNY_SPLITK needs
+ * opts->workspace of at least heal_gemm_workspace_bytes(); other configs need none.   */
+heal_status_t heal_gemm_compensated(int M, int N, int K,
+                                    const float* A, int64_t lda,
+                                    const void* B, int64_t ldb,
+                                    float* C, int64_t ldc,
+                                    heal_split_fmt_t fmt,
+                                    const heal_gemm_opts_t* opts, /* nullable: defaults */
+                                    heal_stream_t stream);
+
+/* Workspace bytes that heal_gemm_compensated needs for this shape and tile config
+ * (0 when the config uses none).  Host-only, no CUDA call.                            */
+size_t heal_gemm_workspace_bytes(int M, int N, int K, const heal_gemm_opts_t* opts);
+
+/* K4. INT16 quantization of Q/K/V rows into a cache (technical summary, section 2.A).
+ *   x : device, bf16 (x_is_bf16 = 1) or float32, logical [B, T, H, D] with element
+ *       strides (x_stride_batch, x_stride_tok, x_stride_head, 1)
+ *   q_cache     : device int16 [B, H, Tmax, D], rows t_offset .. t_offset+T-1 written
+ *   scale_cache : device float32 [B, H, Tmax], same rows written
+ * Per (token, head) row: absmax = max|x|, inv = fp32(32767/absmax),
+ * q = clamp(rint(fp32(x*inv)), +-32767), s = fp32(absmax/32767); an all-zero row gives
+ * q = 0, s = 0.  D must be a multiple of 8 and <= 256; x, q_cache 16-byte aligned;
+ * strides multiples of 8 elements.  t_offset + T <= Tmax.                              */
+heal_status_t heal_kv_quantize_int16(const void* x, int x_is_bf16,
+                                     int B, int T, int H, int D,
+                                     int64_t x_stride_batch, int64_t x_stride_tok,
+                                     int64_t x_stride_head,
+                                     int16_t* q_cache, float* scale_cache,
+                                     int Tmax, int t_offset, heal_stream_t stream);
+
+/* K5. Attention on INT16 Q/K/V (technical summary, section 2.A "Mechanism").
+ *   q          : device int16 [B, Hq, Tq, D]        q_scale : float32 [B, Hq, Tq]
+ *   k_cache    : device int16 [B, Hkv, Tmax, D]     k_scale : float32 [B, Hkv, Tmax]
+ *   v_cache    : device int16 [B, Hkv, Tmax, D]     v_scale : float32 [B, Hkv, Tmax]
+ *   kv_len     : device int32 [B], 1 <= kv_len[b] <= Tmax (tokens 0..kv_len-1 valid)
+ *   out        : device float32 [B, Hq, Tq, D]
+ * Query head h reads KV head h / (Hq/Hkv).  Query i sits at position kv_len - Tq + i;
+ * with causal = 1 it sees tokens t <= its position.  QK^T is the exact integer dot
+ * product (each INT16 value byte-split into two FP16 values, three FP16 tensor-core
+ * products, combined in int64); logit = fp32(S_int * (s_q * s_k) * softmax_scale)
+ * evaluated in double; FP32 online softmax; PV with P split into two FP16 parts and V
+ * byte-split.  The context is cut into chunks whose partial results are merged in
+ * ascending chunk order.
+ * Limits: D in {64, 128}; Hq % Hkv == 0; (Hq/Hkv) * Tq <= 16; Tmax % 64 == 0.
+ * workspace  : device, >= heal_attention_workspace_bytes(B, Hq, Tq, Tmax) bytes
+ * qk_int_out : nullable test hook, int64 [B, Hq, Tq, Tmax]; when given, the exact
+ *              S_int of every visible (query, token) pair is written there.          */
+heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale,
+                                   const int16_t* k_cache, const float* k_scale,
+                                   const int16_t* v_cache, const float* v_scale,
+                                   int B, int Hq, int Hkv, int D, int Tq,
+                                   const int32_t* kv_len, int Tmax,
+                                   float softmax_scale, int causal, float* out,
+                                   void* workspace, size_t workspace_bytes,
+                                   int64_t* qk_int_out, heal_stream_t stream);
+
+/* Scratch bytes for heal_attention_int16 (host-only, no CUDA call).                   */
+size_t heal_attention_workspace_bytes(int B, int Hq, int Tq, int Tmax);
+
+/* Synchronises `stream`, returns HEAL_ERR_TIMEOUT if any kernel of this library gave up
+ * on a bounded wait since the last call (the flag is then cleared), HEAL_ERR_CUDA on a
+ * CUDA error, else HEAL_OK.                                                            */
+heal_status_t heal_get_device_status(heal_stream_t stream);
+
+/* Static English description of a status code.                                         */
+const char* heal_status_string(heal_status_t status);
+
+/* Library version, e.g. "heal-b200 0.1.0 sm_100a".                                     */
+const char* heal_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* HEAL_H_ */

@@ -1,0 +1,63 @@
+"""The C ABI: the library loads without a GPU and exports every symbol include/heal.h
+declares; host-side validation rejects bad arguments before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import error_compensated_gemm_b200 as heal
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    src = open(os.path.join(ROOT, "include", "heal.h")).read()
+    return sorted(set(re.findall(r"^\s*(?:heal_status_t|size_t|const char\*)\s+(heal_\w+)\s*\(", src, re.M)))
+
+
+def test_header_and_binding_agree():
+    assert declared_symbols() == sorted(heal.EXPORTED)
+
+
+def test_library_loads_and_exports_every_symbol():
+    L = heal.lib()
+    for name in declared_symbols():
+        assert hasattr(L, name), name
+    assert heal.heal_version().startswith("heal-b200")
+    assert heal.status_string(heal.HEAL_ERR_TIMEOUT) == "a device-side wait ran out of time"
+
+
+def test_workspace_queries_are_host_only():
+    assert heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK) == 64 * 4096 * 4
+    assert heal.heal_gemm_workspace_bytes(4096, 4096, 4096, heal.TILE_128x128) == 0
+    assert heal.heal_attention_workspace_bytes(8, 32, 1, 8192) > 0
+    assert heal.heal_attention_workspace_bytes(0, 32, 1, 8192) == 0
+
+
+def test_invalid_arguments_rejected_before_launch():
+    L = heal.lib()
+    o = heal.gemm_opts()
+    # null pointers / bad sizes: rejected on the host, no CUDA call needed
+    assert L.heal_gemm_compensated(0, 4, 4, None, 4, None, 4, None, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    assert L.heal_gemm_compensated(4, 4, 4, None, 4, None, 4, None, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    fake = ctypes.c_void_p(1 << 20)   # never dereferenced: validation fails first
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 3, fake, 4, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 4, fake, 4, 7, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.reserved[0] = 1
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 4, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    assert L.heal_split(fake, fake, fake, -1, 0, None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    assert L.heal_split(None, None, None, 0, 0, None) == heal.HEAL_OK       # n == 0 is a no-op
+    assert L.heal_kv_quantize_int16(fake, 1, 1, 1, 1, 96, 96, 96, 96, fake, fake, 1, 0, None) == heal.HEAL_ERR_UNSUPPORTED
+    assert L.heal_kv_quantize_int16(fake, 1, 1, 2, 1, 128, 256, 128, 128, fake, fake, 1, 0, None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    assert L.heal_attention_int16(fake, fake, fake, fake, fake, fake, 1, 32, 8, 256, 1, fake, 64, 0.1, 0, fake,
+                                  fake, 1 << 20, None, None) == heal.HEAL_ERR_UNSUPPORTED
+    assert L.heal_attention_int16(fake, fake, fake, fake, fake, fake, 1, 30, 8, 128, 1, fake, 64, 0.1, 0, fake,
+                                  fake, 1 << 20, None, None) == heal.HEAL_ERR_INVALID_ARGUMENT
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    x = torch.zeros(8)
+    with pytest.raises(ValueError):
+        heal.heal_split(x, torch.zeros(8, dtype=torch.int16), torch.zeros(8, dtype=torch.int16))
