@@ -1,10 +1,553 @@
-// attention.cu -- placeholder until the INT16 attention kernel lands.
+// attention.cu -- K5: decode attention on INT16 Q/K/V (gist.science technical summary,
+// section 2.A, "Mechanism": the INT16 tensor is unpacked into two FP16 tensors for the
+// attention contractions).
+//
+// Unpacking used here: q = 256*hi + lo with hi = q >> 8 in [-128, 127] and lo = q & 255
+// in [0, 255]; both are exact FP16 values.  Then, per (query row, token),
+//     S_int = sum_d q_d k_d = 65536*S_hh + 256*S_x + S_ll
+// with S_hh = sum qh*kh, S_x = sum (qh*kl + ql*kh), S_ll = sum ql*kl.  For head_dim <= 128
+// every partial sum of every term is an integer below 2^24 in magnitude, so the FP16 tensor
+// core products accumulate exactly in FP32; the three sums are combined in int64.
+//   logit = fp32( (double(S_int) * (double(s_q) * double(s_k))) * double(softmax_scale) )
+// FP32 online softmax in base 2; P is folded with the per-token V scale and a per-segment
+// power of two, split into an FP16 pair (P_hi, P_lo * 2^-11), and multiplied with the
+// byte-split V (V_hi = 256*(v >> 8), V_lo = v & 255) on FP16 tensor cores.
+//
+// Work decomposition: a persistent grid; CTA c owns the contiguous slice
+// [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token block)
+// units.  Warp 4 streams 64-token K and V tiles with TMA (128-byte swizzle) into a
+// two-stage ring; warps 0-3 each take 16 tokens of a tile with mma.sync m16n8k16 (the
+// decode GEMV shapes are far below a tcgen05 tile; the kernel is HBM-bound).  Every
+// (CTA, kv head) segment leaves one partial (m, l, o) in the workspace; the combine kernel
+// merges them in ascending token order.  The order is fixed, so results are identical
+// from run to run.
+#include <cuda_fp16.h>
+
+#include <cmath>
+
 #include "heal_internal.h"
+#include "heal_ptx.cuh"
+
 namespace heal {
-size_t attention_workspace_bytes(int B, int Hq, int Tq, int Tmax) { return 16; }
-heal_status_t attention_launch(const int16_t*, const float*, const int16_t*, const float*, const int16_t*,
-                               const float*, int, int, int, int, int, const int32_t*, int, float, int, float*,
-                               void*, size_t, int64_t*, cudaStream_t) {
-  return HEAL_ERR_UNSUPPORTED;
+
+namespace {
+
+constexpr int kBlk = 64;          // tokens per pipeline stage
+constexpr int kCompute = 4;       // compute warps, 16 tokens each per stage
+constexpr int kAttnThreads = (kCompute + 1) * 32;
+constexpr int kRows = 8;          // query rows per CTA: (Hq/Hkv) * Tq <= 8
+constexpr int kMaxGrid = 1024;
+constexpr float kLog2e = 1.4426950408889634f;
+
+struct AttnArgs {
+  const int16_t* q;
+  const float* qs;
+  const float* ks;
+  const float* vs;
+  const int32_t* kv_len;
+  float* ws;
+  long long* qk_out;
+  float* out;
+  int B, Hq, Hkv, G, Tq, R, Tmax, nblk, causal;
+  float scale;
+  long long total;  // B*Hkv*nblk
+  int grid;
+  unsigned int* status;
+};
+
+// -------- INT16 byte split into FP16 pairs (bit construction, exact) --------
+// Two int16 values packed in x -> (lo0, lo1) and (hi0, hi1) as half2.
+__device__ __forceinline__ uint32_t lo_pair(uint32_t x) {
+  // 0x6400 | b is the FP16 value 1024 + b for b in [0, 1023]
+  const uint32_t u = (x & 0x00FF00FFu) | 0x64006400u;
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&u), __half2half2(__ushort_as_half(0x6400)));
+  return *reinterpret_cast<const uint32_t*>(&h);
 }
+__device__ __forceinline__ uint32_t hi_pair(uint32_t x) {
+  // (signed high byte + 128) in [0, 255]: XOR with 0x80, then the same construction
+  const uint32_t u = ((x >> 8) & 0x00FF00FFu) ^ 0x64806480u;
+  const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&u), __half2half2(__ushort_as_half(0x6480)));
+  return *reinterpret_cast<const uint32_t*>(&h);   // 0x6480 = 1152 = 1024 + 128
+}
+__device__ __forceinline__ uint32_t hi256_pair(uint32_t x) {   // 256 * hi, exact in FP16
+  const uint32_t h = hi_pair(x);
+  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&h), __half2half2(__ushort_as_half(0x5C00)));
+  return *reinterpret_cast<const uint32_t*>(&r);   // 0x5C00 = 256.0
+}
+
+__device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                         uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+
+__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kCompute * 32) : "memory"); }
+
+__device__ __forceinline__ long long unit_begin(long long total, int grid, int c) {
+  return (total * c) / grid;
+}
+
+// CTA whose slice contains unit u.
+__device__ __forceinline__ int cta_of(long long u, long long total, int grid) {
+  int c = (int)((u * grid) / total);
+  while (c + 1 < grid && unit_begin(total, grid, c + 1) <= u) ++c;
+  while (c > 0 && unit_begin(total, grid, c) > u) --c;
+  return c;
+}
+
+// partial slot of (cta c, pair p) = c + p; layout: [R][D] o, then [R][2] (m, l)
+__device__ __forceinline__ float* slot_ptr(float* ws, int c, int p, int R, int D) {
+  return ws + (size_t)(c + p) * (size_t)R * (size_t)(D + 2);
+}
+
+template <int D>
+__global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+                                                                       const __grid_constant__ CUtensorMap tmV,
+                                                                       const AttnArgs a) {
+  constexpr int kBoxes = D / 64;                    // 64-dim (128-byte) boxes per row
+  constexpr int kTileBytes = kBlk * D * 2;          // one of K / V
+  constexpr int kStageBytes = 2 * kTileBytes;
+  constexpr int kKSteps = D / 16;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = smem;                                            // 2 x kStageBytes
+  float* o_sm = reinterpret_cast<float*>(smem + 2 * kStageBytes);    // [kRows][D]
+  float* ml_sm = o_sm + kRows * D;                                   // [kCompute][kRows][2]
+  uint64_t* full = reinterpret_cast<uint64_t*>(ml_sm + kCompute * kRows * 2);
+  uint64_t* empty = full + 2;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 2);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int c = blockIdx.x;
+  const long long u0 = unit_begin(a.total, a.grid, c), u1 = unit_begin(a.total, a.grid, c + 1);
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < 2; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kCompute);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == kCompute) {
+    // ----------------------------- TMA producer -----------------------------
+    if (lane == 0) {
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      int it = 0;
+      for (long long u = u0; u < u1; ++u) {
+        const int p = (int)(u / a.nblk), blk = (int)(u % a.nblk);
+        const int b = p / a.Hkv;
+        const int t0 = blk * kBlk;
+        if (t0 >= __ldg(a.kv_len + b)) continue;
+        const int s = it & 1;
+        const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.status, 200)) break;
+        uint8_t* st = stages + s * kStageBytes;
+        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        const int row = p * a.Tmax + t0;
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx) {
+          tma_load_2d(st + bx * 8192, &tmK, &full[s], bx * 64, row);
+          tma_load_2d(st + kTileBytes + bx * 8192, &tmV, &full[s], bx * 64, row);
+        }
+        ++it;
+      }
+      // no copy may still be in flight when the CTA exits
+      for (int j = 0; j < 2 && j < it; ++j) {
+        const int jt = it - 1 - j;
+        volatile int dummy = 0;
+        mbar_wait(&full[jt & 1], (uint32_t)(jt >> 1) & 1u, &dummy, a.status, 201);
+      }
+    }
+    return;
+  }
+
+  // ------------------------------- compute warps -------------------------------
+  const int R = a.R;
+  const int rowS = lane >> 2;                 // S layout: query row of c0/c1
+  const int tokq = 2 * (lane & 3);            // S layout: first token (of 8) of c0/c1
+  uint32_t qh[kKSteps][2], ql[kKSteps][2];    // A fragments (rows 0-7; rows 8-15 are zero)
+  float sq = 0.0f;
+  int pos = 0;
+  float m_run = -INFINITY, l_run = 0.0f;      // S layout, row rowS
+  float om[D / 16][4], oc[D / 16][4];         // O^T main / correction accumulators
+  float vscale = 1.0f;                        // 2^E folded into P
+  float inv_vscale = 1.0f;
+  int cur_p = -1, b = 0, hkv = 0, klen = 0;
+  int it = 0;
+  bool ok = true;
+
+  auto finalize = [&](int p) {
+    // row sums (S layout) and row maxima for this warp
+    float l = l_run;
+    l += __shfl_xor_sync(0xffffffffu, l, 1);
+    l += __shfl_xor_sync(0xffffffffu, l, 2);
+    if ((lane & 3) == 0) {
+      ml_sm[(warp * kRows + rowS) * 2 + 0] = m_run;
+      ml_sm[(warp * kRows + rowS) * 2 + 1] = l;
+    }
+    compute_bar();
+    // rows of this lane's O^T fragments: r0 = tokq, r1 = tokq + 1
+    float f[2], M[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int r = tokq + h;
+      float mx = -INFINITY;
+      for (int w = 0; w < kCompute; ++w) mx = fmaxf(mx, ml_sm[(w * kRows + r) * 2]);
+      const float mw = ml_sm[(warp * kRows + r) * 2];
+      M[h] = mx;
+      f[h] = (mw == -INFINITY) ? 0.0f : exp2f(mw - mx);
+    }
+    // O of this warp, scaled to the CTA max, in true units (x 2^-E)
+    float o[D / 16][4];
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float v = __fmaf_rn(oc[dt][e], 1.0f / 2048.0f, om[dt][e]);
+        o[dt][e] = __fmul_rn(__fmul_rn(v, inv_vscale), f[e & 1]);
+      }
+    // sequential, fixed-order merge of the four warps through shared memory
+    for (int w = 0; w < kCompute; ++w) {
+      if (warp == w) {
+#pragma unroll
+        for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
+            const int r = tokq + (e & 1);
+            float* dst = o_sm + r * D + d;
+            const float v = (w == 0) ? o[dt][e] : __fadd_rn(*dst, o[dt][e]);
+            if (w < kCompute - 1) {
+              *dst = v;
+            } else if (r < R) {
+              slot_ptr(a.ws, c, p, R, D)[r * D + d] = v;
+            }
+          }
+      }
+      compute_bar();
+    }
+    if (warp == 0 && lane < R) {
+      const int r = lane;
+      float mx = -INFINITY;
+      for (int w = 0; w < kCompute; ++w) mx = fmaxf(mx, ml_sm[(w * kRows + r) * 2]);
+      float L = 0.0f;
+      for (int w = 0; w < kCompute; ++w) {
+        const float mw = ml_sm[(w * kRows + r) * 2];
+        if (mw != -INFINITY) L = __fadd_rn(L, __fmul_rn(ml_sm[(w * kRows + r) * 2 + 1], exp2f(mw - mx)));
+      }
+      float* sl = slot_ptr(a.ws, c, p, R, D) + R * D;
+      sl[2 * r] = mx;
+      sl[2 * r + 1] = L;
+    }
+    compute_bar();
+    (void)M;
+  };
+
+  for (long long u = u0; u < u1 && ok; ++u) {
+    const int p = (int)(u / a.nblk), blk = (int)(u % a.nblk);
+    if (p != cur_p) {
+      if (cur_p >= 0) finalize(cur_p);
+      cur_p = p;
+      b = p / a.Hkv;
+      hkv = p % a.Hkv;
+      klen = __ldg(a.kv_len + b);
+      // query rows of this kv head: row r = tq * G + g  ->  head hkv*G + g, query tq
+      const int r = rowS;
+      const bool real = r < R;
+      const int tq = real ? r / a.G : 0, g = real ? r % a.G : 0;
+      const long long qrow = ((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq);
+      sq = real ? __ldg(a.qs + qrow) : 0.0f;
+      pos = klen - a.Tq + tq;
+#pragma unroll
+      for (int ks = 0; ks < kKSteps; ++ks) {
+        uint32_t w0 = 0, w1 = 0;
+        if (real) {
+          const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow * D + ks * 16 + tokq);
+          w0 = __ldg(qp);
+          w1 = __ldg(qp + 4);   // dims + 8
+        }
+        qh[ks][0] = hi_pair(w0);
+        qh[ks][1] = hi_pair(w1);
+        ql[ks][0] = lo_pair(w0);
+        ql[ks][1] = lo_pair(w1);
+      }
+      // power of two that brings this head's V scales near 1 (token 0 is always valid)
+      const float s0 = __ldg(a.vs + (size_t)p * a.Tmax);
+      const int E = (s0 > 0.0f) ? (-ilogbf(s0) - 6) : 0;
+      vscale = ldexpf(1.0f, E);
+      inv_vscale = ldexpf(1.0f, -E);
+      m_run = -INFINITY;
+      l_run = 0.0f;
+#pragma unroll
+      for (int dt = 0; dt < D / 16; ++dt)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) om[dt][e] = oc[dt][e] = 0.0f;
+    }
+    const int t0 = blk * kBlk;
+    if (t0 >= klen) continue;
+    const int s = it & 1;
+    const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+    ++it;
+    if (!mbar_wait(&full[s], ph, abort_flag, a.status, 210)) {
+      ok = false;
+      break;
+    }
+    const uint32_t kst = smem_u32(stages + s * kStageBytes);
+    const uint32_t vst = kst + kTileBytes;
+    const int tw = warp * 16;                 // this warp's first token inside the tile
+
+    // ---- exact S = Q K^T on the byte-split operands ----
+    float x[2][2];                            // [n-block][token] logits * log2(e), row rowS
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+      float shh[4] = {0, 0, 0, 0}, sx[4] = {0, 0, 0, 0}, sll[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int j = 0; j < kKSteps / 2; ++j) {
+        const int trow = tw + nb * 8 + (lane & 7);
+        const int ch = 4 * j + (lane >> 3);   // 16-byte chunk of the 256-byte K row
+        const uint32_t addr = kst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4(addr, r0, r1, r2, r3);
+        {
+          const int ks = 2 * j;
+          const uint32_t kh0 = hi_pair(r0), kh1 = hi_pair(r1), kl0 = lo_pair(r0), kl1 = lo_pair(r1);
+          mma16816(shh, qh[ks][0], 0u, qh[ks][1], 0u, kh0, kh1);
+          mma16816(sx, qh[ks][0], 0u, qh[ks][1], 0u, kl0, kl1);
+          mma16816(sx, ql[ks][0], 0u, ql[ks][1], 0u, kh0, kh1);
+          mma16816(sll, ql[ks][0], 0u, ql[ks][1], 0u, kl0, kl1);
+        }
+        {
+          const int ks = 2 * j + 1;
+          const uint32_t kh0 = hi_pair(r2), kh1 = hi_pair(r3), kl0 = lo_pair(r2), kl1 = lo_pair(r3);
+          mma16816(shh, qh[ks][0], 0u, qh[ks][1], 0u, kh0, kh1);
+          mma16816(sx, qh[ks][0], 0u, qh[ks][1], 0u, kl0, kl1);
+          mma16816(sx, ql[ks][0], 0u, ql[ks][1], 0u, kh0, kh1);
+          mma16816(sll, ql[ks][0], 0u, ql[ks][1], 0u, kl0, kl1);
+        }
+      }
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = t0 + tw + nb * 8 + tokq + e;
+        const long long S = ((long long)__float2int_rn(shh[e]) << 16) + ((long long)__float2int_rn(sx[e]) << 8) +
+                            (long long)__float2int_rn(sll[e]);
+        const bool real = rowS < R;
+        const bool vis = real && t < klen && (!a.causal || t <= pos);
+        float xv;
+        if (!real) {
+          xv = 0.0f;                          // padding row: finite, never written
+        } else if (!vis) {
+          xv = -INFINITY;
+        } else {
+          const double coef = (double)sq * (double)__ldg(a.ks + (size_t)p * a.Tmax + t);
+          const float lg = (float)(((double)S * coef) * (double)a.scale);
+          xv = __fmul_rn(lg, kLog2e);
+          if (a.qk_out) {
+            const int tq = rowS / a.G, g = rowS % a.G;
+            a.qk_out[((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq) * a.Tmax + t] = S;
+          }
+        }
+        x[nb][e] = xv;
+      }
+    }
+
+    // ---- online softmax (base 2), row rowS ----
+    float bm = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
+    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
+    const float m_new = fmaxf(m_run, bm);
+    float alpha, pv[2][2];
+    if (m_new == -INFINITY) {
+      alpha = 1.0f;
+      pv[0][0] = pv[0][1] = pv[1][0] = pv[1][1] = 0.0f;
+    } else {
+      alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) pv[nb][e] = (x[nb][e] == -INFINITY) ? 0.0f : exp2f(x[nb][e] - m_new);
+    }
+    l_run = __fadd_rn(__fmul_rn(l_run, alpha), __fadd_rn(__fadd_rn(pv[0][0], pv[0][1]), __fadd_rn(pv[1][0], pv[1][1])));
+    m_run = m_new;
+    // rescale O^T rows tokq, tokq+1: their alphas live in S-layout lanes 4*tokq, 4*(tokq+1)
+    const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * tokq);
+    const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * (tokq + 1));
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+      om[dt][0] = __fmul_rn(om[dt][0], a0);
+      om[dt][1] = __fmul_rn(om[dt][1], a1);
+      om[dt][2] = __fmul_rn(om[dt][2], a0);
+      om[dt][3] = __fmul_rn(om[dt][3], a1);
+      oc[dt][0] = __fmul_rn(oc[dt][0], a0);
+      oc[dt][1] = __fmul_rn(oc[dt][1], a1);
+      oc[dt][2] = __fmul_rn(oc[dt][2], a0);
+      oc[dt][3] = __fmul_rn(oc[dt][3], a1);
+    }
+
+    // ---- P' = P * s_v * 2^E split into FP16 (hi, lo * 2^-11): B fragments of PV ----
+    uint32_t ph_[2], pl_[2];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
+      float pp[2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const int t = t0 + tw + nb * 8 + tokq + e;
+        const float sv = (pv[nb][e] != 0.0f) ? __fmul_rn(__ldg(a.vs + (size_t)p * a.Tmax + t), vscale) : 0.0f;
+        pp[e] = __fmul_rn(pv[nb][e], sv);
+      }
+      const __half2 h = __floats2half2_rn(pp[0], pp[1]);
+      const float2 hf = __half22float2(h);
+      const __half2 l = __floats2half2_rn(__fmul_rn(__fsub_rn(pp[0], hf.x), 2048.0f),
+                                          __fmul_rn(__fsub_rn(pp[1], hf.y), 2048.0f));
+      ph_[nb] = *reinterpret_cast<const uint32_t*>(&h);
+      pl_[nb] = *reinterpret_cast<const uint32_t*>(&l);
+    }
+
+    // ---- O^T += V'^T P'^T ----
+#pragma unroll
+    for (int dt = 0; dt < D / 16; ++dt) {
+      const int mi = lane >> 3;
+      const int trow = tw + ((mi >> 1) << 3) + (lane & 7);
+      const int ch = 2 * dt + (mi & 1);
+      const uint32_t addr = vst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
+      uint32_t r0, r1, r2, r3;
+      ldsm_x4_t(addr, r0, r1, r2, r3);
+      const uint32_t h0 = hi256_pair(r0), h1 = hi256_pair(r1), h2 = hi256_pair(r2), h3 = hi256_pair(r3);
+      const uint32_t l0 = lo_pair(r0), l1 = lo_pair(r1), l2 = lo_pair(r2), l3 = lo_pair(r3);
+      mma16816(om[dt], h0, h1, h2, h3, ph_[0], ph_[1]);
+      mma16816(om[dt], l0, l1, l2, l3, ph_[0], ph_[1]);
+      mma16816(oc[dt], h0, h1, h2, h3, pl_[0], pl_[1]);
+      mma16816(oc[dt], l0, l1, l2, l3, pl_[0], pl_[1]);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+  }
+  if (!ok) return;   // a wait gave up: the status word is set; leave without a partial
+  if (cur_p >= 0) finalize(cur_p);
+}
+
+// out[b, hq, tq, :] = sum_c o_c 2^(m_c - M) / sum_c l_c 2^(m_c - M), c ascending.
+template <int D>
+__global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) {
+  const int pr = blockIdx.x;            // (pair, row)
+  const int p = pr / a.R, r = pr % a.R;
+  const int d = threadIdx.x;
+  const long long ufirst = (long long)p * a.nblk, ulast = ufirst + a.nblk - 1;
+  const int c0 = cta_of(ufirst, a.total, a.grid), c1 = cta_of(ulast, a.total, a.grid);
+  float M = -INFINITY;
+  for (int c = c0; c <= c1; ++c) M = fmaxf(M, slot_ptr(a.ws, c, p, a.R, D)[a.R * D + 2 * r]);
+  float L = 0.0f, O = 0.0f;
+  for (int c = c0; c <= c1; ++c) {
+    const float* sl = slot_ptr(a.ws, c, p, a.R, D);
+    const float m = sl[a.R * D + 2 * r];
+    if (m == -INFINITY) continue;
+    const float f = exp2f(m - M);
+    L = __fadd_rn(L, __fmul_rn(sl[a.R * D + 2 * r + 1], f));
+    O = __fadd_rn(O, __fmul_rn(sl[r * D + d], f));
+  }
+  const int b = p / a.Hkv, hkv = p % a.Hkv;
+  const int tq = r / a.G, g = r % a.G;
+  a.out[(((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq) * D) + d] = __fdiv_rn(O, L);
+}
+
+template <int D>
+constexpr int attn_smem_bytes() {
+  return 2 * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + 64 + 1024;
+}
+
+}  // namespace
+
+size_t attention_workspace_bytes(int B, int Hq, int Tq, int Tmax) {
+  (void)Tmax;
+  // slots <= grid + B*Hkv; slot = R*(D+2) floats with R*Hkv = Hq*Tq, R <= 8, D <= 128
+  return ((size_t)kMaxGrid * kRows + (size_t)B * Hq * Tq) * 130u * sizeof(float);
+}
+
+heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t* k, const float* ks,
+                               const int16_t* v, const float* vs, int B, int Hq, int Hkv, int D, int Tq,
+                               const int32_t* kv_len, int Tmax, float scale, int causal, float* out, void* ws,
+                               size_t ws_bytes, int64_t* qk_out, cudaStream_t stream) {
+  const int G = Hq / Hkv;
+  const int R = G * Tq;
+  if (R > kRows) return HEAL_ERR_UNSUPPORTED;
+  const long long rows_total = (long long)B * Hkv * Tmax;
+  if (rows_total >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
+  const int sms = device_sm_count();
+  if (sms <= 0) return HEAL_ERR_CUDA;
+  AttnArgs a{};
+  a.q = q;
+  a.qs = qs;
+  a.ks = ks;
+  a.vs = vs;
+  a.kv_len = kv_len;
+  a.ws = static_cast<float*>(ws);
+  a.qk_out = reinterpret_cast<long long*>(qk_out);
+  a.out = out;
+  a.B = B;
+  a.Hq = Hq;
+  a.Hkv = Hkv;
+  a.G = G;
+  a.Tq = Tq;
+  a.R = R;
+  a.Tmax = Tmax;
+  a.nblk = Tmax / kBlk;
+  a.causal = causal;
+  a.scale = scale;
+  a.total = (long long)B * Hkv * a.nblk;
+  long long grid = (long long)sms * 3;
+  if (grid > kMaxGrid) grid = kMaxGrid;
+  if (grid > a.total) grid = a.total;
+  a.grid = (int)grid;
+  a.status = device_status_ptr();
+  if ((size_t)(a.grid + (long long)B * Hkv) * (size_t)R * (size_t)(D + 2) * sizeof(float) > ws_bytes)
+    return HEAL_ERR_INVALID_ARGUMENT;
+
+  CUtensorMap tk{}, tv{};
+  const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows_total};
+  const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
+  const cuuint32_t box[2] = {64, kBlk};
+  const cuuint32_t es[2] = {1, 1};
+  if (!encode_tensor_map(&tk, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<int16_t*>(k), dims, strides, box, es,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return HEAL_ERR_CUDA;
+  if (!encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<int16_t*>(v), dims, strides, box, es,
+                         CU_TENSOR_MAP_SWIZZLE_128B))
+    return HEAL_ERR_CUDA;
+  cudaError_t e;
+  if (D == 128) {
+    auto kern = heal_attn_decode_kernel<128>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<128>());
+    if (e == cudaSuccess) {
+      kern<<<a.grid, kAttnThreads, attn_smem_bytes<128>(), stream>>>(tk, tv, a);
+      heal_attn_combine_kernel<128><<<B * Hkv * R, 128, 0, stream>>>(a);
+    }
+  } else {
+    auto kern = heal_attn_decode_kernel<64>;
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<64>());
+    if (e == cudaSuccess) {
+      kern<<<a.grid, kAttnThreads, attn_smem_bytes<64>(), stream>>>(tk, tv, a);
+      heal_attn_combine_kernel<64><<<B * Hkv * R, 64, 0, stream>>>(a);
+    }
+  }
+  if (e != cudaSuccess) return HEAL_ERR_CUDA;
+  return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+}
+
 }  // namespace heal
