@@ -1,0 +1,415 @@
+#!/usr/bin/env python3
+"""Benchmark of the HEAL hot path on B200 (one JSON line on stdout, rank 0).
+
+One step = one pass of every hot-path kernel over one batch of seeded synthetic input:
+  * compensated GEMM, prefill linear: X[4096x4096] (1% outlier columns x20) . W[4096x14336],
+    both FP32, split to FP16 hi/lo inside the kernel                      (headline)
+  * compensated GEMM, decode: X[M x 4096] . W[4096x4096] for M = 1, 8, 64
+  * INT16 KV writer: Q [8,1,32,128], K and V [8,8192,8,128] bf16 -> INT16 caches
+  * INT16 decode attention over the 8192-token caches, 32 query / 8 KV heads
+Every kernel is timed with CUDA events on the launching stream; `value` is the prefill
+GEMM's effective TFLOP/s (2MNK / time).  All inputs are larger than L2 or are separate
+buffers with more than 1 GB of other traffic between their reuses, so each kernel reads
+cold from HBM.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (torchrun): every rank runs the same step on its own seeded shard, no
+collective on the data path ("weak" scaling); timings are the max over ranks.
+"""
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compensated-GEMM effective TFLOP/s (% of 16-bit TC peak); INT16-KV attn GB/s"
+PREFILL = (4096, 4096, 14336)
+DECODE_M = (1, 8, 64)
+KV = dict(B=8, T=8192, Hkv=8, Hq=32, D=128)
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# --------------------------------------------------------------------------- clocks
+THROTTLE = {"0x0000000000000001": "gpu_idle", "0x0000000000000002": "applications_clocks_setting",
+            "0x0000000000000004": "sw_power_cap", "0x0000000000000008": "hw_slowdown",
+            "0x0000000000000010": "sync_boost", "0x0000000000000020": "sw_thermal_slowdown",
+            "0x0000000000000040": "hw_thermal_slowdown", "0x0000000000000080": "hw_power_brake_slowdown",
+            "0x0000000000000100": "display_clock_setting"}
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), "--query-gpu=clocks.sm,clocks.max.sm,power.draw,"
+                 "clocks_event_reasons.active", "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 4:
+                continue
+            try:
+                s, m = float(parts[0]), float(parts[1])
+            except ValueError:
+                continue
+            mx = m
+            try:
+                bits = int(parts[3], 16)
+            except ValueError:
+                bits = 0
+            if bits & 0x1:
+                continue  # gpu_idle: not a sample under load
+            sm.append(s)
+            for k, name in THROTTLE.items():
+                if bits & int(k, 16) and name != "gpu_idle":
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# --------------------------------------------------------------------------- workload
+class Workload:
+    """Device-resident inputs and outputs of one rank's step."""
+
+    def __init__(self, torch, heal, synthetic, dev, seed_offset=0):
+        self.torch, self.heal = torch, heal
+        M, K, N = PREFILL
+        so = seed_offset
+        X, W = synthetic.gemm_prefill(M=M, K=K, N=N, seed_x=0 + so, seed_w=1 + so)
+        self.X, self.W = X.to(dev), W.to(dev)
+        self.C = torch.empty(M, N, device=dev)
+        self.dec = []
+        for i, m in enumerate(DECODE_M):
+            Xd, Wd = synthetic.gemm_decode(m, seed_x=0 + so, seed_w=1 + so + 10 * (i + 1))
+            ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(m, 4096, 4096) // 4), device=dev)
+            self.dec.append((m, Xd.to(dev), Wd.to(dev), torch.empty(m, 4096, device=dev), ws))
+        B, T, Hkv, Hq, D = KV["B"], KV["T"], KV["Hkv"], KV["Hq"], KV["D"]
+        Qb, Kb, Vb = synthetic.kv_decode(B=B, T=T, Hkv=Hkv, Hq=Hq, D=D, seeds=(2 + so, 3 + so, 4 + so))
+        self.Qb, self.Kb, self.Vb = Qb.to(dev), Kb.to(dev), Vb.to(dev)
+        i16, f32 = torch.int16, torch.float32
+        self.qc = torch.empty(B, Hq, 1, D, dtype=i16, device=dev)
+        self.qs = torch.empty(B, Hq, 1, dtype=f32, device=dev)
+        self.kc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
+        self.ks = torch.empty(B, Hkv, T, dtype=f32, device=dev)
+        self.vc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
+        self.vs = torch.empty(B, Hkv, T, dtype=f32, device=dev)
+        self.kv_len = torch.full((B,), T, dtype=torch.int32, device=dev)
+        self.out = torch.empty(B, Hq, 1, D, device=dev)
+        self.aws = torch.empty(heal.heal_attention_workspace_bytes(B, Hq, 1, T) // 4, device=dev)
+
+    # algorithmic bytes / flops per launch (what the method must touch, once)
+    @staticmethod
+    def units():
+        M, K, N = PREFILL
+        B, T, Hkv, Hq, D = KV["B"], KV["T"], KV["Hkv"], KV["Hq"], KV["D"]
+        kv_elems = B * T * Hkv * D
+        return {
+            "prefill_flop_eff": 2.0 * M * N * K,
+            "prefill_flop_mma": 3 * 2.0 * M * N * K,
+            "decode_bytes": {m: 4.0 * (K * N + m * K + m * N) for m in DECODE_M},
+            "kv_writer_bytes": 2 * (2 * kv_elems + 2 * kv_elems + 4 * B * Hkv * T) + (2 + 2) * B * Hq * D + 4 * B * Hq,
+            "attn_bytes": 2 * (2 * kv_elems + 4 * B * Hkv * T) + 2 * B * Hq * D + 4 * B * Hq + 4 * B * Hq * D,
+        }
+
+    def run(self, ev=None):
+        """One step.  ev: dict name -> (start, end) CUDA events, recorded around each part."""
+        h = self.heal
+
+        def rec(name, i):
+            if ev is not None:
+                ev[name][i].record()
+
+        rec("prefill", 0)
+        h.heal_gemm_compensated(self.X, self.W, self.C)
+        rec("prefill", 1)
+        for (m, Xd, Wd, Cd, ws) in self.dec:
+            rec(f"decode{m}", 0)
+            h.heal_gemm_compensated(Xd, Wd, Cd, workspace=ws)
+            rec(f"decode{m}", 1)
+        rec("kv_writer", 0)
+        h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs)
+        h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks)
+        h.heal_kv_quantize_int16(self.Vb, self.vc, self.vs)
+        rec("kv_writer", 1)
+        rec("attention", 0)
+        h.heal_attention_int16(self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len,
+                               KV["D"] ** -0.5, self.out, self.aws)
+        rec("attention", 1)
+
+    LAUNCHES_PER_STEP = 1 + 2 * len(DECODE_M) + 3 + 2
+
+
+def cpu_baseline_oracle(rows=4096):
+    """The oracle's compensated GEMM (split + three FP64 products) on the prefill workload,
+    restricted to `rows` rows of X; returns (TFLOP/s effective, seconds, threads)."""
+    import numpy as np
+    import synthetic
+    from oracle import gemm as G
+    M, K, N = PREFILL
+    X, W = synthetic.gemm_prefill(M=M, K=K, N=N)
+    Xs = X.numpy()[:rows]
+    Wn = W.numpy()
+    t0 = time.perf_counter()
+    G.gemm_emulated(Xs, Wn)
+    dt = time.perf_counter() - t0
+    threads = os.cpu_count()
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        threads = max((i.get("num_threads", 0) for i in info), default=threads) or threads
+    except Exception:
+        pass
+    return 2.0 * rows * N * K / dt / 1e12, dt, threads
+
+
+def dist_setup():
+    import torch
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if ws > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    return ws, rank, local
+
+
+def reference_arm(args):
+    ws, rank, _ = int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0
+    if rank != 0:
+        return 0
+    import numpy as np
+    import synthetic
+    from oracle import gemm as G
+    M, K, N = PREFILL
+    rows = 256
+    X, W = synthetic.gemm_prefill(M=M, K=K, N=N)
+    Xs, Wn = X.numpy()[:rows], W.numpy()
+    for _ in range(args.warmup):
+        G.gemm_emulated(Xs, Wn)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        G.gemm_emulated(Xs, Wn)
+    dt = time.perf_counter() - t0
+    val = 2.0 * rows * N * K * args.steps / dt / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": val, "unit": "TFLOP/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * dt / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"prefill linear X[{M}x{K}] . W[{K}x{N}] FP32, oracle on a {rows}-row sample of X",
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": val, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                         "sample": f"{rows} of {M} rows of X per step (FP64 split + three FP64 products)"},
+        "e2e": {"value": val, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.impl == "reference":
+        return reference_arm(args)
+
+    import torch
+    import error_compensated_gemm_b200 as heal
+    import synthetic
+    ws, rank, local = dist_setup()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    heal.lib()
+    peaks, peak_src = load_peaks()
+    wl = Workload(torch, heal, synthetic, dev, seed_offset=1000 * rank)
+    stream = torch.cuda.current_stream()
+    for _ in range(max(3, args.warmup)):
+        wl.run()
+    torch.cuda.synchronize()
+    st = heal.heal_get_device_status()
+    if st != heal.HEAL_OK:
+        raise SystemExit(f"device status after warm-up: {heal.status_string(st)}")
+
+    names = ["prefill"] + [f"decode{m}" for m in DECODE_M] + ["kv_writer", "attention"]
+    evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
+           for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    smi_index = local
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    if vis:
+        try:
+            smi_index = int(vis.split(",")[local])
+        except (ValueError, IndexError):
+            smi_index = local
+    with ClockSampler(smi_index) as clk:
+        t_start.record(stream)
+        for i in range(args.steps):
+            wl.run(evs[i])
+        t_end.record(stream)
+        torch.cuda.synchronize()
+    if ws > 1:
+        torch.distributed.barrier()
+    st = heal.heal_get_device_status()
+    if st != heal.HEAL_OK:
+        raise SystemExit(f"device status after timing: {heal.status_string(st)}")
+    total_ms = t_start.elapsed_time(t_end)
+    part_ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) for n in names}
+    if ws > 1:
+        import torch.distributed as dist
+        t = torch.tensor([total_ms] + [part_ms[n] for n in names], device=dev, dtype=torch.float64)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms = float(t[0])
+        part_ms = {n: float(t[1 + i]) for i, n in enumerate(names)}
+
+    u = Workload.units()
+    K = args.steps
+    prefill_s = part_ms["prefill"] / 1e3 / K          # per launch
+    value = ws * u["prefill_flop_eff"] / prefill_s / 1e12
+    mma_tflops = u["prefill_flop_mma"] / prefill_s / 1e12
+    peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
+    peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
+    attn_gbs = u["attn_bytes"] / (part_ms["attention"] / 1e3 / K) / 1e9
+    kvw_gbs = u["kv_writer_bytes"] / (part_ms["kv_writer"] / 1e3 / K) / 1e9
+    dec = {f"M{m}": {"gbs": u["decode_bytes"][m] / (part_ms[f"decode{m}"] / 1e3 / K) / 1e9,
+                     "us": 1e3 * part_ms[f"decode{m}"] / K} for m in DECODE_M}
+    for m in DECODE_M:
+        dec[f"M{m}"]["frac_hbm"] = dec[f"M{m}"]["gbs"] / hbm
+
+    # end to end through the public API: pinned host inputs -> device -> GEMM -> host result
+    M_, K_, N_ = PREFILL
+    e2e = None
+    try:
+        hX = wl.X.cpu().pin_memory()
+        hW = wl.W.cpu().pin_memory()
+        hC = torch.empty(M_, N_, pin_memory=True)
+        dX, dW, dC = torch.empty_like(wl.X), torch.empty_like(wl.W), torch.empty_like(wl.C)
+        reps = max(2, min(args.steps, 5))
+        for _ in range(2):
+            dX.copy_(hX, non_blocking=True); dW.copy_(hW, non_blocking=True)
+            heal.heal_gemm_compensated(dX, dW, dC)
+            hC.copy_(dC, non_blocking=True)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            dX.copy_(hX, non_blocking=True); dW.copy_(hW, non_blocking=True)
+            heal.heal_gemm_compensated(dX, dW, dC)
+            hC.copy_(dC, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_s = e0.elapsed_time(e1) / 1e3 / reps
+        if ws > 1:
+            import torch.distributed as dist
+            t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            e2e_s = float(t[0])
+        e2e = {"value": ws * u["prefill_flop_eff"] / e2e_s / 1e12, "unit": "TFLOP/s",
+               "h2d_bytes_per_step": int(4 * (M_ * K_ + K_ * N_)), "d2h_bytes_per_step": int(4 * M_ * N_)}
+        del dX, dW, dC
+    except Exception as exc:  # report, do not hide
+        e2e = {"error": repr(exc)}
+
+    cpu = None
+    if rank == 0 and ws == 1 and not args.no_cpu_baseline:
+        tf, secs, thr = cpu_baseline_oracle()
+        cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
+               "sample": f"full prefill workload (4096 rows), one run of FP64 split + three FP64 products, {secs:.1f} s"}
+
+    traffic = None
+    prof = os.path.join(ROOT, "profiles", "traffic.json")
+    if os.path.exists(prof):
+        try:
+            traffic = json.load(open(prof)).get("heal_gemm_prefill_bytes_per_launch")
+        except Exception:
+            traffic = None
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": ws, "steps": K, "warmup": args.warmup,
+            "ms_per_step": total_ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f16x2-from-f32 (FP32 in/out, FP16 hi/lo tensor-core products, FP32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": "prefill linear X[4096x4096] (1% columns x20) . W[4096x14336], FP32, "
+                                   "in-kernel FP16 hi/lo split; step also runs decode GEMMs M=1/8/64 "
+                                   "(K=N=4096), the INT16 KV writer and INT16 decode attention "
+                                   "(B=8, 32q/8kv heads, D=128, context 8192)",
+                       "parallelism": f"independent shards x{ws}" if ws > 1 else "single GPU",
+                       "l2": "cold: inputs larger than L2 or separate buffers with >1 GB of other traffic "
+                             "between reuses"},
+            "pct_of_16bit_peak": 100.0 * mma_tflops / peak_sus,
+            "roofline": {"bound": "tensor", "achieved": mma_tflops, "peak": peak_sus, "unit": "TFLOP/s",
+                         "frac": mma_tflops / peak_sus, "traffic": traffic,
+                         "kernel": "heal_gemm_kernel (prefill)", "peak_source": f"bf16_tflops_sustained, {peak_src}",
+                         "frac_of_burst_peak": mma_tflops / peak_burst},
+            "attn_gbs": attn_gbs, "attn_frac_hbm": attn_gbs / hbm,
+            "secondary": {"kv_writer_gbs": kvw_gbs, "kv_writer_frac_hbm": kvw_gbs / hbm, "decode_gemm": dec,
+                          "ms_per_step_parts": {n: part_ms[n] / K for n in names},
+                          "hbm_peak_gbs": hbm, "peak_source": peak_src},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": Workload.LAUNCHES_PER_STEP * K,
+            "clocks": clk.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -464,7 +464,8 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
   }
   const int b = p / a.Hkv, hkv = p % a.Hkv;
   const int tq = r / a.G, g = r % a.G;
-  a.out[(((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq) * D) + d] = __fdiv_rn(O, L);
+  // a query with no visible token (causal, kv_len < Tq) gets zeros
+  a.out[(((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq) * D) + d] = L > 0.0f ? __fdiv_rn(O, L) : 0.0f;
 }
 
 template <int D>
@@ -511,7 +512,15 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   a.causal = causal;
   a.scale = scale;
   a.total = (long long)B * Hkv * a.nblk;
-  long long grid = (long long)sms * 3;
+  int per_sm = 0;
+  if (D == 128)
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<128>, kAttnThreads,
+                                                  attn_smem_bytes<128>());
+  else
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<64>, kAttnThreads,
+                                                  attn_smem_bytes<64>());
+  if (per_sm < 1) per_sm = 1;
+  long long grid = (long long)sms * per_sm;
   if (grid > kMaxGrid) grid = kMaxGrid;
   if (grid > a.total) grid = a.total;
   a.grid = (int)grid;
@@ -519,6 +528,11 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   if ((size_t)(a.grid + (long long)B * Hkv) * (size_t)R * (size_t)(D + 2) * sizeof(float) > ws_bytes)
     return HEAL_ERR_INVALID_ARGUMENT;
 
+  if (cudaFuncSetAttribute(heal_attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           attn_smem_bytes<128>()) != cudaSuccess ||
+      cudaFuncSetAttribute(heal_attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           attn_smem_bytes<64>()) != cudaSuccess)
+    return HEAL_ERR_CUDA;
   CUtensorMap tk{}, tv{};
   const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows_total};
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};
