@@ -47,100 +47,98 @@ def load_peaks():
 
 
 # --------------------------------------------------------------------------- clocks
-THROTTLE = {"0x0000000000000001": "gpu_idle", "0x0000000000000002": "applications_clocks_setting",
-            "0x0000000000000004": "sw_power_cap", "0x0000000000000008": "hw_slowdown",
-            "0x0000000000000010": "sync_boost", "0x0000000000000020": "sw_thermal_slowdown",
-            "0x0000000000000040": "hw_thermal_slowdown", "0x0000000000000080": "hw_power_brake_slowdown",
-            "0x0000000000000100": "display_clock_setting"}
-
-
 class ClockSampler:
-    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+    """Samples the SM clock and the active clock-event (throttle) reasons every ~10 ms
+    through NVML while the timed region runs (read-only queries)."""
+
+    REASONS = {0x1: "gpu_idle", 0x2: "applications_clocks_setting", 0x4: "sw_power_cap", 0x8: "hw_slowdown",
+               0x10: "sync_boost", 0x20: "sw_thermal_slowdown", 0x40: "hw_thermal_slowdown",
+               0x80: "hw_power_brake_slowdown", 0x100: "display_clock_setting"}
 
     def __init__(self, index):
         self.index = index
-        self.proc = None
-        self.lines = []
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self.error = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.index), "--query-gpu=clocks.sm,clocks.max.sm,power.draw,"
-                 "clocks_event_reasons.active", "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.t = threading.Thread(target=self._read, daemon=True)
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(self.index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.t = threading.Thread(target=self._poll, daemon=True)
             self.t.start()
-        except Exception:
-            self.proc = None
+        except Exception as exc:
+            self.error = repr(exc)
+            self.nv = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _poll(self):
+        nv = self.nv
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            getattr(nv, "nvmlDeviceGetCurrentClocksThrottleReasons")
+        while not self._stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM), int(get_reasons(self.h))))
+            except Exception as exc:
+                self.error = repr(exc)
+                return
+            time.sleep(0.01)
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
+        self._stop.set()
+        if self.nv is not None:
             self.t.join(timeout=2)
 
     def summary(self):
-        sm, mx, reasons = [], None, set()
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 4:
-                continue
-            try:
-                s, m = float(parts[0]), float(parts[1])
-            except ValueError:
-                continue
-            mx = m
-            try:
-                bits = int(parts[3], 16)
-            except ValueError:
-                bits = 0
-            if bits & 0x1:
-                continue  # gpu_idle: not a sample under load
-            sm.append(s)
-            for k, name in THROTTLE.items():
-                if bits & int(k, 16) and name != "gpu_idle":
-                    reasons.add(name)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(sm)}
+        loaded = [(mhz, bits) for mhz, bits in self.samples if not bits & 0x1]
+        reasons = sorted({name for _, bits in loaded for b, name in self.REASONS.items() if bits & b})
+        out = {"sm_mhz": statistics.median([m for m, _ in loaded]) if loaded else None,
+               "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(loaded),
+               "source": "nvml"}
+        if self.error:
+            out["error"] = self.error
+        return out
 
 
 # --------------------------------------------------------------------------- workload
 class Workload:
     """Device-resident inputs and outputs of one rank's step."""
 
-    def __init__(self, torch, heal, synthetic, dev, seed_offset=0):
+    def __init__(self, torch, heal, synthetic, dev, seed_offset=0, only=None):
+        """only: None for the whole step, or one part (a profiling case allocates only its buffers)."""
         self.torch, self.heal = torch, heal
+        self.only = only
         M, K, N = PREFILL
         so = seed_offset
-        X, W = synthetic.gemm_prefill(M=M, K=K, N=N, seed_x=0 + so, seed_w=1 + so)
-        self.X, self.W = X.to(dev), W.to(dev)
-        self.C = torch.empty(M, N, device=dev)
+        need = lambda part: only is None or only == part or (part == "kv_writer" and only == "attention")
+        if need("prefill"):
+            X, W = synthetic.gemm_prefill(M=M, K=K, N=N, seed_x=0 + so, seed_w=1 + so)
+            self.X, self.W = X.to(dev), W.to(dev)
+            self.C = torch.empty(M, N, device=dev)
         self.dec = []
-        for i, m in enumerate(DECODE_M):
-            Xd, Wd = synthetic.gemm_decode(m, seed_x=0 + so, seed_w=1 + so + 10 * (i + 1))
-            ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(m, 4096, 4096) // 4), device=dev)
-            self.dec.append((m, Xd.to(dev), Wd.to(dev), torch.empty(m, 4096, device=dev), ws))
-        B, T, Hkv, Hq, D = KV["B"], KV["T"], KV["Hkv"], KV["Hq"], KV["D"]
-        Qb, Kb, Vb = synthetic.kv_decode(B=B, T=T, Hkv=Hkv, Hq=Hq, D=D, seeds=(2 + so, 3 + so, 4 + so))
-        self.Qb, self.Kb, self.Vb = Qb.to(dev), Kb.to(dev), Vb.to(dev)
-        i16, f32 = torch.int16, torch.float32
-        self.qc = torch.empty(B, Hq, 1, D, dtype=i16, device=dev)
-        self.qs = torch.empty(B, Hq, 1, dtype=f32, device=dev)
-        self.kc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
-        self.ks = torch.empty(B, Hkv, T, dtype=f32, device=dev)
-        self.vc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
-        self.vs = torch.empty(B, Hkv, T, dtype=f32, device=dev)
-        self.kv_len = torch.full((B,), T, dtype=torch.int32, device=dev)
-        self.out = torch.empty(B, Hq, 1, D, device=dev)
-        self.aws = torch.empty(heal.heal_attention_workspace_bytes(B, Hq, 1, T) // 4, device=dev)
+        if need("decode"):
+            for i, m in enumerate(DECODE_M):
+                Xd, Wd = synthetic.gemm_decode(m, seed_x=0 + so, seed_w=1 + so + 10 * (i + 1))
+                ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(m, 4096, 4096) // 4), device=dev)
+                self.dec.append((m, Xd.to(dev), Wd.to(dev), torch.empty(m, 4096, device=dev), ws))
+        if need("kv_writer"):
+            B, T, Hkv, Hq, D = KV["B"], KV["T"], KV["Hkv"], KV["Hq"], KV["D"]
+            Qb, Kb, Vb = synthetic.kv_decode(B=B, T=T, Hkv=Hkv, Hq=Hq, D=D, seeds=(2 + so, 3 + so, 4 + so))
+            self.Qb, self.Kb, self.Vb = Qb.to(dev), Kb.to(dev), Vb.to(dev)
+            i16, f32 = torch.int16, torch.float32
+            self.qc = torch.empty(B, Hq, 1, D, dtype=i16, device=dev)
+            self.qs = torch.empty(B, Hq, 1, dtype=f32, device=dev)
+            self.kc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
+            self.ks = torch.empty(B, Hkv, T, dtype=f32, device=dev)
+            self.vc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
+            self.vs = torch.empty(B, Hkv, T, dtype=f32, device=dev)
+            self.kv_len = torch.full((B,), T, dtype=torch.int32, device=dev)
+            self.out = torch.empty(B, Hq, 1, D, device=dev)
+            self.aws = torch.empty(heal.heal_attention_workspace_bytes(B, Hq, 1, T) // 4, device=dev)
 
     # algorithmic bytes / flops per launch (what the method must touch, once)
     @staticmethod
@@ -164,22 +162,27 @@ class Workload:
             if ev is not None:
                 ev[name][i].record()
 
-        rec("prefill", 0)
-        h.heal_gemm_compensated(self.X, self.W, self.C)
-        rec("prefill", 1)
-        for (m, Xd, Wd, Cd, ws) in self.dec:
-            rec(f"decode{m}", 0)
-            h.heal_gemm_compensated(Xd, Wd, Cd, workspace=ws)
-            rec(f"decode{m}", 1)
-        rec("kv_writer", 0)
-        h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs)
-        h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks)
-        h.heal_kv_quantize_int16(self.Vb, self.vc, self.vs)
-        rec("kv_writer", 1)
-        rec("attention", 0)
-        h.heal_attention_int16(self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len,
-                               KV["D"] ** -0.5, self.out, self.aws)
-        rec("attention", 1)
+        only = self.only
+        if only in (None, "prefill"):
+            rec("prefill", 0)
+            h.heal_gemm_compensated(self.X, self.W, self.C)
+            rec("prefill", 1)
+        if only in (None, "decode"):
+            for (m, Xd, Wd, Cd, ws) in self.dec:
+                rec(f"decode{m}", 0)
+                h.heal_gemm_compensated(Xd, Wd, Cd, workspace=ws)
+                rec(f"decode{m}", 1)
+        if only in (None, "kv_writer", "attention"):
+            rec("kv_writer", 0)
+            h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs)
+            h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks)
+            h.heal_kv_quantize_int16(self.Vb, self.vc, self.vs)
+            rec("kv_writer", 1)
+        if only in (None, "attention"):
+            rec("attention", 0)
+            h.heal_attention_int16(self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len,
+                                   KV["D"] ** -0.5, self.out, self.aws)
+            rec("attention", 1)
 
     LAUNCHES_PER_STEP = 1 + 2 * len(DECODE_M) + 3 + 2
 
@@ -254,11 +257,20 @@ def reference_arm(args):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=10)
-    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--only", choices=["prefill", "decode", "kv_writer", "attention"],
+                    help="profiling case: run only this part of the step")
+    ap.add_argument("--prefill-shape", default=None, help="M,N,K of the prefill GEMM (profiling case)")
+    ap.add_argument("--kv-batch", type=int, default=None, help="batch of the KV workload (profiling case)")
     args = ap.parse_args()
+    if args.prefill_shape:
+        global PREFILL
+        PREFILL = tuple(int(v) for v in args.prefill_shape.split(","))
+    if args.kv_batch:
+        KV["B"] = args.kv_batch
     if args.impl == "reference":
         return reference_arm(args)
 
@@ -270,7 +282,7 @@ def main():
     dev = torch.device("cuda", local)
     heal.lib()
     peaks, peak_src = load_peaks()
-    wl = Workload(torch, heal, synthetic, dev, seed_offset=1000 * rank)
+    wl = Workload(torch, heal, synthetic, dev, seed_offset=1000 * rank, only=args.only)
     stream = torch.cuda.current_stream()
     for _ in range(max(3, args.warmup)):
         wl.run()
@@ -280,6 +292,10 @@ def main():
         raise SystemExit(f"device status after warm-up: {heal.status_string(st)}")
 
     names = ["prefill"] + [f"decode{m}" for m in DECODE_M] + ["kv_writer", "attention"]
+    if args.only:
+        keep = {"prefill": ["prefill"], "decode": [f"decode{m}" for m in DECODE_M],
+                "kv_writer": ["kv_writer"], "attention": ["kv_writer", "attention"]}[args.only]
+        names = keep
     evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
            for _ in range(args.steps)]
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -315,6 +331,12 @@ def main():
 
     u = Workload.units()
     K = args.steps
+    if args.only:
+        if rank == 0:
+            print(json.dumps({"profiling_case": args.only, "steps": K,
+                              "ms_per_launch": {n: part_ms[n] / K for n in names},
+                              "prefill_shape": PREFILL, "kv": KV}), flush=True)
+        return 0
     prefill_s = part_ms["prefill"] / 1e3 / K          # per launch
     value = ws * u["prefill_flop_eff"] / prefill_s / 1e12
     mma_tflops = u["prefill_flop_mma"] / prefill_s / 1e12
