@@ -14,7 +14,7 @@ TILE_AUTO, TILE_128x128, TILE_128x256, TILE_SKINNY_SPLITK = -1, 0, 1, 2
 # every symbol the public header declares
 EXPORTED = ("heal_split", "heal_gemm_compensated", "heal_gemm_workspace_bytes", "heal_kv_quantize_int16",
             "heal_attention_int16", "heal_attention_workspace_bytes", "heal_get_device_status",
-            "heal_status_string", "heal_version")
+            "heal_status_string", "heal_version", "heal_attention_int16_noalloc")
 
 
 class HealError(RuntimeError):
@@ -50,6 +50,8 @@ def lib():
         "heal_attention_int16": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _f, _i, _vp, _vp, _sz,
                                   _vp, _vp], _i),
         "heal_attention_workspace_bytes": ([_i, _i, _i, _i], _sz),
+        "heal_attention_int16_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _f, _i, _vp,
+                                          _vp, _vp], _i),
         "heal_get_device_status": ([_vp], _i),
         "heal_status_string": ([_i], ctypes.c_char_p),
         "heal_version": ([], ctypes.c_char_p),
@@ -175,6 +177,23 @@ def heal_attention_int16(q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len,
                                     workspace.numel() * workspace.element_size(), _ptr(qk_int_out),
                                     _stream(stream))
     _check(st, "heal_attention_int16")
+
+
+def heal_attention_int16_noalloc(q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len, softmax_scale, out,
+                                 causal=False, qk_int_out=None, stream=None):
+    """heal_attention_int16 without a workspace: the library's fixed device scratch holds the
+    partial results (for callers that cannot allocate; see include/heal.h)."""
+    _cuda(q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len, out, qk_int_out)
+    for t in (q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len, out):
+        if not t.is_contiguous():
+            raise ValueError("attention tensors must be contiguous")
+    B, Hq, Tq, D = q.shape
+    Hkv, Tmax = k_cache.shape[1], k_cache.shape[2]
+    st = lib().heal_attention_int16_noalloc(_ptr(q), _ptr(q_scale), _ptr(k_cache), _ptr(k_scale), _ptr(v_cache),
+                                            _ptr(v_scale), B, Hq, Hkv, D, Tq, _ptr(kv_len), Tmax,
+                                            float(softmax_scale), 1 if causal else 0, _ptr(out), _ptr(qk_int_out),
+                                            _stream(stream))
+    _check(st, "heal_attention_int16_noalloc")
 
 
 def heal_get_device_status(stream=None):

@@ -159,6 +159,35 @@ heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale,
 /* Scratch bytes for heal_attention_int16 (host-only, no CUDA call).                   */
 size_t heal_attention_workspace_bytes(int B, int Hq, int Tq, int Tmax);
 
+/* Fixed-scratch variant of heal_attention_int16.  The paper has no counterpart to this
+ * entry point; it exists for callers that cannot allocate device memory when they call
+ * attention, and so cannot pass a `workspace`: code that runs while a stream is being
+ * captured into a CUDA graph (allocation is not allowed during capture), serving loops
+ * that forbid allocation after start-up to keep a fixed memory budget, and plugin hosts
+ * that hand an operator only its input and output tensors.
+ * Arguments and results are those of heal_attention_int16 without workspace and
+ * workspace_bytes.  The split-context partial results go instead to one array of
+ * HEAL_ATTN_STATIC_SCRATCH_BYTES bytes in libheal.so's own device memory, which every GPU
+ * that loads the library holds until the process exits.  This call allocates and frees
+ * nothing.
+ *   - The first call on a device looks up that array's device address, with that device
+ *     current.  Make this first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents.  Nothing in it
+ *     needs to start at zero: every partial result a call reads was written earlier in the
+ *     same call.  Calls whose kernels overlap on the GPU (other streams, other host
+ *     threads) race on the array and corrupt each other's results: serialise them.
+ *   - Size limit: B * Hq * Tq <= 7939 (the scratch the workspace variant would need,
+ *     heal_attention_workspace_bytes(B, Hq, Tq, Tmax), must fit the array).  Larger
+ *     problems return HEAL_ERR_UNSUPPORTED and launch nothing.                            */
+#define HEAL_ATTN_STATIC_SCRATCH_BYTES (8u << 20)
+heal_status_t heal_attention_int16_noalloc(const int16_t* q, const float* q_scale,
+                                           const int16_t* k_cache, const float* k_scale,
+                                           const int16_t* v_cache, const float* v_scale,
+                                           int B, int Hq, int Hkv, int D, int Tq,
+                                           const int32_t* kv_len, int Tmax,
+                                           float softmax_scale, int causal, float* out,
+                                           int64_t* qk_int_out, heal_stream_t stream);
+
 /* Synchronises `stream`, returns HEAL_ERR_TIMEOUT if any kernel of this library gave up
  * on a bounded wait since the last call (the flag is then cleared), HEAL_ERR_CUDA on a
  * CUDA error, else HEAL_OK.                                                            */
