@@ -288,8 +288,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
+  constexpr bool kRegSplit = (BN == 128);   // epilogue holds 128 FP32 sums per thread
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
+    if constexpr (kRegSplit) setmaxnreg_dec<96>();
     if (lane == 0) {
       int it = 0;
       for (WorkIter w(args); w.valid(); w.advance(), ++it) {
@@ -314,6 +316,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer ------------------------------
+    if constexpr (kRegSplit) setmaxnreg_dec<96>();
     if (lane == 0) {
       int it = 0;
       for (WorkIter w(args); w.valid(); w.advance(), ++it) {
@@ -355,6 +358,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else if (warp < kEpiWarp0) {
     // ------------------------------ split warps ------------------------------
+    if constexpr (kRegSplit) setmaxnreg_dec<96>();
     const int sw = warp - kSplitWarp0;
     constexpr int kPairsA = kBM / 8, kPairsB = BN / 8;
     int it = 0;
@@ -382,6 +386,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------ epilogue ------------------------------
+    if constexpr (kRegSplit) setmaxnreg_inc<240>();
     const int quarter = warp & 3;            // TMEM lanes this warp may access
     const int i_local = quarter * 32 + lane; // tile row
     float acc[BN];
@@ -463,6 +468,254 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem_base, C::kTmemCols);
 }
 
+// ---------------------------------------------------------------------------------
+// CTA-pair kernel (cluster of 2, tcgen05 cta_group::2): one 256 x 256 tile of C per pair.
+// Each CTA stages its own 128 rows of A and its own 128 columns of B (64 KB per stage,
+// three stages) and splits them in place, exactly as the single-CTA kernel does; the
+// leader's MMA thread issues M=256, N=256 MMAs that read both CTAs' shared memory, and
+// each CTA's TMEM receives its 128 rows x 256 columns.  Barriers that the peer must reach
+// are addressed through the cluster window (mapa); completions are committed separately
+// to each CTA's barrier.  16 warps: 0 TMA, 1 MMA (leader), 2-7 split, 8-15 epilogue
+// (two warps per TMEM lane quarter, 128 columns each, 168 registers via setmaxnreg).
+// Chunk arithmetic and the ascending FP32 chunk sum are those of heal_gemm_kernel, so C is
+// identical bit for bit.
+// ---------------------------------------------------------------------------------
+constexpr int kPairThreads = 512;
+constexpr int kPairSplitWarps = 6;
+constexpr int kPairEpiWarp0 = 8, kPairEpiWarps = 8;
+constexpr int kPairRows = 128;                      // rows of A and of B per CTA
+constexpr int kPairN = 256;                         // MMA N (= B columns per pair)
+constexpr int kPairStageBytes = 2 * kPairRows * kBK * 4;
+constexpr int kPairStages = 3;
+constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 1024 + 1024;
+
+template <bool B_MN, int FMT, bool B_PRE>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
+    heal_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmB_lo, const GemmArgs args) {
+  constexpr int S = kPairStages;
+  constexpr int kLoShift = FMT == 0 ? 11 : 0;
+  constexpr uint32_t kIdesc = idesc_f16(256, kPairN, FMT, 0, B_MN ? 1 : 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
+  uint8_t* stages = smem;
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * kPairStageBytes);
+  uint64_t* full = bars;                   // TMA -> split (local)
+  uint64_t* split_done = bars + S;         // split warps of both CTAs -> leader's MMA thread
+  uint64_t* empty = bars + 2 * S;          // MMA commit -> TMA (both CTAs)
+  uint64_t* acc_full = bars + 3 * S;       // MMA commit -> epilogue (both CTAs)
+  uint64_t* acc_empty = bars + 3 * S + 2;  // epilogue warps of both CTAs -> leader
+  uint64_t* mma_done = bars + 3 * S + 4;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
+  const int ntiles = args.tiles_m * args.tiles_n, nc = args.num_chunks;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&split_done[s], 2 * kPairSplitWarps);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], 2 * kPairEpiWarps);
+    }
+    mbar_init(mma_done, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0) {
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  if (warp == 0) {
+    // ------------------------------ TMA producer ------------------------------
+    setmaxnreg_dec<88>();
+    if (lane == 0) {
+      tma_prefetch_desc(&tmA);
+      tma_prefetch_desc(&tmB);
+      if (B_PRE) tma_prefetch_desc(&tmB_lo);
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; tile < ntiles && ok; tile += ncl) {
+        int tm, tn;
+        tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
+        for (int ch = 0; ch < nc; ++ch, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          if (!mbar_wait_cluster(&empty[s], ph ^ 1u, abort_flag, args.status, 300)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = stages + s * kPairStageBytes;
+          mbar_arrive_expect_tx(&full[s], kPairStageBytes);
+          load_operand<kPairRows, false, false>(st, &tmA, &tmA, &full[s], tm * 256 + kPairRows * (int)rank,
+                                                ch * kBK);
+          load_operand<kPairRows, B_MN, B_PRE>(st + kPairRows * kBK * 4, &tmB, &tmB_lo, &full[s],
+                                               tn * kPairN + kPairRows * (int)rank, ch * kBK);
+        }
+      }
+      for (int j = 0; j < S && j < it; ++j) {
+        const int jt = it - 1 - j;
+        volatile int dummy = 0;
+        mbar_wait(&full[jt % S], (uint32_t)(jt / S) & 1u, &dummy, args.status, 301);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------ MMA issuer (leader CTA) ------------------------------
+    setmaxnreg_dec<88>();
+    if (rank == 0 && lane == 0) {
+      const uint32_t peer = 1u;
+      int it = 0;
+      bool ok = true;
+      for (int tile = cid; tile < ntiles && ok; tile += ncl) {
+        for (int ch = 0; ch < nc; ++ch, ++it) {
+          const int s = it % S;
+          const uint32_t ph = (uint32_t)(it / S) & 1u;
+          const int b = it & 1;
+          const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+          if (!mbar_wait_cluster(&split_done[s], ph, abort_flag, args.status, 310) ||
+              !mbar_wait_cluster(&acc_empty[b], aph ^ 1u, abort_flag, args.status, 311)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = smem_u32(stages + s * kPairStageBytes);
+          const uint32_t sb = sa + kPairRows * kBK * 4;
+          const uint64_t a_hi = OperandDesc<kPairRows, false>::hi(sa), a_lo = OperandDesc<kPairRows, false>::lo(sa);
+          const uint64_t b_hi = OperandDesc<kPairRows, B_MN>::hi(sb), b_lo = OperandDesc<kPairRows, B_MN>::lo(sb);
+          constexpr uint64_t dA = OperandDesc<kPairRows, false>::kStep, dB = OperandDesc<kPairRows, B_MN>::kStep;
+          const uint32_t d = tmem_base + (uint32_t)(b * kPairN);
+#pragma unroll
+          for (int j = 0; j < kBK / 16; ++j) {
+            mma_f16_pair(d, a_hi + j * dA, b_lo + j * dB, kIdesc, j > 0 ? 1u : 0u);
+            mma_f16_pair(d, a_lo + j * dA, b_hi + j * dB, kIdesc, 1u);
+          }
+          mma_f16_pair_scale_d<kLoShift>(d, a_hi, b_hi, kIdesc);
+#pragma unroll
+          for (int j = 1; j < kBK / 16; ++j) mma_f16_pair(d, a_hi + j * dA, b_hi + j * dB, kIdesc, 1u);
+          const uint32_t e_loc = smem_u32(&empty[s]), f_loc = smem_u32(&acc_full[b]);
+          tc_commit_pair(mapa_shared(e_loc, 0u));
+          tc_commit_pair(mapa_shared(e_loc, peer));
+          tc_commit_pair(mapa_shared(f_loc, 0u));
+          tc_commit_pair(mapa_shared(f_loc, peer));
+        }
+      }
+      tc_commit_pair(mapa_shared(smem_u32(mma_done), 0u));
+      volatile int dummy = 0;
+      mbar_wait(mma_done, 0, &dummy, args.status, 312);
+    }
+  } else if (warp < kPairEpiWarp0) {
+    // ------------------------------ split warps (both CTAs) ------------------------------
+    setmaxnreg_dec<88>();
+    const int sw = warp - 2;
+    constexpr int kPairsA = kPairRows / 8, kPairsB = kPairRows / 8;
+    const uint32_t sd_leader0 = mapa_shared(smem_u32(&split_done[0]), 0u);
+    int it = 0;
+    bool ok = true;
+    for (int tile = cid; tile < ntiles && ok; tile += ncl) {
+      for (int ch = 0; ch < nc; ++ch, ++it) {
+        const int s = it % S;
+        const uint32_t ph = (uint32_t)(it / S) & 1u;
+        if (!mbar_wait(&full[s], ph, abort_flag, args.status, 320)) {
+          ok = false;
+          break;
+        }
+        uint8_t* st = stages + s * kPairStageBytes;
+        const int k0 = ch * kBK;
+        constexpr int kLast = B_PRE ? kPairsA : kPairsA + kPairsB;
+        for (int t = sw; t < kLast; t += kPairSplitWarps) {
+          uint8_t *s0, *s1;
+          int kboff;
+          if (t < kPairsA) {
+            pair_addr<kPairRows, false>(st, t, s0, s1, kboff);
+            split_pair<FMT, false>(s0, s1, lane, args.chan_exp, args.expA_sign, k0 + kboff, args.K);
+          } else {
+            pair_addr<kPairRows, B_MN>(st + kPairRows * kBK * 4, t - kPairsA, s0, s1, kboff);
+            split_pair<FMT, B_MN>(s0, s1, lane, args.chan_exp, args.expB_sign, k0 + kboff, args.K);
+          }
+        }
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(sd_leader0 + (uint32_t)(s * 8));
+      }
+    }
+  } else {
+    // ------------------------------ epilogue (both CTAs) ------------------------------
+    setmaxnreg_inc<168>();
+    const int quarter = warp & 3;
+    const int half = (warp - kPairEpiWarp0) >> 2;
+    const int i_local = quarter * 32 + lane;
+    const uint32_t ae_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0u);
+    float acc[128];
+#pragma unroll
+    for (int t = 0; t < 128; ++t) acc[t] = 0.0f;
+    int it = 0;
+    bool ok = true;
+    for (int tile = cid; tile < ntiles && ok; tile += ncl) {
+      int tm, tn;
+      tile_coords(tile, args.tiles_m, args.tiles_n, tm, tn);
+      const int gi = tm * 256 + kPairRows * (int)rank + i_local;
+      for (int ch = 0; ch < nc; ++ch, ++it) {
+        const int b = it & 1;
+        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        if (!mbar_wait_cluster(&acc_full[b], aph, abort_flag, args.status, 330)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t taddr = tmem_base + ((uint32_t)(quarter * 32) << 16) + (uint32_t)(b * kPairN + half * 128);
+        const bool first = (ch == 0);
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          uint32_t r[16];
+          tmem_ld16(taddr + c * 16, r);
+          tmem_ld_wait();
+#pragma unroll
+          for (int t = 0; t < 16; ++t) {
+            const float dv = __uint_as_float(r[t]);
+            acc[c * 16 + t] = first ? dv : __fadd_rn(acc[c * 16 + t], dv);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_cluster(ae_leader0 + (uint32_t)(b * 8));
+      }
+      if (!ok) break;
+      if (gi < args.Mk) {
+        const int gj0 = tn * kPairN + half * 128;
+        float* orow = args.out + (size_t)gi * args.out_si + gj0;
+        if (((reinterpret_cast<uintptr_t>(orow) & 15) == 0) && (gj0 + 128 <= args.Nk)) {
+#pragma unroll
+          for (int t = 0; t < 128; t += 4)
+            *reinterpret_cast<float4*>(orow + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
+        } else {
+#pragma unroll
+          for (int t = 0; t < 128; ++t)
+            if (gj0 + t < args.Nk) orow[t] = acc[t];
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync_all();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc_pair(tmem_base, 512);
+}
+
 // Ordered sum of chunk values: out(i, j) = ((ws[0] + ws[1]) + ws[2]) + ...
 __global__ void heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk, int Nk, float* out,
                                          long long si, long long sj) {
@@ -520,6 +773,16 @@ cudaError_t launch_fmt(int fmt, const CUtensorMap& a, const CUtensorMap& alo, co
   return launch_variant<BN, A_MN, B_MN, 1, CORR_SWAP, A_PRE, B_PRE>(a, alo, b, blo, args, grid, stream);
 }
 
+template <bool B_MN, int FMT, bool B_PRE>
+cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& blo, const GemmArgs& args,
+                        int grid, cudaStream_t stream) {
+  auto kern = heal_gemm_pair_kernel<B_MN, FMT, B_PRE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
+  if (e != cudaSuccess) return e;
+  kern<<<grid, kPairThreads, kPairSmemBytes, stream>>>(a, b, blo, args);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 size_t gemm_workspace_bytes(int M, int N, int K, int tile_config) {
@@ -534,10 +797,13 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
                           float* Cout, long long ldc, int fmt, const heal_gemm_opts_t& o, cudaStream_t stream) {
   int cfg = o.tile_config;
   if (cfg == HEAL_TILE_AUTO) {
-    cfg = (M <= 64 && o.workspace != nullptr && o.workspace_bytes >= gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK) &&
-           !o.b_presplit)
-              ? HEAL_TILE_SKINNY_SPLITK
-              : HEAL_TILE_128x128;
+    if (M <= 64 && o.workspace != nullptr && o.workspace_bytes >= gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK) &&
+        !o.b_presplit)
+      cfg = HEAL_TILE_SKINNY_SPLITK;
+    else if (M >= 256 && N >= 256)
+      cfg = HEAL_TILE_256x256_PAIR;
+    else
+      cfg = HEAL_TILE_128x128;
   }
   const int sms = device_sm_count();
   if (sms <= 0) return HEAL_ERR_CUDA;
@@ -551,8 +817,47 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
   args.status = device_status_ptr();
   cudaError_t err = cudaSuccess;
 
-  if (cfg == HEAL_TILE_128x128 || cfg == HEAL_TILE_128x256) {
-    if (cfg == HEAL_TILE_128x256) return HEAL_ERR_UNSUPPORTED;   // not built in this version
+  if (cfg == HEAL_TILE_256x256_PAIR) {
+    args.Mk = M;
+    args.Nk = N;
+    args.tiles_m = (M + 255) / 256;
+    args.tiles_n = (N + 255) / 256;
+    args.splitk = 0;
+    args.out = Cout;
+    args.out_si = ldc;
+    args.out_sj = 1;
+    args.expA_sign = -1;
+    args.expB_sign = +1;
+    if (!operand_map(&ta, A, false, false, M, K, lda, kPairRows)) return HEAL_ERR_CUDA;
+    if (!o.b_presplit) {
+      if (!operand_map(&tb, B, b_mn, false, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
+    } else {
+      if (!operand_map(&tb, B, b_mn, true, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
+      if (!operand_map(&tblo, o.b_lo, b_mn, true, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
+    }
+    const long long pairs = (long long)args.tiles_m * args.tiles_n;
+    const int max_pairs = sms / 2;
+    const int grid = 2 * (int)(pairs < max_pairs ? pairs : max_pairs);
+    if (grid < 2) return HEAL_ERR_CUDA;
+    if (!o.b_presplit) {
+      if (fmt == 0)
+        err = b_mn ? launch_pair<true, 0, false>(ta, tb, tblo, args, grid, stream)
+                   : launch_pair<false, 0, false>(ta, tb, tblo, args, grid, stream);
+      else
+        err = b_mn ? launch_pair<true, 1, false>(ta, tb, tblo, args, grid, stream)
+                   : launch_pair<false, 1, false>(ta, tb, tblo, args, grid, stream);
+    } else {
+      if (fmt == 0)
+        err = b_mn ? launch_pair<true, 0, true>(ta, tb, tblo, args, grid, stream)
+                   : launch_pair<false, 0, true>(ta, tb, tblo, args, grid, stream);
+      else
+        err = b_mn ? launch_pair<true, 1, true>(ta, tb, tblo, args, grid, stream)
+                   : launch_pair<false, 1, true>(ta, tb, tblo, args, grid, stream);
+    }
+    return err == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+  }
+
+  if (cfg == HEAL_TILE_128x128) {
     constexpr int BN = 128;
     args.Mk = M;
     args.Nk = N;

@@ -56,7 +56,9 @@ typedef enum { HEAL_SPLIT_FP16_S11 = 0, HEAL_SPLIT_BF16 = 1 } heal_split_fmt_t;
 enum {
   HEAL_TILE_AUTO = -1,
   HEAL_TILE_128x128 = 0,      /* 1 CTA per tile, full K per tile                        */
-  HEAL_TILE_128x256 = 1,      /* 1 CTA per tile, wider N                                */
+  HEAL_TILE_256x256_PAIR = 1, /* a cluster of 2 CTAs per 256x256 tile (tcgen05 cta_group::2):
+                                 each CTA stages and splits 128 rows of A and 128 columns of
+                                 B; the default for M, N >= 256                           */
   HEAL_TILE_SKINNY_SPLITK = 2 /* operands swapped (weights on the MMA M side), K split
                                  over CTAs; needs a workspace                           */
 };

@@ -53,10 +53,11 @@ def test_ragged_shapes_against_oracle(shape, b_layout):
     assert np.all(np.isfinite(C))
 
 
-def test_repeat_runs_bitwise_identical():
+@pytest.mark.parametrize("tile", [heal.TILE_128x128, heal.TILE_256x256_PAIR])
+def test_repeat_runs_bitwise_identical(tile):
     X, W = synthetic.gemm_prefill(M=384, K=1024, N=512)
     X, W = X.numpy(), W.numpy()
-    outs = [gemm(X, W, tile=heal.TILE_128x128) for _ in range(5)]
+    outs = [gemm(X, W, tile=tile) for _ in range(5)]
     for o in outs[1:]:
         assert np.array_equal(o.view(np.uint64), outs[0].view(np.uint64))
 
@@ -69,7 +70,9 @@ def test_tile_configs_bitwise_identical(M, b_layout):
     Bin = W if b_layout == 0 else np.ascontiguousarray(W.T)
     c_full = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_128x128)
     c_skinny = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_SKINNY_SPLITK)
+    c_pair = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_256x256_PAIR)
     assert np.array_equal(c_full, c_skinny)
+    assert np.array_equal(c_full, c_pair)
     assert G.normwise_rel_err(c_full, G.gemm_ref(X, W)) <= TOL_FP16
 
 
@@ -133,3 +136,32 @@ def test_prefill_full_size_sampled_rows():
     got = C[torch.as_tensor(rows, device=d)].cpu().numpy()
     assert G.normwise_rel_err(got, ref) <= TOL_FP16
     assert torch.isfinite(C).all()
+
+
+@pytest.mark.parametrize("shape", [(512, 512, 512), (300, 520, 333), (256, 1000, 64), (777, 300, 1500)])
+@pytest.mark.parametrize("b_layout", [0, 1])
+def test_cta_pair_config_bitwise_and_oracle(shape, b_layout):
+    """The 256x256 CTA-pair kernel (tcgen05 cta_group::2) gives the same bits as the
+    single-CTA kernel and meets the oracle bound, ragged edges included."""
+    M, N, K = shape
+    X, W = synthetic.gemm_prefill(M=M, K=K, N=N)
+    X, W = X.numpy(), W.numpy()
+    Bin = W if b_layout == 0 else np.ascontiguousarray(W.T)
+    c_pair = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_256x256_PAIR)
+    c_single = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_128x128)
+    assert np.array_equal(c_pair, c_single)
+    assert G.normwise_rel_err(c_pair, G.gemm_ref(X, W)) <= TOL_FP16
+
+
+@pytest.mark.parametrize("fmt", [heal.SPLIT_FP16_S11, heal.SPLIT_BF16])
+def test_cta_pair_presplit_and_bf16(fmt):
+    d = dev()
+    X, W = synthetic.gemm_prefill(M=512, K=768, N=640)
+    W_d = W.to(d)
+    hi = torch.empty(W_d.shape, dtype=torch.int16, device=d)
+    lo = torch.empty(W_d.shape, dtype=torch.int16, device=d)
+    heal.heal_split(W_d, hi, lo, fmt)
+    c_pre = gemm(X.numpy(), hi, fmt=fmt, tile=heal.TILE_256x256_PAIR, b_lo=lo)
+    c_in = gemm(X.numpy(), W.numpy(), fmt=fmt, tile=heal.TILE_256x256_PAIR)
+    c_single = gemm(X.numpy(), W.numpy(), fmt=fmt, tile=heal.TILE_128x128)
+    assert np.array_equal(c_pre, c_in) and np.array_equal(c_in, c_single)
