@@ -9,9 +9,11 @@
 // every partial sum of every term is an integer below 2^24 in magnitude, so the FP16 tensor
 // core products accumulate exactly in FP32; the three sums are combined in int64.
 //   logit = fp32( (double(S_int) * (double(s_q) * double(s_k))) * double(softmax_scale) )
-// FP32 online softmax in base 2; P is folded with the per-token V scale and a per-segment
-// power of two, split into an FP16 pair (P_hi, P_lo * 2^-11), and multiplied with the
-// byte-split V (V_hi = 256*(v >> 8), V_lo = v & 255) on FP16 tensor cores.
+// FP32 online softmax in base 2.  P is folded with the per-token V scale and a per-block
+// power of two 2^E (chosen so the block's largest V scale times 2^E lies in [32, 64)),
+// then split into FP16 P_hi and the FP16 residual r = P - P_hi; the byte-split V
+// (hi = v >> 8, lo = v & 255) meets (256*P_hi, P_hi, 256*r, r) in four FP16 tensor-core
+// products that accumulate into one FP32 accumulator: sum 256*hi*P + lo*P = v*P.
 //
 // Work decomposition: a persistent grid; CTA c owns the contiguous slice
 // [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token block)
@@ -69,11 +71,6 @@ __device__ __forceinline__ uint32_t hi_pair(uint32_t x) {
   const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&u), __half2half2(__ushort_as_half(0x6480)));
   return *reinterpret_cast<const uint32_t*>(&h);   // 0x6480 = 1152 = 1024 + 128
 }
-__device__ __forceinline__ uint32_t hi256_pair(uint32_t x) {   // 256 * hi, exact in FP16
-  const uint32_t h = hi_pair(x);
-  const __half2 r = __hmul2(*reinterpret_cast<const __half2*>(&h), __half2half2(__ushort_as_half(0x5C00)));
-  return *reinterpret_cast<const uint32_t*>(&r);   // 0x5C00 = 256.0
-}
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                          uint32_t b0, uint32_t b1) {
@@ -115,7 +112,7 @@ __device__ __forceinline__ float* slot_ptr(float* ws, int c, int p, int R, int D
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                        const __grid_constant__ CUtensorMap tmV,
                                                                        const AttnArgs a) {
   constexpr int kBoxes = D / 64;                    // 64-dim (128-byte) boxes per row
@@ -127,7 +124,8 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
   uint8_t* stages = smem;                                            // 2 x kStageBytes
   float* o_sm = reinterpret_cast<float*>(smem + 2 * kStageBytes);    // [kRows][D]
   float* ml_sm = o_sm + kRows * D;                                   // [kCompute][kRows][2]
-  uint64_t* full = reinterpret_cast<uint64_t*>(ml_sm + kCompute * kRows * 2);
+  uint4* qf_sm = reinterpret_cast<uint4*>(ml_sm + kCompute * kRows * 2); // [kKSteps][32 lanes]
+  uint64_t* full = reinterpret_cast<uint64_t*>(qf_sm + kKSteps * 32);
   uint64_t* empty = full + 2;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 2);
 
@@ -183,13 +181,12 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
   const int R = a.R;
   const int rowS = lane >> 2;                 // S layout: query row of c0/c1
   const int tokq = 2 * (lane & 3);            // S layout: first token (of 8) of c0/c1
-  uint32_t qh[kKSteps][2], ql[kKSteps][2];    // A fragments (rows 0-7; rows 8-15 are zero)
   float sq = 0.0f;
   int pos = 0;
   float m_run = -INFINITY, l_run = 0.0f;      // S layout, row rowS
-  float om[D / 16][4], oc[D / 16][4];         // O^T main / correction accumulators
-  float vscale = 1.0f;                        // 2^E folded into P
-  float inv_vscale = 1.0f;
+  float om[D / 16][4];                        // O^T accumulator (units of 2^E_run)
+  int E_run = 0;                              // power of two folded into P (decreases only)
+  bool have_E = false;
   int cur_p = -1, b = 0, hkv = 0, klen = 0;
   int it = 0;
   bool ok = true;
@@ -215,15 +212,12 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
       M[h] = mx;
       f[h] = (mw == -INFINITY) ? 0.0f : exp2f(mw - mx);
     }
-    // O of this warp, scaled to the CTA max, in true units (x 2^-E)
-    float o[D / 16][4];
+    // O of this warp, scaled to the CTA max, in true units (x 2^-E_run), in place
+    const float u = ldexpf(1.0f, -E_run);
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const float v = __fmaf_rn(oc[dt][e], 1.0f / 2048.0f, om[dt][e]);
-        o[dt][e] = __fmul_rn(__fmul_rn(v, inv_vscale), f[e & 1]);
-      }
+      for (int e = 0; e < 4; ++e) om[dt][e] = __fmul_rn(__fmul_rn(om[dt][e], u), f[e & 1]);
     // sequential, fixed-order merge of the four warps through shared memory
     for (int w = 0; w < kCompute; ++w) {
       if (warp == w) {
@@ -234,7 +228,7 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
             const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
             const int r = tokq + (e & 1);
             float* dst = o_sm + r * D + d;
-            const float v = (w == 0) ? o[dt][e] : __fadd_rn(*dst, o[dt][e]);
+            const float v = (w == 0) ? om[dt][e] : __fadd_rn(*dst, om[dt][e]);
             if (w < kCompute - 1) {
               *dst = v;
             } else if (r < R) {
@@ -276,30 +270,29 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
       const long long qrow = ((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq);
       sq = real ? __ldg(a.qs + qrow) : 0.0f;
       pos = klen - a.Tq + tq;
+      // A fragments of Q (rows 0-7; rows 8-15 are zero), byte-split, one table per CTA:
+      // entry [ks][lane] = (hi dims 2t.., hi dims 2t+8.., lo dims 2t.., lo dims 2t+8..)
+      if (warp == 0) {
 #pragma unroll
-      for (int ks = 0; ks < kKSteps; ++ks) {
-        uint32_t w0 = 0, w1 = 0;
-        if (real) {
-          const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow * D + ks * 16 + tokq);
-          w0 = __ldg(qp);
-          w1 = __ldg(qp + 4);   // dims + 8
+        for (int ks = 0; ks < kKSteps; ++ks) {
+          uint32_t w0 = 0, w1 = 0;
+          if (real) {
+            const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow * D + ks * 16 + tokq);
+            w0 = __ldg(qp);
+            w1 = __ldg(qp + 4);   // dims + 8
+          }
+          qf_sm[ks * 32 + lane] = make_uint4(hi_pair(w0), hi_pair(w1), lo_pair(w0), lo_pair(w1));
         }
-        qh[ks][0] = hi_pair(w0);
-        qh[ks][1] = hi_pair(w1);
-        ql[ks][0] = lo_pair(w0);
-        ql[ks][1] = lo_pair(w1);
       }
-      // power of two that brings this head's V scales near 1 (token 0 is always valid)
-      const float s0 = __ldg(a.vs + (size_t)p * a.Tmax);
-      const int E = (s0 > 0.0f) ? (-ilogbf(s0) - 6) : 0;
-      vscale = ldexpf(1.0f, E);
-      inv_vscale = ldexpf(1.0f, -E);
+      compute_bar();
       m_run = -INFINITY;
       l_run = 0.0f;
+      E_run = 0;
+      have_E = false;
 #pragma unroll
       for (int dt = 0; dt < D / 16; ++dt)
 #pragma unroll
-        for (int e = 0; e < 4; ++e) om[dt][e] = oc[dt][e] = 0.0f;
+        for (int e = 0; e < 4; ++e) om[dt][e] = 0.0f;
     }
     const int t0 = blk * kBlk;
     if (t0 >= klen) continue;
@@ -316,38 +309,45 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
 
     // ---- exact S = Q K^T on the byte-split operands ----
     float x[2][2];                            // [n-block][token] logits * log2(e), row rowS
+    float shh[2][4], sx[2][4], sll[2][4];
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      float shh[4] = {0, 0, 0, 0}, sx[4] = {0, 0, 0, 0}, sll[4] = {0, 0, 0, 0};
+    for (int nb = 0; nb < 2; ++nb)
 #pragma unroll
-      for (int j = 0; j < kKSteps / 2; ++j) {
+      for (int e = 0; e < 4; ++e) shh[nb][e] = sx[nb][e] = sll[nb][e] = 0.0f;
+#pragma unroll
+    for (int j = 0; j < kKSteps / 2; ++j) {
+      const uint4 qa = qf_sm[(2 * j) * 32 + lane];
+      const uint4 qb = qf_sm[(2 * j + 1) * 32 + lane];
+#pragma unroll
+      for (int nb = 0; nb < 2; ++nb) {
         const int trow = tw + nb * 8 + (lane & 7);
         const int ch = 4 * j + (lane >> 3);   // 16-byte chunk of the 256-byte K row
         const uint32_t addr = kst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
         uint32_t r0, r1, r2, r3;
         ldsm_x4(addr, r0, r1, r2, r3);
         {
-          const int ks = 2 * j;
           const uint32_t kh0 = hi_pair(r0), kh1 = hi_pair(r1), kl0 = lo_pair(r0), kl1 = lo_pair(r1);
-          mma16816(shh, qh[ks][0], 0u, qh[ks][1], 0u, kh0, kh1);
-          mma16816(sx, qh[ks][0], 0u, qh[ks][1], 0u, kl0, kl1);
-          mma16816(sx, ql[ks][0], 0u, ql[ks][1], 0u, kh0, kh1);
-          mma16816(sll, ql[ks][0], 0u, ql[ks][1], 0u, kl0, kl1);
+          mma16816(shh[nb], qa.x, 0u, qa.y, 0u, kh0, kh1);
+          mma16816(sx[nb], qa.x, 0u, qa.y, 0u, kl0, kl1);
+          mma16816(sx[nb], qa.z, 0u, qa.w, 0u, kh0, kh1);
+          mma16816(sll[nb], qa.z, 0u, qa.w, 0u, kl0, kl1);
         }
         {
-          const int ks = 2 * j + 1;
           const uint32_t kh0 = hi_pair(r2), kh1 = hi_pair(r3), kl0 = lo_pair(r2), kl1 = lo_pair(r3);
-          mma16816(shh, qh[ks][0], 0u, qh[ks][1], 0u, kh0, kh1);
-          mma16816(sx, qh[ks][0], 0u, qh[ks][1], 0u, kl0, kl1);
-          mma16816(sx, ql[ks][0], 0u, ql[ks][1], 0u, kh0, kh1);
-          mma16816(sll, ql[ks][0], 0u, ql[ks][1], 0u, kl0, kl1);
+          mma16816(shh[nb], qb.x, 0u, qb.y, 0u, kh0, kh1);
+          mma16816(sx[nb], qb.x, 0u, qb.y, 0u, kl0, kl1);
+          mma16816(sx[nb], qb.z, 0u, qb.w, 0u, kh0, kh1);
+          mma16816(sll[nb], qb.z, 0u, qb.w, 0u, kl0, kl1);
         }
       }
+    }
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int t = t0 + tw + nb * 8 + tokq + e;
-        const long long S = ((long long)__float2int_rn(shh[e]) << 16) + ((long long)__float2int_rn(sx[e]) << 8) +
-                            (long long)__float2int_rn(sll[e]);
+        const long long S = ((long long)__float2int_rn(shh[nb][e]) << 16) +
+                            ((long long)__float2int_rn(sx[nb][e]) << 8) + (long long)__float2int_rn(sll[nb][e]);
         const bool real = rowS < R;
         const bool vis = real && t < klen && (!a.causal || t <= pos);
         float xv;
@@ -386,41 +386,61 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
     }
     l_run = __fadd_rn(__fmul_rn(l_run, alpha), __fadd_rn(__fadd_rn(pv[0][0], pv[0][1]), __fadd_rn(pv[1][0], pv[1][1])));
     m_run = m_new;
+    // power of two for this block: the largest visible V scale times 2^E in [32, 64)
+    float smax = 0.0f;
+    {
+      const int ta = t0 + lane, tb = t0 + 32 + lane;
+      if (ta < klen) smax = __ldg(a.vs + (size_t)p * a.Tmax + ta);
+      if (tb < klen) smax = fmaxf(smax, __ldg(a.vs + (size_t)p * a.Tmax + tb));
+#pragma unroll
+      for (int o = 16; o >= 1; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+    }
+    float escale = 1.0f;                       // 2^(E_new - E_run) applied to O
+    if (smax > 0.0f) {
+      const int E_blk = 5 - ilogbf(smax);
+      if (!have_E) {
+        E_run = E_blk;
+        have_E = true;
+      } else if (E_blk < E_run) {
+        escale = ldexpf(1.0f, E_blk - E_run);
+        E_run = E_blk;
+      }
+    }
     // rescale O^T rows tokq, tokq+1: their alphas live in S-layout lanes 4*tokq, 4*(tokq+1)
-    const float a0 = __shfl_sync(0xffffffffu, alpha, 4 * tokq);
-    const float a1 = __shfl_sync(0xffffffffu, alpha, 4 * (tokq + 1));
+    const float a0 = __fmul_rn(__shfl_sync(0xffffffffu, alpha, 4 * tokq), escale);
+    const float a1 = __fmul_rn(__shfl_sync(0xffffffffu, alpha, 4 * (tokq + 1)), escale);
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt) {
       om[dt][0] = __fmul_rn(om[dt][0], a0);
       om[dt][1] = __fmul_rn(om[dt][1], a1);
       om[dt][2] = __fmul_rn(om[dt][2], a0);
       om[dt][3] = __fmul_rn(om[dt][3], a1);
-      oc[dt][0] = __fmul_rn(oc[dt][0], a0);
-      oc[dt][1] = __fmul_rn(oc[dt][1], a1);
-      oc[dt][2] = __fmul_rn(oc[dt][2], a0);
-      oc[dt][3] = __fmul_rn(oc[dt][3], a1);
     }
 
-    // ---- P' = P * s_v * 2^E split into FP16 (hi, lo * 2^-11): B fragments of PV ----
-    uint32_t ph_[2], pl_[2];
+    // ---- P' = P * s_v * 2^E as FP16 (P_hi, r = P' - P_hi): B fragments of PV ----
+    const float e2 = ldexpf(1.0f, E_run);
+    uint32_t ph_[2], pr_[2], ph256[2], pr256[2];
 #pragma unroll
     for (int nb = 0; nb < 2; ++nb) {
       float pp[2];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int t = t0 + tw + nb * 8 + tokq + e;
-        const float sv = (pv[nb][e] != 0.0f) ? __fmul_rn(__ldg(a.vs + (size_t)p * a.Tmax + t), vscale) : 0.0f;
+        const float sv = (pv[nb][e] != 0.0f) ? __fmul_rn(__ldg(a.vs + (size_t)p * a.Tmax + t), e2) : 0.0f;
         pp[e] = __fmul_rn(pv[nb][e], sv);
       }
       const __half2 h = __floats2half2_rn(pp[0], pp[1]);
       const float2 hf = __half22float2(h);
-      const __half2 l = __floats2half2_rn(__fmul_rn(__fsub_rn(pp[0], hf.x), 2048.0f),
-                                          __fmul_rn(__fsub_rn(pp[1], hf.y), 2048.0f));
+      const __half2 r = __floats2half2_rn(__fsub_rn(pp[0], hf.x), __fsub_rn(pp[1], hf.y));
+      const __half2 k256 = __half2half2(__ushort_as_half(0x5C00));   // 256.0
+      const __half2 h256 = __hmul2(h, k256), r256 = __hmul2(r, k256); // exact: powers of two
       ph_[nb] = *reinterpret_cast<const uint32_t*>(&h);
-      pl_[nb] = *reinterpret_cast<const uint32_t*>(&l);
+      pr_[nb] = *reinterpret_cast<const uint32_t*>(&r);
+      ph256[nb] = *reinterpret_cast<const uint32_t*>(&h256);
+      pr256[nb] = *reinterpret_cast<const uint32_t*>(&r256);
     }
 
-    // ---- O^T += V'^T P'^T ----
+    // ---- O^T += V^T P'^T  (256*hi*P + lo*P with P = P_hi + r) ----
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt) {
       const int mi = lane >> 3;
@@ -429,12 +449,12 @@ __global__ void __launch_bounds__(kAttnThreads) heal_attn_decode_kernel(const __
       const uint32_t addr = vst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
       uint32_t r0, r1, r2, r3;
       ldsm_x4_t(addr, r0, r1, r2, r3);
-      const uint32_t h0 = hi256_pair(r0), h1 = hi256_pair(r1), h2 = hi256_pair(r2), h3 = hi256_pair(r3);
+      const uint32_t h0 = hi_pair(r0), h1 = hi_pair(r1), h2 = hi_pair(r2), h3 = hi_pair(r3);
       const uint32_t l0 = lo_pair(r0), l1 = lo_pair(r1), l2 = lo_pair(r2), l3 = lo_pair(r3);
-      mma16816(om[dt], h0, h1, h2, h3, ph_[0], ph_[1]);
+      mma16816(om[dt], h0, h1, h2, h3, ph256[0], ph256[1]);
       mma16816(om[dt], l0, l1, l2, l3, ph_[0], ph_[1]);
-      mma16816(oc[dt], h0, h1, h2, h3, pl_[0], pl_[1]);
-      mma16816(oc[dt], l0, l1, l2, l3, pl_[0], pl_[1]);
+      mma16816(om[dt], h0, h1, h2, h3, pr256[0], pr256[1]);
+      mma16816(om[dt], l0, l1, l2, l3, pr_[0], pr_[1]);
     }
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
@@ -470,7 +490,7 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
 
 template <int D>
 constexpr int attn_smem_bytes() {
-  return 2 * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + 64 + 1024;
+  return 2 * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + (D / 16) * 32 * 16 + 64 + 1024;
 }
 
 }  // namespace
