@@ -125,7 +125,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
   float* o_sm = reinterpret_cast<float*>(smem + 2 * kStageBytes);    // [kRows][D]
   float* ml_sm = o_sm + kRows * D;                                   // [kCompute][kRows][2]
   uint4* qf_sm = reinterpret_cast<uint4*>(ml_sm + kCompute * kRows * 2); // [kKSteps][32 lanes]
-  uint64_t* full = reinterpret_cast<uint64_t*>(qf_sm + kKSteps * 32);
+  float* sc_sm = reinterpret_cast<float*>(qf_sm + kKSteps * 32);        // [2 stages][K, V][kBlk]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sc_sm + 2 * 2 * kBlk);
   uint64_t* empty = full + 2;
   volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 2);
 
@@ -158,8 +159,10 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         const uint32_t ph = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.status, 200)) break;
         uint8_t* st = stages + s * kStageBytes;
-        mbar_arrive_expect_tx(&full[s], kStageBytes);
+        mbar_arrive_expect_tx(&full[s], kStageBytes + 2 * kBlk * 4);
         const int row = p * a.Tmax + t0;
+        bulk_load_1d(sc_sm + (s * 2 + 0) * kBlk, a.ks + (size_t)row, kBlk * 4, &full[s]);
+        bulk_load_1d(sc_sm + (s * 2 + 1) * kBlk, a.vs + (size_t)row, kBlk * 4, &full[s]);
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) {
           tma_load_2d(st + bx * 8192, &tmK, &full[s], bx * 64, row);
@@ -305,6 +308,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
     }
     const uint32_t kst = smem_u32(stages + s * kStageBytes);
     const uint32_t vst = kst + kTileBytes;
+    const float* sks = sc_sm + (s * 2 + 0) * kBlk;   // K scales of this block's 64 tokens
+    const float* svs = sc_sm + (s * 2 + 1) * kBlk;   // V scales
     const int tw = warp * 16;                 // this warp's first token inside the tile
 
     // ---- exact S = Q K^T on the byte-split operands ----
@@ -356,7 +361,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         } else if (!vis) {
           xv = -INFINITY;
         } else {
-          const double coef = (double)sq * (double)__ldg(a.ks + (size_t)p * a.Tmax + t);
+          const double coef = (double)sq * (double)sks[t - t0];
           const float lg = (float)(((double)S * coef) * (double)a.scale);
           xv = __fmul_rn(lg, kLog2e);
           if (a.qk_out) {
@@ -390,8 +395,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
     float smax = 0.0f;
     {
       const int ta = t0 + lane, tb = t0 + 32 + lane;
-      if (ta < klen) smax = __ldg(a.vs + (size_t)p * a.Tmax + ta);
-      if (tb < klen) smax = fmaxf(smax, __ldg(a.vs + (size_t)p * a.Tmax + tb));
+      if (ta < klen) smax = svs[lane];
+      if (tb < klen) smax = fmaxf(smax, svs[32 + lane]);
 #pragma unroll
       for (int o = 16; o >= 1; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
     }
@@ -426,7 +431,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int t = t0 + tw + nb * 8 + tokq + e;
-        const float sv = (pv[nb][e] != 0.0f) ? __fmul_rn(__ldg(a.vs + (size_t)p * a.Tmax + t), e2) : 0.0f;
+        const float sv = (pv[nb][e] != 0.0f) ? __fmul_rn(svs[t - t0], e2) : 0.0f;
         pp[e] = __fmul_rn(pv[nb][e], sv);
       }
       const __half2 h = __floats2half2_rn(pp[0], pp[1]);
@@ -490,7 +495,8 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
 
 template <int D>
 constexpr int attn_smem_bytes() {
-  return 2 * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + (D / 16) * 32 * 16 + 64 + 1024;
+  return 2 * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + (D / 16) * 32 * 16 + 2 * 2 * kBlk * 4 +
+         64 + 1024;
 }
 
 }  // namespace
@@ -532,6 +538,12 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   a.causal = causal;
   a.scale = scale;
   a.total = (long long)B * Hkv * a.nblk;
+  // opt in to the large shared-memory carve-out first: the occupancy query depends on it
+  if (cudaFuncSetAttribute(heal_attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           attn_smem_bytes<128>()) != cudaSuccess ||
+      cudaFuncSetAttribute(heal_attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           attn_smem_bytes<64>()) != cudaSuccess)
+    return HEAL_ERR_CUDA;
   int per_sm = 0;
   if (D == 128)
     cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<128>, kAttnThreads,
@@ -548,11 +560,6 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   if ((size_t)(a.grid + (long long)B * Hkv) * (size_t)R * (size_t)(D + 2) * sizeof(float) > ws_bytes)
     return HEAL_ERR_INVALID_ARGUMENT;
 
-  if (cudaFuncSetAttribute(heal_attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           attn_smem_bytes<128>()) != cudaSuccess ||
-      cudaFuncSetAttribute(heal_attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           attn_smem_bytes<64>()) != cudaSuccess)
-    return HEAL_ERR_CUDA;
   CUtensorMap tk{}, tv{};
   const cuuint64_t dims[2] = {(cuuint64_t)D, (cuuint64_t)rows_total};
   const cuuint64_t strides[1] = {(cuuint64_t)D * 2};

@@ -145,7 +145,7 @@ heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale, const
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tmax <= 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (Hq % Hkv != 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (D != 64 && D != 128) return HEAL_ERR_UNSUPPORTED;
-  if ((Hq / Hkv) * Tq > 16) return HEAL_ERR_UNSUPPORTED;
+  if ((Hq / Hkv) * Tq > 8) return HEAL_ERR_UNSUPPORTED;
   if (Tmax % 64 != 0) return HEAL_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return HEAL_ERR_INVALID_ARGUMENT;
   if (!(softmax_scale > 0.0f) || softmax_scale != softmax_scale) return HEAL_ERR_INVALID_ARGUMENT;
@@ -154,7 +154,7 @@ heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale, const
   if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(out, 16) ||
       !aligned(workspace, 16))
     return HEAL_ERR_INVALID_ARGUMENT;
-  if (!aligned(q_scale, 4) || !aligned(k_scale, 4) || !aligned(v_scale, 4) || !aligned(kv_len, 4))
+  if (!aligned(q_scale, 4) || !aligned(k_scale, 16) || !aligned(v_scale, 16) || !aligned(kv_len, 4))
     return HEAL_ERR_INVALID_ARGUMENT;
   if (qk_int_out && !aligned(qk_int_out, 8)) return HEAL_ERR_INVALID_ARGUMENT;
   if (workspace_bytes < attention_workspace_bytes(B, Hq, Tq, Tmax)) return HEAL_ERR_INVALID_ARGUMENT;

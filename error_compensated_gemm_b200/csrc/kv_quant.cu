@@ -35,38 +35,46 @@ __global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restri
     const int b = bt / T, t = bt - b * T;
     const char* xrow = static_cast<const char*>(x) + (size_t)(b * sb + (long long)t * st) * (BF16 ? 2 : 4);
     for (int h0 = 0; h0 < H; h0 += kRowsPerPass * kUnroll) {
-      float v[kUnroll][8];
+      // all loads of the pass group first, kept as raw words (4 registers per 16 bytes)
+      uint4 raw[kUnroll][BF16 ? 1 : 2];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
         const int h = h0 + u * kRowsPerPass + grp;
         if (h < H) {
           if constexpr (BF16) {
-            const uint4 raw = __ldcs(reinterpret_cast<const uint4*>(
-                reinterpret_cast<const __nv_bfloat16*>(xrow) + (size_t)h * sh + sub * 8));
-            const __nv_bfloat162* pb = reinterpret_cast<const __nv_bfloat162*>(&raw);
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-              const float2 f = __bfloat1622float2(pb[j]);
-              v[u][2 * j] = f.x;
-              v[u][2 * j + 1] = f.y;
-            }
+            raw[u][0] = __ldcs(reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(xrow) +
+                                                              (size_t)h * sh + sub * 8));
           } else {
-            const float4* pf = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(xrow) + (size_t)h * sh +
-                                                               sub * 8);
-            const float4 a0 = __ldcs(pf), a1 = __ldcs(pf + 1);
-            v[u][0] = a0.x; v[u][1] = a0.y; v[u][2] = a0.z; v[u][3] = a0.w;
-            v[u][4] = a1.x; v[u][5] = a1.y; v[u][6] = a1.z; v[u][7] = a1.w;
+            const uint4* pf = reinterpret_cast<const uint4*>(reinterpret_cast<const float*>(xrow) + (size_t)h * sh +
+                                                             sub * 8);
+            raw[u][0] = __ldcs(pf);
+            raw[u][1] = __ldcs(pf + 1);
           }
         } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v[u][j] = 0.0f;
+          raw[u][0] = make_uint4(0, 0, 0, 0);
+          if constexpr (!BF16) raw[u][1] = make_uint4(0, 0, 0, 0);
         }
       }
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
+        float vv[8];
+        if constexpr (BF16) {
+          // bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 pattern
+          const uint32_t w[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            vv[2 * j] = __uint_as_float(w[j] << 16);
+            vv[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+          }
+        } else {
+          const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
+                                 raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) vv[j] = __uint_as_float(w[j]);
+        }
         float m = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(v[u][j]));
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(vv[j]));
 #pragma unroll
         for (int o = L / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
         const int h = h0 + u * kRowsPerPass + grp;
@@ -77,7 +85,7 @@ __global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restri
           const float inv = __fdiv_rn(32767.0f, m);
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int qi = __float2int_rn(__fmul_rn(v[u][j], inv));
+            const int qi = __float2int_rn(__fmul_rn(vv[j], inv));
             qv[j] = qi > 32767 ? 32767 : (qi < -32767 ? -32767 : qi);
           }
         } else {

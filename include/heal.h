@@ -123,7 +123,7 @@ size_t heal_gemm_workspace_bytes(int M, int N, int K, const heal_gemm_opts_t* op
  *   scale_cache : device float32 [B, H, Tmax], same rows written
  * Per (token, head) row: absmax = max|x|, inv = fp32(32767/absmax),
  * q = clamp(rint(fp32(x*inv)), +-32767), s = fp32(absmax/32767); an all-zero row gives
- * q = 0, s = 0.  D must be a multiple of 8 and <= 256; x, q_cache 16-byte aligned;
+ * q = 0, s = 0.  D must be a power of two in [8, 256]; x, q_cache 16-byte aligned;
  * strides multiples of 8 elements.  t_offset + T <= Tmax.                              */
 heal_status_t heal_kv_quantize_int16(const void* x, int x_is_bf16,
                                      int B, int T, int H, int D,
@@ -145,7 +145,8 @@ heal_status_t heal_kv_quantize_int16(const void* x, int x_is_bf16,
  * evaluated in double; FP32 online softmax; PV with P split into two FP16 parts and V
  * byte-split.  The context is cut into chunks whose partial results are merged in
  * ascending chunk order.
- * Limits: D in {64, 128}; Hq % Hkv == 0; (Hq/Hkv) * Tq <= 16; Tmax % 64 == 0.
+ * Limits: D in {64, 128}; Hq % Hkv == 0; (Hq/Hkv) * Tq <= 8; Tmax % 64 == 0;
+ * q, the caches, k_scale, v_scale, out and workspace 16-byte aligned.
  * workspace  : device, >= heal_attention_workspace_bytes(B, Hq, Tq, Tmax) bytes
  * qk_int_out : nullable test hook, int64 [B, Hq, Tq, Tmax]; when given, the exact
  *              S_int of every visible (query, token) pair is written there.          */
