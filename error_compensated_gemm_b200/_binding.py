@@ -14,7 +14,8 @@ TILE_AUTO, TILE_128x128, TILE_256x256_PAIR, TILE_SKINNY_SPLITK = -1, 0, 1, 2
 # every symbol the public header declares
 EXPORTED = ("heal_split", "heal_gemm_compensated", "heal_gemm_workspace_bytes", "heal_kv_quantize_int16",
             "heal_attention_int16", "heal_attention_workspace_bytes", "heal_get_device_status",
-            "heal_status_string", "heal_version", "heal_attention_int16_noalloc")
+            "heal_status_string", "heal_version", "heal_attention_int16_noalloc", "heal_embedding_gather",
+            "heal_rmsnorm", "heal_rope", "heal_swiglu", "heal_add", "heal_argmax")
 
 
 class HealError(RuntimeError):
@@ -53,6 +54,12 @@ def lib():
         "heal_attention_int16_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _f, _i, _vp,
                                           _vp, _vp], _i),
         "heal_get_device_status": ([_vp], _i),
+        "heal_embedding_gather": ([_vp, _i, _i, _vp, _i, _vp, _vp], _i),
+        "heal_rmsnorm": ([_vp, _vp, _i, _i, _f, _vp, _vp], _i),
+        "heal_rope": ([_vp, _i, _i, _i, _i64, _vp, _vp, _vp, _vp], _i),
+        "heal_swiglu": ([_vp, _i, _i, _vp, _vp], _i),
+        "heal_add": ([_vp, _vp, _i64, _vp], _i),
+        "heal_argmax": ([_vp, _i, _i, _vp, _vp], _i),
         "heal_status_string": ([_i], ctypes.c_char_p),
         "heal_version": ([], ctypes.c_char_p),
     }
@@ -194,6 +201,43 @@ def heal_attention_int16_noalloc(q, q_scale, k_cache, k_scale, v_cache, v_scale,
                                             float(softmax_scale), 1 if causal else 0, _ptr(out), _ptr(qk_int_out),
                                             _stream(stream))
     _check(st, "heal_attention_int16_noalloc")
+
+
+def heal_embedding_gather(table, ids, out, stream=None):
+    _cuda(table, ids, out)
+    vocab, H = table.shape
+    _check(lib().heal_embedding_gather(_ptr(table), vocab, H, _ptr(ids), ids.numel(), _ptr(out), _stream(stream)),
+           "heal_embedding_gather")
+
+
+def heal_rmsnorm(x, w, y, eps=1e-5, stream=None):
+    _cuda(x, w, y)
+    n, H = x.shape
+    _check(lib().heal_rmsnorm(_ptr(x), _ptr(w), n, H, float(eps), _ptr(y), _stream(stream)), "heal_rmsnorm")
+
+
+def heal_rope(x, heads, D, pos, cos_t, sin_t, stream=None):
+    """In place on x [n, >= heads*D] (row stride x.stride(0))."""
+    _cuda(x, pos, cos_t, sin_t)
+    _check(lib().heal_rope(_ptr(x), x.shape[0], heads, D, x.stride(0), _ptr(pos), _ptr(cos_t), _ptr(sin_t),
+                           _stream(stream)), "heal_rope")
+
+
+def heal_swiglu(gate_up, out, stream=None):
+    _cuda(gate_up, out)
+    n, F = out.shape
+    _check(lib().heal_swiglu(_ptr(gate_up), n, F, _ptr(out), _stream(stream)), "heal_swiglu")
+
+
+def heal_add(x, y, stream=None):
+    _cuda(x, y)
+    _check(lib().heal_add(_ptr(x), _ptr(y), x.numel(), _stream(stream)), "heal_add")
+
+
+def heal_argmax(x, out, stream=None):
+    _cuda(x, out)
+    rows, n = x.shape
+    _check(lib().heal_argmax(_ptr(x), rows, n, _ptr(out), _stream(stream)), "heal_argmax")
 
 
 def heal_get_device_status(stream=None):

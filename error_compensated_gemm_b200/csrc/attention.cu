@@ -18,7 +18,7 @@
 // Work decomposition: a persistent grid; CTA c owns the contiguous slice
 // [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token block)
 // units.  Warp 4 streams 64-token K and V tiles with TMA (128-byte swizzle) into a
-// two-stage ring; warps 0-3 each take 16 tokens of a tile with mma.sync m16n8k16 (the
+// two-stage ring (the K half of a stage is released after QK^T, the V half after PV); warps 0-3 each take 16 tokens of a tile with mma.sync m16n8k16 (the
 // decode GEMV shapes are far below a tcgen05 tile; the kernel is HBM-bound).  Every
 // (CTA, kv head) segment leaves one partial (m, l, o) in the workspace; the combine kernel
 // merges them in ascending token order.  The order is fixed, so results are identical
@@ -126,16 +126,16 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
   float* ml_sm = o_sm + kRows * D;                                   // [kCompute][kRows][2]
   uint4* qf_sm = reinterpret_cast<uint4*>(ml_sm + kCompute * kRows * 2); // [kKSteps][32 lanes]
   float* sc_sm = reinterpret_cast<float*>(qf_sm + kKSteps * 32);        // [2 stages][K, V][kBlk]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sc_sm + 2 * 2 * kBlk);
-  uint64_t* empty = full + 2;
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 2);
+  uint64_t* full = reinterpret_cast<uint64_t*>(sc_sm + 2 * 2 * kBlk);  // [2] K tile, [2] V tile + scales
+  uint64_t* empty = full + 4;                                          // [2] K released, [2] V released
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   const long long u0 = unit_begin(a.total, a.grid, c), u1 = unit_begin(a.total, a.grid, c + 1);
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < 4; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCompute);
     }
@@ -157,17 +157,21 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         if (t0 >= __ldg(a.kv_len + b)) continue;
         const int s = it & 1;
         const uint32_t ph = (uint32_t)(it >> 1) & 1u;
-        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.status, 200)) break;
         uint8_t* st = stages + s * kStageBytes;
-        mbar_arrive_expect_tx(&full[s], kStageBytes + 2 * kBlk * 4);
         const int row = p * a.Tmax + t0;
+        // K half: refilled as soon as the compute warps finish QK^T on the previous tile
+        if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.status, 200)) break;
+        mbar_arrive_expect_tx(&full[s], kTileBytes + kBlk * 4);
         bulk_load_1d(sc_sm + (s * 2 + 0) * kBlk, a.ks + (size_t)row, kBlk * 4, &full[s]);
-        bulk_load_1d(sc_sm + (s * 2 + 1) * kBlk, a.vs + (size_t)row, kBlk * 4, &full[s]);
 #pragma unroll
-        for (int bx = 0; bx < kBoxes; ++bx) {
-          tma_load_2d(st + bx * 8192, &tmK, &full[s], bx * 64, row);
-          tma_load_2d(st + kTileBytes + bx * 8192, &tmV, &full[s], bx * 64, row);
-        }
+        for (int bx = 0; bx < kBoxes; ++bx) tma_load_2d(st + bx * 8192, &tmK, &full[s], bx * 64, row);
+        // V half and V scales
+        if (!mbar_wait(&empty[2 + s], ph ^ 1u, abort_flag, a.status, 202)) break;
+        mbar_arrive_expect_tx(&full[2 + s], kTileBytes + kBlk * 4);
+        bulk_load_1d(sc_sm + (s * 2 + 1) * kBlk, a.vs + (size_t)row, kBlk * 4, &full[2 + s]);
+#pragma unroll
+        for (int bx = 0; bx < kBoxes; ++bx)
+          tma_load_2d(st + kTileBytes + bx * 8192, &tmV, &full[2 + s], bx * 64, row);
         ++it;
       }
       // no copy may still be in flight when the CTA exits
@@ -175,6 +179,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         const int jt = it - 1 - j;
         volatile int dummy = 0;
         mbar_wait(&full[jt & 1], (uint32_t)(jt >> 1) & 1u, &dummy, a.status, 201);
+        mbar_wait(&full[2 + (jt & 1)], (uint32_t)(jt >> 1) & 1u, &dummy, a.status, 203);
       }
     }
     return;
@@ -373,6 +378,14 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
       }
     }
 
+    // K tile consumed: let the producer refill it while the rest of the block runs
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
+    if (!mbar_wait(&full[2 + s], ph, abort_flag, a.status, 211)) {
+      ok = false;
+      break;
+    }
+
     // ---- online softmax (base 2), row rowS ----
     float bm = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
     bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
@@ -414,12 +427,14 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
     // rescale O^T rows tokq, tokq+1: their alphas live in S-layout lanes 4*tokq, 4*(tokq+1)
     const float a0 = __fmul_rn(__shfl_sync(0xffffffffu, alpha, 4 * tokq), escale);
     const float a1 = __fmul_rn(__shfl_sync(0xffffffffu, alpha, 4 * (tokq + 1)), escale);
+    if (!__all_sync(0xffffffffu, a0 == 1.0f && a1 == 1.0f)) {
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt) {
       om[dt][0] = __fmul_rn(om[dt][0], a0);
       om[dt][1] = __fmul_rn(om[dt][1], a1);
       om[dt][2] = __fmul_rn(om[dt][2], a0);
       om[dt][3] = __fmul_rn(om[dt][3], a1);
+    }
     }
 
     // ---- P' = P * s_v * 2^E as FP16 (P_hi, r = P' - P_hi): B fragments of PV ----
@@ -462,7 +477,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
       mma16816(om[dt], l0, l1, l2, l3, pr_[0], pr_[1]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
+    if (lane == 0) mbar_arrive(&empty[2 + s]);
   }
   if (!ok) return;   // a wait gave up: the status word is set; leave without a partial
   if (cur_p >= 0) finalize(cur_p);
@@ -496,7 +511,7 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
 template <int D>
 constexpr int attn_smem_bytes() {
   return 2 * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + (D / 16) * 32 * 16 + 2 * 2 * kBlk * 4 +
-         64 + 1024;
+         96 + 1024;
 }
 
 }  // namespace
@@ -538,20 +553,28 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   a.causal = causal;
   a.scale = scale;
   a.total = (long long)B * Hkv * a.nblk;
-  // opt in to the large shared-memory carve-out first: the occupancy query depends on it
-  if (cudaFuncSetAttribute(heal_attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           attn_smem_bytes<128>()) != cudaSuccess ||
-      cudaFuncSetAttribute(heal_attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           attn_smem_bytes<64>()) != cudaSuccess)
-    return HEAL_ERR_CUDA;
-  int per_sm = 0;
-  if (D == 128)
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<128>, kAttnThreads,
-                                                  attn_smem_bytes<128>());
-  else
-    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<64>, kAttnThreads,
-                                                  attn_smem_bytes<64>());
-  if (per_sm < 1) per_sm = 1;
+  // once per device: opt in to the large shared-memory carve-out (the occupancy query
+  // depends on it), then ask how many CTAs fit per SM
+  static int per_sm_cache[64][2] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HEAL_ERR_CUDA;
+  const int di = (D == 128) ? 0 : 1;
+  int per_sm = per_sm_cache[dev][di];
+  if (per_sm == 0) {
+    if (cudaFuncSetAttribute(heal_attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn_smem_bytes<128>()) != cudaSuccess ||
+        cudaFuncSetAttribute(heal_attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn_smem_bytes<64>()) != cudaSuccess)
+      return HEAL_ERR_CUDA;
+    if (D == 128)
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<128>, kAttnThreads,
+                                                    attn_smem_bytes<128>());
+    else
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<64>, kAttnThreads,
+                                                    attn_smem_bytes<64>());
+    if (per_sm < 1) per_sm = 1;
+    per_sm_cache[dev][di] = per_sm;
+  }
   long long grid = (long long)sms * per_sm;
   if (grid > kMaxGrid) grid = kMaxGrid;
   if (grid > a.total) grid = a.total;
@@ -571,23 +594,13 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   if (!encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<int16_t*>(v), dims, strides, box, es,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return HEAL_ERR_CUDA;
-  cudaError_t e;
   if (D == 128) {
-    auto kern = heal_attn_decode_kernel<128>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<128>());
-    if (e == cudaSuccess) {
-      kern<<<a.grid, kAttnThreads, attn_smem_bytes<128>(), stream>>>(tk, tv, a);
-      heal_attn_combine_kernel<128><<<B * Hkv * R, 128, 0, stream>>>(a);
-    }
+    heal_attn_decode_kernel<128><<<a.grid, kAttnThreads, attn_smem_bytes<128>(), stream>>>(tk, tv, a);
+    heal_attn_combine_kernel<128><<<B * Hkv * R, 128, 0, stream>>>(a);
   } else {
-    auto kern = heal_attn_decode_kernel<64>;
-    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, attn_smem_bytes<64>());
-    if (e == cudaSuccess) {
-      kern<<<a.grid, kAttnThreads, attn_smem_bytes<64>(), stream>>>(tk, tv, a);
-      heal_attn_combine_kernel<64><<<B * Hkv * R, 64, 0, stream>>>(a);
-    }
+    heal_attn_decode_kernel<64><<<a.grid, kAttnThreads, attn_smem_bytes<64>(), stream>>>(tk, tv, a);
+    heal_attn_combine_kernel<64><<<B * Hkv * R, 64, 0, stream>>>(a);
   }
-  if (e != cudaSuccess) return HEAL_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 

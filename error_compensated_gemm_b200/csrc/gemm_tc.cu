@@ -760,8 +760,15 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& alo, const C
                            const CUtensorMap& blo, const GemmArgs& args, int grid, cudaStream_t stream) {
   auto kern = heal_gemm_kernel<BN, A_MN, B_MN, FMT, CORR_SWAP, A_PRE, B_PRE>;
   const int smem = Cfg<BN>::kSmemBytes;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   kern<<<grid, kThreads, smem, stream>>>(a, alo, b, blo, args);
   return cudaGetLastError();
 }
@@ -777,8 +784,15 @@ template <bool B_MN, int FMT, bool B_PRE>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& blo, const GemmArgs& args,
                         int grid, cudaStream_t stream) {
   auto kern = heal_gemm_pair_kernel<B_MN, FMT, B_PRE>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
+  static bool attr_set[64] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) attr_set[dev] = true;
+  }
   kern<<<grid, kPairThreads, kPairSmemBytes, stream>>>(a, b, blo, args);
   return cudaGetLastError();
 }

@@ -1,0 +1,192 @@
+// glue.cu -- K6: the FP32 decoder glue around the compensated GEMMs and the INT16
+// attention in a Llama-style block (embedding gather, RMSNorm, rotary position
+// embedding, SwiGLU, residual add, greedy argmax).  None of these steps is on the pages;
+// they are the plain FP32 operations of the 8B-class decoder the paper evaluates, kept in
+// FP32 end to end so that no 16-bit store happens at a kernel boundary (the truncation the
+// gist.science technical summary, section 1, identifies as the root cause).
+#include <cuda_runtime.h>
+
+#include <cfloat>
+#include <cstdint>
+
+#include "heal_internal.h"
+#include "heal_ptx.cuh"
+
+namespace heal {
+namespace {
+
+constexpr int kThreads = 256;
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+// out[i, :] = table[ids[i], :]
+__global__ void embed_kernel(const float* __restrict__ table, const int32_t* __restrict__ ids, int n, int H,
+                             int vocab, float* __restrict__ out, unsigned int* status) {
+  const int i = blockIdx.x;
+  const int id = ids[i];
+  if (id < 0 || id >= vocab) {   // invalid id: zero row and flag it (never read out of bounds)
+    if (threadIdx.x == 0 && status) atomicOr(&status[0], kStatusBadInput);
+    for (int j = threadIdx.x; j < H; j += blockDim.x) out[(size_t)i * H + j] = 0.0f;
+    return;
+  }
+  const float* src = table + (size_t)id * H;
+  for (int j = threadIdx.x; j < H; j += blockDim.x) out[(size_t)i * H + j] = src[j];
+}
+
+// y[i, :] = x[i, :] / sqrt(mean(x[i, :]^2) + eps) * w   (sum in a fixed order: per thread,
+// then warp shuffles, then warps in index order)
+__global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ w, int H, float eps,
+                               float* __restrict__ y) {
+  __shared__ float part[kThreads / 32];
+  const int i = blockIdx.x;
+  const float* xr = x + (size_t)i * H;
+  float s = 0.0f;
+  for (int j = threadIdx.x; j < H; j += blockDim.x) s = __fmaf_rn(xr[j], xr[j], s);
+  s = warp_sum(s);
+  if ((threadIdx.x & 31) == 0) part[threadIdx.x >> 5] = s;
+  __syncthreads();
+  float tot = 0.0f;
+  for (int k = 0; k < (int)(blockDim.x >> 5); ++k) tot += part[k];
+  const float r = rsqrtf(tot / (float)H + eps);
+  for (int j = threadIdx.x; j < H; j += blockDim.x) y[(size_t)i * H + j] = xr[j] * r * (w ? w[j] : 1.0f);
+}
+
+// Rotary embedding on [n, heads, D] rows (rotate-half convention): for d < D/2,
+//   (x[d], x[d + D/2]) <- (x[d] c - x[d + D/2] s, x[d + D/2] c + x[d] s)
+// with c = cos_t[pos_i, d], s = sin_t[pos_i, d] from host-made FP32 tables [maxpos, D/2].
+__global__ void rope_kernel(float* __restrict__ x, int n, int heads, int D, long long row_stride,
+                            const int32_t* __restrict__ pos, const float* __restrict__ cos_t,
+                            const float* __restrict__ sin_t) {
+  const int i = blockIdx.x / heads, h = blockIdx.x % heads;
+  float* r = x + (size_t)i * row_stride + (size_t)h * D;
+  const int p = pos[i];
+  const int half = D / 2;
+  for (int d = threadIdx.x; d < half; d += blockDim.x) {
+    const float c = cos_t[(size_t)p * half + d], s = sin_t[(size_t)p * half + d];
+    const float a = r[d], b = r[d + half];
+    r[d] = a * c - b * s;
+    r[d + half] = b * c + a * s;
+  }
+}
+
+// out[i, j] = silu(g[i, j]) * u[i, j] with g = gu[i, j], u = gu[i, F + j]
+__global__ void swiglu_kernel(const float* __restrict__ gu, int n, int F, float* __restrict__ out) {
+  const long long total = (long long)n * F;
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
+       e += (long long)gridDim.x * blockDim.x) {
+    const long long i = e / F, j = e % F;
+    const float g = gu[i * 2 * F + j], u = gu[i * 2 * F + F + j];
+    out[e] = (g / (1.0f + expf(-g))) * u;
+  }
+}
+
+// x += y
+__global__ void add_kernel(float* __restrict__ x, const float* __restrict__ y, long long n) {
+  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
+    x[e] += y[e];
+}
+
+// index of the largest value of each row (lowest index among equal maxima; NaN never wins)
+__global__ void argmax_kernel(const float* __restrict__ x, int rows, int n, int32_t* __restrict__ out) {
+  __shared__ float bv[kThreads];
+  __shared__ int bi[kThreads];
+  const int r = blockIdx.x;
+  const float* xr = x + (size_t)r * n;
+  float best = -FLT_MAX;
+  int idx = 0x7fffffff;
+  for (int j = threadIdx.x; j < n; j += blockDim.x) {
+    const float v = xr[j];
+    if (v > best || (v == best && j < idx)) {
+      best = v;
+      idx = j;
+    }
+  }
+  bv[threadIdx.x] = best;
+  bi[threadIdx.x] = idx;
+  __syncthreads();
+  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
+    if ((int)threadIdx.x < s) {
+      const float v = bv[threadIdx.x + s];
+      const int j = bi[threadIdx.x + s];
+      if (v > bv[threadIdx.x] || (v == bv[threadIdx.x] && j < bi[threadIdx.x])) {
+        bv[threadIdx.x] = v;
+        bi[threadIdx.x] = j;
+      }
+    }
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) out[r] = bi[0] == 0x7fffffff ? 0 : bi[0];
+}
+
+int grid_for(long long n) {
+  const int sms = device_sm_count();
+  long long g = (n + kThreads - 1) / kThreads;
+  const long long cap = (long long)(sms > 0 ? sms : 148) * 8;
+  if (g > cap) g = cap;
+  return (int)(g < 1 ? 1 : g);
+}
+
+heal_status_t done() { return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA; }
+
+}  // namespace
+}  // namespace heal
+
+using namespace heal;
+
+extern "C" {
+
+heal_status_t heal_embedding_gather(const float* table, int vocab, int H, const int32_t* ids, int n, float* out,
+                                    heal_stream_t stream) {
+  if (n < 0 || H <= 0 || vocab <= 0) return HEAL_ERR_INVALID_ARGUMENT;
+  if (n == 0) return HEAL_OK;
+  if (!table || !ids || !out) return HEAL_ERR_INVALID_ARGUMENT;
+  embed_kernel<<<n, kThreads, 0, (cudaStream_t)stream>>>(table, ids, n, H, vocab, out, device_status_ptr());
+  return done();
+}
+
+heal_status_t heal_rmsnorm(const float* x, const float* w, int n, int H, float eps, float* y, heal_stream_t stream) {
+  if (n < 0 || H <= 0 || !(eps >= 0.0f)) return HEAL_ERR_INVALID_ARGUMENT;
+  if (n == 0) return HEAL_OK;
+  if (!x || !y) return HEAL_ERR_INVALID_ARGUMENT;
+  rmsnorm_kernel<<<n, kThreads, 0, (cudaStream_t)stream>>>(x, w, H, eps, y);
+  return done();
+}
+
+heal_status_t heal_rope(float* x, int n, int heads, int D, int64_t row_stride, const int32_t* pos,
+                        const float* cos_t, const float* sin_t, heal_stream_t stream) {
+  if (n < 0 || heads <= 0 || D <= 0 || (D & 1) || row_stride < (int64_t)heads * D) return HEAL_ERR_INVALID_ARGUMENT;
+  if (n == 0) return HEAL_OK;
+  if (!x || !pos || !cos_t || !sin_t) return HEAL_ERR_INVALID_ARGUMENT;
+  rope_kernel<<<n * heads, 64, 0, (cudaStream_t)stream>>>(x, n, heads, D, row_stride, pos, cos_t, sin_t);
+  return done();
+}
+
+heal_status_t heal_swiglu(const float* gate_up, int n, int F, float* out, heal_stream_t stream) {
+  if (n < 0 || F <= 0) return HEAL_ERR_INVALID_ARGUMENT;
+  if (n == 0) return HEAL_OK;
+  if (!gate_up || !out) return HEAL_ERR_INVALID_ARGUMENT;
+  swiglu_kernel<<<grid_for((long long)n * F), kThreads, 0, (cudaStream_t)stream>>>(gate_up, n, F, out);
+  return done();
+}
+
+heal_status_t heal_add(float* x, const float* y, int64_t n, heal_stream_t stream) {
+  if (n < 0) return HEAL_ERR_INVALID_ARGUMENT;
+  if (n == 0) return HEAL_OK;
+  if (!x || !y) return HEAL_ERR_INVALID_ARGUMENT;
+  add_kernel<<<grid_for(n), kThreads, 0, (cudaStream_t)stream>>>(x, y, n);
+  return done();
+}
+
+heal_status_t heal_argmax(const float* x, int rows, int n, int32_t* out, heal_stream_t stream) {
+  if (rows < 0 || n <= 0) return HEAL_ERR_INVALID_ARGUMENT;
+  if (rows == 0) return HEAL_OK;
+  if (!x || !out) return HEAL_ERR_INVALID_ARGUMENT;
+  argmax_kernel<<<rows, kThreads, 0, (cudaStream_t)stream>>>(x, rows, n, out);
+  return done();
+}
+
+}  // extern "C"

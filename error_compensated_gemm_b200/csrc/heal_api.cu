@@ -182,6 +182,7 @@ heal_status_t heal_get_device_status(heal_stream_t stream) {
       return HEAL_ERR_CUDA;
     }
     if (st[0] & kStatusTimeout) return HEAL_ERR_TIMEOUT;
+    if (st[0] & kStatusBadInput) return HEAL_ERR_INVALID_ARGUMENT;
   }
   return HEAL_OK;
 }

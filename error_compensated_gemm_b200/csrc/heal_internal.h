@@ -4,7 +4,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
-#include "../../include/heal.h"
+#include "heal.h"
 
 namespace heal {
 

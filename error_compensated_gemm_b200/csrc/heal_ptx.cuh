@@ -15,6 +15,7 @@ namespace heal {
 // there when a bounded wait runs out; heal_get_device_status() reads and clears it.
 // ---------------------------------------------------------------------------------
 constexpr unsigned int kStatusTimeout = 1u;
+constexpr unsigned int kStatusBadInput = 2u;   // a device-side input was out of range
 // A bounded wait gives up after this many nanoseconds of %globaltimer.
 constexpr unsigned long long kWaitLimitNs = 2000000000ull;
 

@@ -191,9 +191,35 @@ heal_status_t heal_attention_int16_noalloc(const int16_t* q, const float* q_scal
                                            float softmax_scale, int causal, float* out,
                                            int64_t* qk_int_out, heal_stream_t stream);
 
+/* K6. FP32 decoder glue of a Llama-style block (the 8B-class decoder shape the paper's
+ * evaluation uses; gist.science technical summary, Results).  The pages describe none of
+ * these steps; they stay in FP32 so that no 16-bit store happens at a kernel boundary
+ * (technical summary, section 1).  All pointers are device pointers; rows are contiguous.
+ *   heal_embedding_gather: out[i, :] = table[ids[i], :], table [vocab, H].  An id outside
+ *     [0, vocab) gives a zero row and makes heal_get_device_status report
+ *     HEAL_ERR_INVALID_ARGUMENT.
+ *   heal_rmsnorm: y[i, :] = x[i, :] / sqrt(mean(x[i, :]^2) + eps) * w (w nullable = 1).
+ *   heal_rope: in place on x viewed as [n, heads, D] with row stride `row_stride` floats;
+ *     rotate-half pairs (d, d + D/2) by the angle of position pos[i]; cos_t and sin_t are
+ *     FP32 tables [max_pos, D/2] made by the caller.
+ *   heal_swiglu: out[i, j] = silu(gu[i, j]) * gu[i, F + j], gu [n, 2F], out [n, F].
+ *   heal_add: x[e] += y[e] for e < n.
+ *   heal_argmax: out[r] = index of the largest x[r, :] (lowest index on ties), x [rows, n]. */
+heal_status_t heal_embedding_gather(const float* table, int vocab, int H, const int32_t* ids,
+                                    int n, float* out, heal_stream_t stream);
+heal_status_t heal_rmsnorm(const float* x, const float* w, int n, int H, float eps, float* y,
+                           heal_stream_t stream);
+heal_status_t heal_rope(float* x, int n, int heads, int D, int64_t row_stride,
+                        const int32_t* pos, const float* cos_t, const float* sin_t,
+                        heal_stream_t stream);
+heal_status_t heal_swiglu(const float* gate_up, int n, int F, float* out, heal_stream_t stream);
+heal_status_t heal_add(float* x, const float* y, int64_t n, heal_stream_t stream);
+heal_status_t heal_argmax(const float* x, int rows, int n, int32_t* out, heal_stream_t stream);
+
 /* Synchronises `stream`, returns HEAL_ERR_TIMEOUT if any kernel of this library gave up
- * on a bounded wait since the last call (the flag is then cleared), HEAL_ERR_CUDA on a
- * CUDA error, else HEAL_OK.                                                            */
+ * on a bounded wait since the last call, HEAL_ERR_INVALID_ARGUMENT if a kernel met an
+ * invalid device-side input (an out-of-range token id), HEAL_ERR_CUDA on a CUDA error,
+ * else HEAL_OK.  The flags are cleared by the call.                                     */
 heal_status_t heal_get_device_status(heal_stream_t stream);
 
 /* Static English description of a status code.                                         */

@@ -78,3 +78,38 @@ def kv_decode(B=8, T=8192, Hkv=8, Hq=32, D=128, Tq=1, seeds=(2, 3, 4), outlier_f
 
 def rand_int16(shape, seed, lo=-32767, hi=32767):
     return torch.randint(lo, hi + 1, shape, generator=_gen(seed), dtype=torch.int32).to(torch.int16)
+
+
+class DecoderConfig:
+    """Shape of the random-init decoder stack (8B-class Llama-style block by default)."""
+
+    def __init__(self, vocab=128256, hidden=4096, heads=32, kv_heads=8, head_dim=128, ffn=14336, layers=2,
+                 rope_theta=500000.0, eps=1e-5, max_pos=1024):
+        self.vocab, self.hidden, self.heads, self.kv_heads = vocab, hidden, heads, kv_heads
+        self.head_dim, self.ffn, self.layers = head_dim, ffn, layers
+        self.rope_theta, self.eps, self.max_pos = rope_theta, eps, max_pos
+
+    @property
+    def qkv_dim(self):
+        return (self.heads + 2 * self.kv_heads) * self.head_dim
+
+
+def decoder_weights(cfg, seed=10):
+    """FP32 CPU tensors: embedding [vocab, H] ~ N(0,1); per layer wqkv [H, (Hq+2Hkv)D],
+    wo [Hq*D, H], w_gate_up [H, 2F] (gate columns first), w_down [F, H]; lm_head [H, vocab];
+    every linear ~ N(0, 0.02).  RMSNorm weights are 1 and not stored."""
+    H = cfg.hidden
+    w = {"embed": normal((cfg.vocab, H), seed)}
+    for l in range(cfg.layers):
+        s = seed + 1 + 10 * l
+        w[f"wqkv{l}"] = normal((H, cfg.qkv_dim), s, std=0.02)
+        w[f"wo{l}"] = normal((cfg.heads * cfg.head_dim, H), s + 1, std=0.02)
+        w[f"wgu{l}"] = normal((H, 2 * cfg.ffn), s + 2, std=0.02)
+        w[f"wdown{l}"] = normal((cfg.ffn, H), s + 3, std=0.02)
+    w["lm_head"] = normal((H, cfg.vocab), seed + 9, std=0.02)
+    return w
+
+
+def prompt_ids(n, vocab, seed=5):
+    """Uniform random token ids (int32)."""
+    return torch.randint(0, vocab, (n,), generator=_gen(seed), dtype=torch.int32)
