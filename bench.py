@@ -187,6 +187,38 @@ class Workload:
     LAUNCHES_PER_STEP = 1 + 2 * len(DECODE_M) + 3 + 2
 
 
+def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=128):
+    """2-layer random-init decoder (hidden 4096, 32q/8kv heads, FFN 14336, vocab 128256):
+    time of the 512-token prefill and per greedy decode step, and a bitwise repeat check."""
+    from error_compensated_gemm_b200.decoder import Decoder
+    cfg = synthetic.DecoderConfig(max_pos=prompt_len + steps + 64)
+    w = synthetic.decoder_weights(cfg)
+    prompt = synthetic.prompt_ids(prompt_len, cfg.vocab).to(dev)
+    dec = Decoder(cfg, w, dev, max_len=prompt_len + steps + 64)
+    del w
+    t_ref, _ = dec.generate(prompt, 8)                      # warm-up
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+    tok = torch.empty(steps, dtype=torch.int32, device=dev)
+    torch.cuda.synchronize()
+    dec.pos_len = 0
+    ev[0].record(stream)
+    logits = dec.forward(prompt)
+    ev[1].record(stream)
+    for s in range(steps):
+        heal.heal_argmax(logits, tok[s:s + 1].view(1))
+        if s + 1 < steps:
+            logits = dec.forward(tok[s:s + 1])
+    ev[2].record(stream)
+    torch.cuda.synchronize()
+    t_again, _ = dec.generate(prompt, steps)
+    torch.cuda.synchronize()
+    pre = ev[0].elapsed_time(ev[1])
+    per = ev[1].elapsed_time(ev[2]) / steps
+    return {"prefill_ms": pre, "decode_ms_per_token": per, "decode_tokens_per_s": 1e3 / per,
+            "prompt": prompt_len, "steps": steps, "bitwise_repeat": bool(torch.equal(tok, t_again)),
+            "note": "decode steps are launched from Python one kernel at a time (host-bound)"}
+
+
 def cpu_baseline_oracle(rows=4096):
     """The oracle's compensated GEMM (split + three FP64 products) on the prefill workload,
     restricted to `rows` rows of X; returns (TFLOP/s effective, seconds, threads)."""
@@ -265,6 +297,7 @@ def main():
                     help="profiling case: run only this part of the step")
     ap.add_argument("--prefill-shape", default=None, help="M,N,K of the prefill GEMM (profiling case)")
     ap.add_argument("--kv-batch", type=int, default=None, help="batch of the KV workload (profiling case)")
+    ap.add_argument("--no-decoder", action="store_true", help="skip the 2-layer decoder measurement")
     args = ap.parse_args()
     if args.prefill_shape:
         global PREFILL
@@ -277,6 +310,7 @@ def main():
     import torch
     import error_compensated_gemm_b200 as heal
     import synthetic
+    from error_compensated_gemm_b200.shard import max_over_ranks
     ws, rank, local = dist_setup()
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
@@ -323,11 +357,9 @@ def main():
     total_ms = t_start.elapsed_time(t_end)
     part_ms = {n: sum(e[n][0].elapsed_time(e[n][1]) for e in evs) for n in names}
     if ws > 1:
-        import torch.distributed as dist
-        t = torch.tensor([total_ms] + [part_ms[n] for n in names], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms = float(t[0])
-        part_ms = {n: float(t[1 + i]) for i, n in enumerate(names)}
+        vals = max_over_ranks([total_ms] + [part_ms[n] for n in names], device=dev)
+        total_ms = vals[0]
+        part_ms = {n: vals[1 + i] for i, n in enumerate(names)}
 
     u = Workload.units()
     K = args.steps
@@ -374,10 +406,7 @@ def main():
         torch.cuda.synchronize()
         e2e_s = e0.elapsed_time(e1) / 1e3 / reps
         if ws > 1:
-            import torch.distributed as dist
-            t = torch.tensor([e2e_s], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            e2e_s = float(t[0])
+            e2e_s = max_over_ranks([e2e_s], device=dev)[0]
         e2e = {"value": ws * u["prefill_flop_eff"] / e2e_s / 1e12, "unit": "TFLOP/s",
                "h2d_bytes_per_step": int(4 * (M_ * K_ + K_ * N_)), "d2h_bytes_per_step": int(4 * M_ * N_)}
         del dX, dW, dC
@@ -389,6 +418,13 @@ def main():
         tf, secs, thr = cpu_baseline_oracle()
         cpu = {"value": tf, "unit": "TFLOP/s", "cores": thr, "kind": "oracle",
                "sample": f"full prefill workload (4096 rows), one run of FP64 split + three FP64 products, {secs:.1f} s"}
+
+    dec_res = None
+    if not args.no_decoder:
+        dec_res = decoder_section(torch, heal, synthetic, dev, stream)
+        if ws > 1:
+            dec_res["prefill_ms"], dec_res["decode_ms_per_token"] = max_over_ranks(
+                [dec_res["prefill_ms"], dec_res["decode_ms_per_token"]], device=dev)
 
     traffic = None
     prof = os.path.join(ROOT, "profiles", "traffic.json")
@@ -420,6 +456,7 @@ def main():
             "secondary": {"kv_writer_gbs": kvw_gbs, "kv_writer_frac_hbm": kvw_gbs / hbm, "decode_gemm": dec,
                           "ms_per_step_parts": {n: part_ms[n] / K for n in names},
                           "hbm_peak_gbs": hbm, "peak_source": peak_src},
+            "decoder": dec_res,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": Workload.LAUNCHES_PER_STEP * K,

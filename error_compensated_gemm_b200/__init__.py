@@ -12,6 +12,7 @@ from ._binding import (  # noqa: F401
     SPLIT_BF16, SPLIT_FP16_S11, TILE_128x128, TILE_256x256_PAIR, TILE_AUTO, TILE_SKINNY_SPLITK, GemmOpts, HealError,
     gemm_opts, heal_attention_int16, heal_attention_int16_noalloc, heal_attention_workspace_bytes, heal_gemm_compensated,
     heal_gemm_workspace_bytes, heal_get_device_status, heal_kv_quantize_int16, heal_split, heal_version, lib,
-    status_string, heal_embedding_gather, heal_rmsnorm, heal_rope, heal_swiglu, heal_add, heal_argmax)
+    status_string, heal_embedding_gather, heal_rmsnorm, heal_rope, heal_swiglu, heal_add, heal_argmax,
+    heal_probe_wait_timeout)
 
 __version__ = "0.1.0"

@@ -15,7 +15,7 @@ TILE_AUTO, TILE_128x128, TILE_256x256_PAIR, TILE_SKINNY_SPLITK = -1, 0, 1, 2
 EXPORTED = ("heal_split", "heal_gemm_compensated", "heal_gemm_workspace_bytes", "heal_kv_quantize_int16",
             "heal_attention_int16", "heal_attention_workspace_bytes", "heal_get_device_status",
             "heal_status_string", "heal_version", "heal_attention_int16_noalloc", "heal_embedding_gather",
-            "heal_rmsnorm", "heal_rope", "heal_swiglu", "heal_add", "heal_argmax")
+            "heal_rmsnorm", "heal_rope", "heal_swiglu", "heal_add", "heal_argmax", "heal_probe_wait_timeout")
 
 
 class HealError(RuntimeError):
@@ -54,6 +54,7 @@ def lib():
         "heal_attention_int16_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _f, _i, _vp,
                                           _vp, _vp], _i),
         "heal_get_device_status": ([_vp], _i),
+        "heal_probe_wait_timeout": ([_i, _vp], _i),
         "heal_embedding_gather": ([_vp, _i, _i, _vp, _i, _vp, _vp], _i),
         "heal_rmsnorm": ([_vp, _vp, _i, _i, _f, _vp, _vp], _i),
         "heal_rope": ([_vp, _i, _i, _i, _i64, _vp, _vp, _vp, _vp], _i),
@@ -238,6 +239,10 @@ def heal_argmax(x, out, stream=None):
     _cuda(x, out)
     rows, n = x.shape
     _check(lib().heal_argmax(_ptr(x), rows, n, _ptr(out), _stream(stream)), "heal_argmax")
+
+
+def heal_probe_wait_timeout(limit_ms=200, stream=None):
+    _check(lib().heal_probe_wait_timeout(int(limit_ms), _stream(stream)), "heal_probe_wait_timeout")
 
 
 def heal_get_device_status(stream=None):

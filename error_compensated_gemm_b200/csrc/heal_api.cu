@@ -63,6 +63,20 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, cuuint32_t rank
 
 static inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
+// One warp waits, through the same bounded wait every kernel uses, on an mbarrier that
+// nothing arrives on; the wait gives up after limit_ns and records a timeout.
+__global__ void heal_wait_probe_kernel(unsigned int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  mbar_wait(&bar, 0u, &abort_flag, status, 900, limit_ns);
+}
+
 }  // namespace heal
 
 using namespace heal;
@@ -184,6 +198,15 @@ heal_status_t heal_get_device_status(heal_stream_t stream) {
     if (st[0] & kStatusTimeout) return HEAL_ERR_TIMEOUT;
     if (st[0] & kStatusBadInput) return HEAL_ERR_INVALID_ARGUMENT;
   }
+  return HEAL_OK;
+}
+
+heal_status_t heal_probe_wait_timeout(int limit_ms, heal_stream_t stream) {
+  if (limit_ms < 1 || limit_ms > 10000) return HEAL_ERR_INVALID_ARGUMENT;
+  unsigned int* st = device_status_ptr();
+  if (!st) return HEAL_ERR_CUDA;
+  heal_wait_probe_kernel<<<1, 32, 0, (cudaStream_t)stream>>>(st, (unsigned long long)limit_ms * 1000000ull);
+  if (cudaGetLastError() != cudaSuccess) return HEAL_ERR_CUDA;
   return HEAL_OK;
 }
 

@@ -222,6 +222,13 @@ heal_status_t heal_argmax(const float* x, int rows, int n, int32_t* out, heal_st
  * else HEAL_OK.  The flags are cleared by the call.                                     */
 heal_status_t heal_get_device_status(heal_stream_t stream);
 
+/* Failure-detection check: launches one warp that waits, with the same bounded wait as
+ * every kernel of the library, on an mbarrier that nothing arrives on.  After limit_ms
+ * (1 .. 10000) the wait gives up, the device status records a timeout and the kernel
+ * returns; heal_get_device_status() then reports HEAL_ERR_TIMEOUT and the CUDA context
+ * stays usable.  Nothing faults, traps or hangs.                                        */
+heal_status_t heal_probe_wait_timeout(int limit_ms, heal_stream_t stream);
+
 /* Static English description of a status code.                                         */
 const char* heal_status_string(heal_status_t status);
 
