@@ -133,6 +133,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
   const long long u0 = unit_begin(a.total, a.grid, c), u1 = unit_begin(a.total, a.grid, c + 1);
+  pdl_launch_dependents();   // the combine kernel may be scheduled; it waits for us
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < 4; ++s) {
@@ -486,6 +487,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
 // out[b, hq, tq, :] = sum_c o_c 2^(m_c - M) / sum_c l_c 2^(m_c - M), c ascending.
 template <int D>
 __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) {
+  pdl_wait_prerequisites();             // the decode kernel that wrote the partials has completed
   const int pr = blockIdx.x;            // (pair, row)
   const int p = pr / a.R, r = pr % a.R;
   const int d = threadIdx.x;
@@ -594,13 +596,15 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   if (!encode_tensor_map(&tv, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, const_cast<int16_t*>(v), dims, strides, box, es,
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return HEAL_ERR_CUDA;
+  cudaError_t e;
   if (D == 128) {
     heal_attn_decode_kernel<128><<<a.grid, kAttnThreads, attn_smem_bytes<128>(), stream>>>(tk, tv, a);
-    heal_attn_combine_kernel<128><<<B * Hkv * R, 128, 0, stream>>>(a);
+    e = launch_pdl(heal_attn_combine_kernel<128>, dim3(B * Hkv * R), dim3(128), 0, stream, a);
   } else {
     heal_attn_decode_kernel<64><<<a.grid, kAttnThreads, attn_smem_bytes<64>(), stream>>>(tk, tv, a);
-    heal_attn_combine_kernel<64><<<B * Hkv * R, 64, 0, stream>>>(a);
+    e = launch_pdl(heal_attn_combine_kernel<64>, dim3(B * Hkv * R), dim3(64), 0, stream, a);
   }
+  if (e != cudaSuccess) return HEAL_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 

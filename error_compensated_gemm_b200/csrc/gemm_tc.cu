@@ -60,7 +60,7 @@ struct Cfg {
   static constexpr int kABytes = kBM * kBK * 4;             // 32 KB of FP32
   static constexpr int kBBytes = BN * kBK * 4;
   static constexpr int kStageBytes = kABytes + kBBytes;
-  static constexpr int kStages = (200 * 1024) / kStageBytes > 8 ? 8 : (200 * 1024) / kStageBytes;
+  static constexpr int kStages = (216 * 1024) / kStageBytes > 8 ? 8 : (216 * 1024) / kStageBytes;
   static constexpr int kTmemCols = (2 * BN) <= 32 ? 32 : (2 * BN) <= 64 ? 64 : (2 * BN) <= 128 ? 128 : (2 * BN) <= 256 ? 256 : 512;
   static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
   static_assert(kStages >= 2, "at least two stages");
@@ -258,6 +258,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  pdl_launch_dependents();   // a following reduce kernel may be scheduled; it waits for us
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -717,17 +718,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 }
 
 // Ordered sum of chunk values: out(i, j) = ((ws[0] + ws[1]) + ws[2]) + ...
-__global__ void heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk, int Nk, float* out,
-                                         long long si, long long sj) {
-  const long long total = (long long)Mk * Nk;
-  for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
-       e += (long long)gridDim.x * blockDim.x) {
-    const int i = (int)(e % Mk), j = (int)(e / Mk);
-    const float* p = ws + (size_t)j * Mk + i;
-    float acc = p[0];
-    for (int c = 1; c < num_chunks; ++c) acc = __fadd_rn(acc, p[(size_t)c * Mk * Nk]);
-    out[(size_t)i * si + (size_t)j * sj] = acc;
+// One block per 32 consecutive i of one j: the block stages the chunk values of those 32
+// outputs (pieces of up to kRedChunks chunks, coalesced 128-byte rows) in shared memory,
+// then 32 threads add them in ascending chunk order, carrying the sum across pieces.
+constexpr int kRedChunks = 128;
+__global__ void __launch_bounds__(256) heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk,
+                                                                int Nk, float* out, long long si, long long sj) {
+  __shared__ float tile[kRedChunks][33];
+  pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed
+  const int tiles_i = (Mk + 31) / 32;
+  const int ti = blockIdx.x % tiles_i, j = blockIdx.x / tiles_i;
+  const int i0 = ti * 32;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const size_t plane = (size_t)Mk * Nk;
+  const float* base = ws + (size_t)j * Mk + i0;
+  float acc = 0.0f;
+  for (int c0 = 0; c0 < num_chunks; c0 += kRedChunks) {
+    const int cn = min(kRedChunks, num_chunks - c0);
+    __syncthreads();
+    for (int c = warp; c < cn; c += 8)
+      tile[c][lane] = (i0 + lane < Mk) ? __ldcs(base + (size_t)(c0 + c) * plane + lane) : 0.0f;
+    __syncthreads();
+    if (warp == 0) {
+      int c = 0;
+      if (c0 == 0) {
+        acc = tile[0][lane];
+        c = 1;
+      }
+      // 16 values at a time into registers, then added in ascending chunk order
+      for (; c + 16 <= cn; c += 16) {
+        float v[16];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) v[t] = tile[c + t][lane];
+#pragma unroll
+        for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, v[t]);
+      }
+      for (; c < cn; ++c) acc = __fadd_rn(acc, tile[c][lane]);
+    }
   }
+  if (warp == 0 && i0 + lane < Mk) out[(size_t)(i0 + lane) * si + (size_t)j * sj] = acc;
 }
 
 // ---------------------------------------------------------------------------------
@@ -902,16 +931,18 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     return err == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
   }
 
-  if (cfg == HEAL_TILE_SKINNY_SPLITK) {
+  if (cfg == HEAL_TILE_SKINNY_SPLITK || cfg == HEAL_TILE_SKINNY_FULLK) {
+    const bool split = (cfg == HEAL_TILE_SKINNY_SPLITK);
     if (o.b_presplit) return HEAL_ERR_UNSUPPORTED;
     if (M > 64) return HEAL_ERR_UNSUPPORTED;
-    if (o.workspace == nullptr || o.workspace_bytes < gemm_workspace_bytes(M, N, K, cfg)) return HEAL_ERR_INVALID_ARGUMENT;
+    if (split && (o.workspace == nullptr || o.workspace_bytes < gemm_workspace_bytes(M, N, K, cfg)))
+      return HEAL_ERR_INVALID_ARGUMENT;
     // swapped roles: kernel-A = B^T (N rows), kernel-B = A (M rows), C written transposed
     args.Mk = N;
     args.Nk = M;
     args.tiles_m = (N + kBM - 1) / kBM;
     args.tiles_n = 1;
-    args.splitk = 1;
+    args.splitk = split ? 1 : 0;
     args.ws = static_cast<float*>(o.workspace);
     args.out = Cout;
     args.out_si = 1;
@@ -921,7 +952,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     const int BNk = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
     if (!operand_map(&ta, B, b_mn, false, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (!operand_map(&tb, A, false, false, M, K, lda, BNk)) return HEAL_ERR_CUDA;
-    const long long units = (long long)args.tiles_m * nc;
+    const long long units = split ? (long long)args.tiles_m * nc : (long long)args.tiles_m;
     const int grid = (int)(units < sms ? units : sms);
     if (BNk == 16)
       err = b_mn ? launch_fmt<16, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
@@ -933,11 +964,12 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
       err = b_mn ? launch_fmt<64, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
                  : launch_fmt<64, false, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
     if (err != cudaSuccess) return HEAL_ERR_CUDA;
-    const long long total = (long long)M * N;
-    int rgrid = (int)((total + 255) / 256);
-    if (rgrid > 4 * sms) rgrid = 4 * sms;
-    heal_chunk_reduce_kernel<<<rgrid, 256, 0, stream>>>(args.ws, nc, N, M, Cout, 1, ldc);
-    return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+    if (!split) return HEAL_OK;
+    const long long rblocks = (long long)((N + 31) / 32) * M;
+    if (rblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
+    const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(256), 0, stream,
+                                     (const float*)args.ws, nc, N, M, Cout, 1LL, (long long)ldc);
+    return e == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
   }
   return HEAL_ERR_UNSUPPORTED;
 }

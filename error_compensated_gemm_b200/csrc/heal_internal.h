@@ -19,6 +19,24 @@ bool encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dt, cuuint32_t rank
                        const cuuint64_t* dims, const cuuint64_t* strides, const cuuint32_t* box,
                        const cuuint32_t* elem_strides, CUtensorMapSwizzle swizzle);
 
+// Launch `kern` with programmatic stream serialization: it may be scheduled before the
+// previous kernel on `s` finishes and must call griddepcontrol.wait before reading that
+// kernel's results.
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Params>(args)...);
+}
+
 heal_status_t split_launch(const float* x, void* hi, void* lo, long long n, int fmt, cudaStream_t s);
 
 size_t gemm_workspace_bytes(int M, int N, int K, int tile_config);

@@ -298,6 +298,12 @@ __device__ __forceinline__ void mma_f16_pair_scale_d(uint32_t d_tmem, uint64_t a
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(one), "n"(SHIFT));
   }
 }
+// Programmatic dependent launch: let the next kernel on the stream be scheduled now, and
+// (in that kernel) wait until every prerequisite grid has completed and its writes are
+// visible.
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+__device__ __forceinline__ void pdl_wait_prerequisites() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 template <int N>
 __device__ __forceinline__ void setmaxnreg_inc() {
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));

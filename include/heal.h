@@ -59,8 +59,9 @@ enum {
   HEAL_TILE_256x256_PAIR = 1, /* a cluster of 2 CTAs per 256x256 tile (tcgen05 cta_group::2):
                                  each CTA stages and splits 128 rows of A and 128 columns of
                                  B; the default for M, N >= 256                           */
-  HEAL_TILE_SKINNY_SPLITK = 2 /* operands swapped (weights on the MMA M side), K split
-                                 over CTAs; needs a workspace                           */
+  HEAL_TILE_SKINNY_SPLITK = 2, /* operands swapped (weights on the MMA M side), K split
+                                 over CTAs; needs a workspace (M <= 64)                 */
+  HEAL_TILE_SKINNY_FULLK = 3   /* operands swapped, full K per CTA, no workspace (M <= 64) */
 };
 
 typedef struct {

@@ -70,8 +70,10 @@ def test_tile_configs_bitwise_identical(M, b_layout):
     Bin = W if b_layout == 0 else np.ascontiguousarray(W.T)
     c_full = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_128x128)
     c_skinny = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_SKINNY_SPLITK)
+    c_fullk = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_SKINNY_FULLK)
     c_pair = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_256x256_PAIR)
     assert np.array_equal(c_full, c_skinny)
+    assert np.array_equal(c_full, c_fullk)
     assert np.array_equal(c_full, c_pair)
     assert G.normwise_rel_err(c_full, G.gemm_ref(X, W)) <= TOL_FP16
 
