@@ -352,6 +352,16 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         }
       }
     }
+    // every ldmatrix of the K tile has been consumed by the MMAs above and the K scales
+    // this lane needs are copied to registers: release the K half now, before the logit
+    // arithmetic, so the producer can refill it sooner
+    float skr[2][2];
+#pragma unroll
+    for (int nb = 0; nb < 2; ++nb)
+#pragma unroll
+      for (int e = 0; e < 2; ++e) skr[nb][e] = sks[tw + nb * 8 + tokq + e];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&empty[s]);
 #pragma unroll
     for (int nb = 0; nb < 2; ++nb) {
 #pragma unroll
@@ -367,7 +377,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         } else if (!vis) {
           xv = -INFINITY;
         } else {
-          const double coef = (double)sq * (double)sks[t - t0];
+          const double coef = (double)sq * (double)skr[nb][e];
           const float lg = (float)(((double)S * coef) * (double)a.scale);
           xv = __fmul_rn(lg, kLog2e);
           if (a.qk_out) {
@@ -379,9 +389,6 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
       }
     }
 
-    // K tile consumed: let the producer refill it while the rest of the block runs
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
     if (!mbar_wait(&full[2 + s], ph, abort_flag, a.status, 211)) {
       ok = false;
       break;
