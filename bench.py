@@ -124,8 +124,14 @@ class Workload:
         if need("decode"):
             for i, m in enumerate(DECODE_M):
                 Xd, Wd = synthetic.gemm_decode(m, seed_x=0 + so, seed_w=1 + so + 10 * (i + 1))
-                ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(m, 4096, 4096) // 4), device=dev)
-                self.dec.append((m, Xd.to(dev), Wd.to(dev), torch.empty(m, 4096, device=dev), ws))
+                ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(m, 4096, 4096, heal.TILE_SKINNY_SPLITK) // 4),
+                                 device=dev)
+                Wd = Wd.to(dev)
+                # the same weights split once (as a deployment would at load time): hi / lo
+                whi = torch.empty(Wd.shape, dtype=torch.int16, device=dev)
+                wlo = torch.empty(Wd.shape, dtype=torch.int16, device=dev)
+                heal.heal_split(Wd, whi, wlo)
+                self.dec.append((m, Xd.to(dev), Wd, torch.empty(m, 4096, device=dev), ws, whi, wlo))
         if need("kv_writer"):
             B, T, Hkv, Hq, D = KV["B"], KV["T"], KV["Hkv"], KV["Hq"], KV["D"]
             Qb, Kb, Vb = synthetic.kv_decode(B=B, T=T, Hkv=Hkv, Hq=Hq, D=D, seeds=(2 + so, 3 + so, 4 + so))
@@ -163,9 +169,12 @@ class Workload:
         if only in (None, "prefill"):
             out.append(("prefill", lambda: h.heal_gemm_compensated(self.X, self.W, self.C)))
         if only in (None, "decode"):
-            for (m, Xd, Wd, Cd, ws) in self.dec:
+            for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
                 out.append((f"decode{m}", lambda Xd=Xd, Wd=Wd, Cd=Cd, ws=ws: h.heal_gemm_compensated(
                     Xd, Wd, Cd, workspace=ws)))
+            for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
+                out.append((f"decode{m}_presplit", lambda Xd=Xd, whi=whi, wlo=wlo, Cd=Cd, ws=ws:
+                            h.heal_gemm_compensated(Xd, whi, Cd, b_lo=wlo, workspace=ws)))
         if only in (None, "kv_writer", "attention"):
             out.append(("kv_writer", lambda: (h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs),
                                               h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks),
@@ -209,10 +218,14 @@ class Workload:
             h.heal_gemm_compensated(self.X, self.W, self.C)
             rec("prefill", 1)
         if only in (None, "decode"):
-            for (m, Xd, Wd, Cd, ws) in self.dec:
+            for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
                 rec(f"decode{m}", 0)
                 h.heal_gemm_compensated(Xd, Wd, Cd, workspace=ws)
                 rec(f"decode{m}", 1)
+            for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
+                rec(f"decode{m}_presplit", 0)
+                h.heal_gemm_compensated(Xd, whi, Cd, b_lo=wlo, workspace=ws)
+                rec(f"decode{m}_presplit", 1)
         if only in (None, "kv_writer", "attention"):
             rec("kv_writer", 0)
             h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs)
@@ -225,7 +238,7 @@ class Workload:
                                    KV["D"] ** -0.5, self.out, self.aws)
             rec("attention", 1)
 
-    LAUNCHES_PER_STEP = 1 + 2 * len(DECODE_M) + 3 + 2
+    LAUNCHES_PER_STEP = 1 + 2 * 2 * len(DECODE_M) + 3 + 2
 
 
 def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=128):
@@ -371,9 +384,10 @@ def main():
     if st != heal.HEAL_OK:
         raise SystemExit(f"device status after warm-up: {heal.status_string(st)}")
 
-    names = ["prefill"] + [f"decode{m}" for m in DECODE_M] + ["kv_writer", "attention"]
+    dec_names = [f"decode{m}" for m in DECODE_M] + [f"decode{m}_presplit" for m in DECODE_M]
+    names = ["prefill"] + dec_names + ["kv_writer", "attention"]
     if args.only:
-        keep = {"prefill": ["prefill"], "decode": [f"decode{m}" for m in DECODE_M],
+        keep = {"prefill": ["prefill"], "decode": dec_names,
                 "kv_writer": ["kv_writer"], "attention": ["kv_writer", "attention"]}[args.only]
         names = keep
     evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
@@ -423,10 +437,12 @@ def main():
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     attn_gbs = u["attn_bytes"] / (part_ms["attention"] / 1e3 / K) / 1e9
     kvw_gbs = u["kv_writer_bytes"] / (part_ms["kv_writer"] / 1e3 / K) / 1e9
-    dec = {f"M{m}": {"gbs": u["decode_bytes"][m] / (part_ms[f"decode{m}"] / 1e3 / K) / 1e9,
-                     "us": 1e3 * part_ms[f"decode{m}"] / K} for m in DECODE_M}
+    dec = {}
     for m in DECODE_M:
-        dec[f"M{m}"]["frac_hbm"] = dec[f"M{m}"]["gbs"] / hbm
+        for suffix, key in (("", f"M{m}"), ("_presplit", f"M{m}_presplit_weights")):
+            t = part_ms[f"decode{m}{suffix}"] / 1e3 / K
+            dec[key] = {"gbs": u["decode_bytes"][m] / t / 1e9, "us": 1e6 * t,
+                        "frac_hbm": u["decode_bytes"][m] / t / 1e9 / hbm}
 
     # end to end through the public API: pinned host inputs -> device -> GEMM -> host result
     M_, K_, N_ = PREFILL
@@ -496,7 +512,7 @@ def main():
             "pct_of_16bit_peak": 100.0 * mma_tflops / peak_sus,
             "roofline": {"bound": "tensor", "achieved": mma_tflops, "peak": peak_sus, "unit": "TFLOP/s",
                          "frac": mma_tflops / peak_sus, "traffic": traffic,
-                         "kernel": "heal_gemm_kernel (prefill)", "peak_source": f"bf16_tflops_sustained, {peak_src}",
+                         "kernel": "heal_gemm_pair_kernel (prefill, 256x256 CTA pair)", "peak_source": f"bf16_tflops_sustained, {peak_src}",
                          "frac_of_burst_peak": mma_tflops / peak_burst},
             "attn_gbs": attn_gbs, "attn_frac_hbm": attn_gbs / hbm,
             "secondary": {"kv_writer_gbs": kvw_gbs, "kv_writer_frac_hbm": kvw_gbs / hbm, "decode_gemm": dec,

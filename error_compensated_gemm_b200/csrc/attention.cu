@@ -3,26 +3,29 @@
 // attention contractions).
 //
 // Unpacking used here: q = 256*hi + lo with hi = q >> 8 in [-128, 127] and lo = q & 255
-// in [0, 255]; both are exact FP16 values.  Then, per (query row, token),
+// in [0, 255].  Then, per (query row, token),
 //     S_int = sum_d q_d k_d = 65536*S_hh + 256*S_x + S_ll
-// with S_hh = sum qh*kh, S_x = sum (qh*kl + ql*kh), S_ll = sum ql*kl.  For head_dim <= 128
-// every partial sum of every term is an integer below 2^24 in magnitude, so the FP16 tensor
-// core products accumulate exactly in FP32; the three sums are combined in int64.
+// with S_hh = sum qh*kh, S_x = sum (qh*kl + ql*kh), S_ll = sum ql*kl.  QK^T runs these four
+// byte products on the integer tensor cores (mma.sync m16n8k32, signed hi bytes and
+// unsigned lo bytes, exact int32 accumulation: for head_dim <= 128 no partial sum exceeds
+// 2^24); the three sums are combined in int64.
 //   logit = fp32( (double(S_int) * (double(s_q) * double(s_k))) * double(softmax_scale) )
 // FP32 online softmax in base 2.  P is folded with the per-token V scale and a per-block
 // power of two 2^E (chosen so the block's largest V scale times 2^E lies in [32, 64)),
 // then split into FP16 P_hi and the FP16 residual r = P - P_hi; the byte-split V
-// (hi = v >> 8, lo = v & 255) meets (256*P_hi, P_hi, 256*r, r) in four FP16 tensor-core
-// products that accumulate into one FP32 accumulator: sum 256*hi*P + lo*P = v*P.
+// (hi = v >> 8, lo = v & 255, each an exact FP16 value) meets (256*P_hi, P_hi, 256*r, r) in
+// four FP16 tensor-core products that accumulate into one FP32 accumulator:
+// sum 256*hi*P + lo*P = v*P.  These are the two FP16 tensors the INT16 value is unpacked
+// into for the floating-point contraction.
 //
 // Work decomposition: a persistent grid; CTA c owns the contiguous slice
 // [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token block)
 // units.  Warp 4 streams 64-token K and V tiles with TMA (128-byte swizzle) into a
-// two-stage ring (the K half of a stage is released after QK^T, the V half after PV); warps 0-3 each take 16 tokens of a tile with mma.sync m16n8k16 (the
-// decode GEMV shapes are far below a tcgen05 tile; the kernel is HBM-bound).  Every
-// (CTA, kv head) segment leaves one partial (m, l, o) in the workspace; the combine kernel
-// merges them in ascending token order.  The order is fixed, so results are identical
-// from run to run.
+// two-stage ring (the K half of a stage is released after QK^T, the V half after PV);
+// warps 0-3 each take 16 tokens of a tile with mma.sync (the decode GEMV shapes are far
+// below a tcgen05 tile; the kernel is HBM-bound).  Every (CTA, kv head) segment leaves one
+// partial (m, l, o) in the workspace; the combine kernel merges them in ascending token
+// order.  The order is fixed, so results are identical from run to run.
 #include <cuda_fp16.h>
 
 #include <cmath>
@@ -35,6 +38,11 @@ namespace heal {
 namespace {
 
 constexpr int kBlk = 64;          // tokens per pipeline stage
+// K/V stages per CTA.  Two stages leave room for three CTAs (15 warps) per SM; on the
+// 8 x 8192 x 8 x 128 decode cache three stages (two CTAs per SM) measured 9% slower and
+// four or six (one CTA per SM) 44% slower: warps per SM matter more than ring depth here.
+constexpr int kStages = 2;
+constexpr int kMinBlocks = kStages <= 2 ? 3 : (kStages == 3 ? 2 : 1);   // CTAs per SM the ring allows
 constexpr int kCompute = 4;       // compute warps, 16 tokens each per stage
 constexpr int kAttnThreads = (kCompute + 1) * 32;
 constexpr int kRows = 8;          // query rows per CTA: (Hq/Hkv) * Tq <= 8
@@ -70,6 +78,33 @@ __device__ __forceinline__ uint32_t hi_pair(uint32_t x) {
   const uint32_t u = ((x >> 8) & 0x00FF00FFu) ^ 0x64806480u;
   const __half2 h = __hsub2(*reinterpret_cast<const __half2*>(&u), __half2half2(__ushort_as_half(0x6480)));
   return *reinterpret_cast<const uint32_t*>(&h);   // 0x6480 = 1152 = 1024 + 128
+}
+
+// Bytes of two registers holding int16 pairs (x = (v0, v1), y = (v2, v3)):
+// lo_bytes -> (v0 & 255, v1 & 255, v2 & 255, v3 & 255) as u8; hi_bytes -> their high bytes (s8).
+__device__ __forceinline__ uint32_t lo_bytes(uint32_t x, uint32_t y) { return __byte_perm(x, y, 0x6420); }
+__device__ __forceinline__ uint32_t hi_bytes(uint32_t x, uint32_t y) { return __byte_perm(x, y, 0x7531); }
+
+// Exact integer MMA m16n8k32, s32 accumulate; A_U / B_U: the operand holds unsigned bytes.
+template <bool A_U, bool B_U>
+__device__ __forceinline__ void imma16832(int (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                          uint32_t b0, uint32_t b1) {
+  if constexpr (!A_U && !B_U)
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else if constexpr (!A_U && B_U)
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else if constexpr (A_U && !B_U)
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  else
+    asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+                 : "+r"(c[0]), "+r"(c[1]), "+r"(c[2]), "+r"(c[3])
+                 : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
 }
 
 __device__ __forceinline__ void mma16816(float (&c)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
@@ -112,23 +147,23 @@ __device__ __forceinline__ float* slot_ptr(float* ws, int c, int p, int R, int D
 }
 
 template <int D>
-__global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
+__global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                        const __grid_constant__ CUtensorMap tmV,
                                                                        const AttnArgs a) {
   constexpr int kBoxes = D / 64;                    // 64-dim (128-byte) boxes per row
   constexpr int kTileBytes = kBlk * D * 2;          // one of K / V
   constexpr int kStageBytes = 2 * kTileBytes;
-  constexpr int kKSteps = D / 16;
+  constexpr int kKSteps32 = D / 32;                 // k32 steps of the integer MMA
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint8_t* stages = smem;                                            // 2 x kStageBytes
-  float* o_sm = reinterpret_cast<float*>(smem + 2 * kStageBytes);    // [kRows][D]
+  uint8_t* stages = smem;                                                  // kStages x kStageBytes
+  float* o_sm = reinterpret_cast<float*>(smem + kStages * kStageBytes);    // [kRows][D]
   float* ml_sm = o_sm + kRows * D;                                   // [kCompute][kRows][2]
-  uint4* qf_sm = reinterpret_cast<uint4*>(ml_sm + kCompute * kRows * 2); // [kKSteps][32 lanes]
-  float* sc_sm = reinterpret_cast<float*>(qf_sm + kKSteps * 32);        // [2 stages][K, V][kBlk]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sc_sm + 2 * 2 * kBlk);  // [2] K tile, [2] V tile + scales
-  uint64_t* empty = full + 4;                                          // [2] K released, [2] V released
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 4);
+  uint4* qf_sm = reinterpret_cast<uint4*>(ml_sm + kCompute * kRows * 2); // [kKSteps32][32 lanes]
+  float* sc_sm = reinterpret_cast<float*>(qf_sm + kKSteps32 * 32);      // [kStages][K, V][kBlk]
+  uint64_t* full = reinterpret_cast<uint64_t*>(sc_sm + kStages * 2 * kBlk);  // [S] K tile, [S] V tile + scales
+  uint64_t* empty = full + 2 * kStages;                                // [S] K released, [S] V released
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 2 * kStages);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
@@ -136,7 +171,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
   pdl_launch_dependents();   // the combine kernel may be scheduled; it waits for us
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 4; ++s) {
+    for (int s = 0; s < 2 * kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], kCompute);
     }
@@ -156,8 +191,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         const int b = p / a.Hkv;
         const int t0 = blk * kBlk;
         if (t0 >= __ldg(a.kv_len + b)) continue;
-        const int s = it & 1;
-        const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+        const int s = it % kStages;
+        const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         uint8_t* st = stages + s * kStageBytes;
         const int row = p * a.Tmax + t0;
         // K half: refilled as soon as the compute warps finish QK^T on the previous tile
@@ -167,32 +202,40 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx) tma_load_2d(st + bx * 8192, &tmK, &full[s], bx * 64, row);
         // V half and V scales
-        if (!mbar_wait(&empty[2 + s], ph ^ 1u, abort_flag, a.status, 202)) break;
-        mbar_arrive_expect_tx(&full[2 + s], kTileBytes + kBlk * 4);
-        bulk_load_1d(sc_sm + (s * 2 + 1) * kBlk, a.vs + (size_t)row, kBlk * 4, &full[2 + s]);
+        if (!mbar_wait(&empty[kStages + s], ph ^ 1u, abort_flag, a.status, 202)) break;
+        mbar_arrive_expect_tx(&full[kStages + s], kTileBytes + kBlk * 4);
+        bulk_load_1d(sc_sm + (s * 2 + 1) * kBlk, a.vs + (size_t)row, kBlk * 4, &full[kStages + s]);
 #pragma unroll
         for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_2d(st + kTileBytes + bx * 8192, &tmV, &full[2 + s], bx * 64, row);
+          tma_load_2d(st + kTileBytes + bx * 8192, &tmV, &full[kStages + s], bx * 64, row);
         ++it;
       }
       // no copy may still be in flight when the CTA exits
-      for (int j = 0; j < 2 && j < it; ++j) {
+      for (int j = 0; j < kStages && j < it; ++j) {
         const int jt = it - 1 - j;
         volatile int dummy = 0;
-        mbar_wait(&full[jt & 1], (uint32_t)(jt >> 1) & 1u, &dummy, a.status, 201);
-        mbar_wait(&full[2 + (jt & 1)], (uint32_t)(jt >> 1) & 1u, &dummy, a.status, 203);
+        mbar_wait(&full[jt % kStages], (uint32_t)(jt / kStages) & 1u, &dummy, a.status, 201);
+        mbar_wait(&full[kStages + jt % kStages], (uint32_t)(jt / kStages) & 1u, &dummy, a.status, 203);
       }
     }
     return;
   }
 
   // ------------------------------- compute warps -------------------------------
+  // Fragment layouts (mma.sync, g = lane / 4, c = lane % 4):
+  //   S^T = K Q^T with m16n8k32 integer MMAs: rows = this warp's 16 tokens, columns = the
+  //   8 query rows.  C fragment of this lane: tokens g and g + 8, query rows 2c and 2c + 1.
+  //   O^T = V^T P'^T with m16n8k16 FP16 MMAs: rows = 16 dims, columns = query rows; the
+  //   lane holds dims g, g + 8 of query rows 2c, 2c + 1 (the same query rows as S^T).
+  // Byte order inside the K dimension of the integer MMA: slot 4c + j of a 16-slot half
+  // holds dim {2c, 2c + 1, 2c + 8, 2c + 9}[j] of that half; both operands use this order,
+  // and a dot product does not depend on the order of its terms.
   const int R = a.R;
-  const int rowS = lane >> 2;                 // S layout: query row of c0/c1
-  const int tokq = 2 * (lane & 3);            // S layout: first token (of 8) of c0/c1
-  float sq = 0.0f;
-  int pos = 0;
-  float m_run = -INFINITY, l_run = 0.0f;      // S layout, row rowS
+  const int g8 = lane >> 2;                   // token row (S^T) / dim row (O^T) / query of B fragments
+  const int qc = 2 * (lane & 3);              // this lane's query rows qc, qc + 1
+  float sq[2] = {0.0f, 0.0f};
+  int pos[2] = {0, 0};
+  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};   // query rows qc + e
   float om[D / 16][4];                        // O^T accumulator (units of 2^E_run)
   int E_run = 0;                              // power of two folded into P (decreases only)
   bool have_E = false;
@@ -201,24 +244,27 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
   bool ok = true;
 
   auto finalize = [&](int p) {
-    // row sums (S layout) and row maxima for this warp
-    float l = l_run;
-    l += __shfl_xor_sync(0xffffffffu, l, 1);
-    l += __shfl_xor_sync(0xffffffffu, l, 2);
-    if ((lane & 3) == 0) {
-      ml_sm[(warp * kRows + rowS) * 2 + 0] = m_run;
-      ml_sm[(warp * kRows + rowS) * 2 + 1] = l;
+    // per query row: the warp's maximum (replicated over g8) and its sum over all lanes
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      float l = l_run[e];
+      l += __shfl_xor_sync(0xffffffffu, l, 4);
+      l += __shfl_xor_sync(0xffffffffu, l, 8);
+      l += __shfl_xor_sync(0xffffffffu, l, 16);
+      if (g8 == 0) {
+        ml_sm[(warp * kRows + qc + e) * 2 + 0] = m_run[e];
+        ml_sm[(warp * kRows + qc + e) * 2 + 1] = l;
+      }
     }
     compute_bar();
-    // rows of this lane's O^T fragments: r0 = tokq, r1 = tokq + 1
-    float f[2], M[2];
+    // query rows of this lane's O^T fragments: qc, qc + 1
+    float f[2];
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int r = tokq + h;
+      const int r = qc + h;
       float mx = -INFINITY;
       for (int w = 0; w < kCompute; ++w) mx = fmaxf(mx, ml_sm[(w * kRows + r) * 2]);
       const float mw = ml_sm[(warp * kRows + r) * 2];
-      M[h] = mx;
       f[h] = (mw == -INFINITY) ? 0.0f : exp2f(mw - mx);
     }
     // O of this warp, scaled to the CTA max, in true units (x 2^-E_run), in place
@@ -234,8 +280,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         for (int dt = 0; dt < D / 16; ++dt)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int d = dt * 16 + (lane >> 2) + ((e >> 1) << 3);
-            const int r = tokq + (e & 1);
+            const int d = dt * 16 + g8 + ((e >> 1) << 3);
+            const int r = qc + (e & 1);
             float* dst = o_sm + r * D + d;
             const float v = (w == 0) ? om[dt][e] : __fadd_rn(*dst, om[dt][e]);
             if (w < kCompute - 1) {
@@ -261,7 +307,6 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
       sl[2 * r + 1] = L;
     }
     compute_bar();
-    (void)M;
   };
 
   for (long long u = u0; u < u1 && ok; ++u) {
@@ -272,30 +317,40 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
       b = p / a.Hkv;
       hkv = p % a.Hkv;
       klen = __ldg(a.kv_len + b);
-      // query rows of this kv head: row r = tq * G + g  ->  head hkv*G + g, query tq
-      const int r = rowS;
-      const bool real = r < R;
-      const int tq = real ? r / a.G : 0, g = real ? r % a.G : 0;
-      const long long qrow = ((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq);
-      sq = real ? __ldg(a.qs + qrow) : 0.0f;
-      pos = klen - a.Tq + tq;
-      // A fragments of Q (rows 0-7; rows 8-15 are zero), byte-split, one table per CTA:
-      // entry [ks][lane] = (hi dims 2t.., hi dims 2t+8.., lo dims 2t.., lo dims 2t+8..)
-      if (warp == 0) {
+      // query row r = tq * G + g of this kv head  ->  head hkv*G + g, query tq
 #pragma unroll
-        for (int ks = 0; ks < kKSteps; ++ks) {
-          uint32_t w0 = 0, w1 = 0;
+      for (int e = 0; e < 2; ++e) {
+        const int r = qc + e;
+        const bool real = r < R;
+        const int tq = real ? r / a.G : 0, gq = real ? r % a.G : 0;
+        sq[e] = real ? __ldg(a.qs + ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq)) : 0.0f;
+        pos[e] = klen - a.Tq + tq;
+      }
+      // B fragments of Q^T (query row g8), byte-split, one table per CTA:
+      // entry [s][lane] = (hi slots 0-15, hi slots 16-31, lo slots 0-15, lo slots 16-31)
+      if (warp == 0) {
+        const int r = g8;
+        const bool real = r < R;
+        const int tq = real ? r / a.G : 0, gq = real ? r % a.G : 0;
+        const long long qrow = ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq);
+#pragma unroll
+        for (int s32 = 0; s32 < kKSteps32; ++s32) {
+          uint32_t w[4] = {0u, 0u, 0u, 0u};
           if (real) {
-            const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow * D + ks * 16 + tokq);
-            w0 = __ldg(qp);
-            w1 = __ldg(qp + 4);   // dims + 8
+            const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow * D + s32 * 32 + qc);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) w[i] = __ldg(qp + 4 * i);   // dims 32s + 8i + 2c, +1
           }
-          qf_sm[ks * 32 + lane] = make_uint4(hi_pair(w0), hi_pair(w1), lo_pair(w0), lo_pair(w1));
+          qf_sm[s32 * 32 + lane] = make_uint4(hi_bytes(w[0], w[1]), hi_bytes(w[2], w[3]), lo_bytes(w[0], w[1]),
+                                              lo_bytes(w[2], w[3]));
         }
       }
       compute_bar();
-      m_run = -INFINITY;
-      l_run = 0.0f;
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        m_run[e] = -INFINITY;
+        l_run[e] = 0.0f;
+      }
       E_run = 0;
       have_E = false;
 #pragma unroll
@@ -305,8 +360,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
     }
     const int t0 = blk * kBlk;
     if (t0 >= klen) continue;
-    const int s = it & 1;
-    const uint32_t ph = (uint32_t)(it >> 1) & 1u;
+    const int s = it % kStages;
+    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
     ++it;
     if (!mbar_wait(&full[s], ph, abort_flag, a.status, 210)) {
       ok = false;
@@ -318,100 +373,91 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
     const float* svs = sc_sm + (s * 2 + 1) * kBlk;   // V scales
     const int tw = warp * 16;                 // this warp's first token inside the tile
 
-    // ---- exact S = Q K^T on the byte-split operands ----
-    float x[2][2];                            // [n-block][token] logits * log2(e), row rowS
-    float shh[2][4], sx[2][4], sll[2][4];
+    // ---- exact S^T = K Q^T on the byte-split operands (integer tensor cores) ----
+    int shh[4] = {0, 0, 0, 0}, sx[4] = {0, 0, 0, 0}, sll[4] = {0, 0, 0, 0};
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb)
+    for (int s32 = 0; s32 < kKSteps32; ++s32) {
+      const uint4 qf = qf_sm[s32 * 32 + lane];
+      uint32_t r[2][4];                       // [token half][16-byte chunk 4*s32 + i]
 #pragma unroll
-      for (int e = 0; e < 4; ++e) shh[nb][e] = sx[nb][e] = sll[nb][e] = 0.0f;
-#pragma unroll
-    for (int j = 0; j < kKSteps / 2; ++j) {
-      const uint4 qa = qf_sm[(2 * j) * 32 + lane];
-      const uint4 qb = qf_sm[(2 * j + 1) * 32 + lane];
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        const int trow = tw + nb * 8 + (lane & 7);
-        const int ch = 4 * j + (lane >> 3);   // 16-byte chunk of the 256-byte K row
+      for (int th = 0; th < 2; ++th) {
+        const int trow = tw + th * 8 + (lane & 7);
+        const int ch = 4 * s32 + (lane >> 3);   // 16-byte chunk of the K row
         const uint32_t addr = kst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4(addr, r0, r1, r2, r3);
-        {
-          const uint32_t kh0 = hi_pair(r0), kh1 = hi_pair(r1), kl0 = lo_pair(r0), kl1 = lo_pair(r1);
-          mma16816(shh[nb], qa.x, 0u, qa.y, 0u, kh0, kh1);
-          mma16816(sx[nb], qa.x, 0u, qa.y, 0u, kl0, kl1);
-          mma16816(sx[nb], qa.z, 0u, qa.w, 0u, kh0, kh1);
-          mma16816(sll[nb], qa.z, 0u, qa.w, 0u, kl0, kl1);
-        }
-        {
-          const uint32_t kh0 = hi_pair(r2), kh1 = hi_pair(r3), kl0 = lo_pair(r2), kl1 = lo_pair(r3);
-          mma16816(shh[nb], qb.x, 0u, qb.y, 0u, kh0, kh1);
-          mma16816(sx[nb], qb.x, 0u, qb.y, 0u, kl0, kl1);
-          mma16816(sx[nb], qb.z, 0u, qb.w, 0u, kh0, kh1);
-          mma16816(sll[nb], qb.z, 0u, qb.w, 0u, kl0, kl1);
-        }
+        ldsm_x4(addr, r[th][0], r[th][1], r[th][2], r[th][3]);
       }
+      // A fragments: a0 token g8 slots 0-15, a1 token g8+8, a2 token g8 slots 16-31, a3 token g8+8
+      const uint32_t ah0 = hi_bytes(r[0][0], r[0][1]), ah1 = hi_bytes(r[1][0], r[1][1]);
+      const uint32_t ah2 = hi_bytes(r[0][2], r[0][3]), ah3 = hi_bytes(r[1][2], r[1][3]);
+      const uint32_t al0 = lo_bytes(r[0][0], r[0][1]), al1 = lo_bytes(r[1][0], r[1][1]);
+      const uint32_t al2 = lo_bytes(r[0][2], r[0][3]), al3 = lo_bytes(r[1][2], r[1][3]);
+      imma16832<false, false>(shh, ah0, ah1, ah2, ah3, qf.x, qf.y);
+      imma16832<false, true>(sx, ah0, ah1, ah2, ah3, qf.z, qf.w);
+      imma16832<true, false>(sx, al0, al1, al2, al3, qf.x, qf.y);
+      imma16832<true, true>(sll, al0, al1, al2, al3, qf.z, qf.w);
     }
     // every ldmatrix of the K tile has been consumed by the MMAs above and the K scales
     // this lane needs are copied to registers: release the K half now, before the logit
     // arithmetic, so the producer can refill it sooner
-    float skr[2][2];
+    float skr[2];
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb)
-#pragma unroll
-      for (int e = 0; e < 2; ++e) skr[nb][e] = sks[tw + nb * 8 + tokq + e];
+    for (int th = 0; th < 2; ++th) skr[th] = sks[tw + th * 8 + g8];
     __syncwarp();
     if (lane == 0) mbar_arrive(&empty[s]);
+    float x[2][2];                            // [token half][query e]: logit * log2(e)
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
+    for (int th = 0; th < 2; ++th) {
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int t = t0 + tw + nb * 8 + tokq + e;
-        const long long S = ((long long)__float2int_rn(shh[nb][e]) << 16) +
-                            ((long long)__float2int_rn(sx[nb][e]) << 8) + (long long)__float2int_rn(sll[nb][e]);
-        const bool real = rowS < R;
-        const bool vis = real && t < klen && (!a.causal || t <= pos);
+        const int i = 2 * th + e;
+        const int t = t0 + tw + th * 8 + g8;
+        const int r = qc + e;
+        const long long S = ((long long)shh[i] << 16) + ((long long)sx[i] << 8) + (long long)sll[i];
+        const bool real = r < R;
+        const bool vis = real && t < klen && (!a.causal || t <= pos[e]);
         float xv;
         if (!real) {
-          xv = 0.0f;                          // padding row: finite, never written
+          xv = 0.0f;                          // padding query row: finite, never written
         } else if (!vis) {
           xv = -INFINITY;
         } else {
-          const double coef = (double)sq * (double)skr[nb][e];
+          const double coef = (double)sq[e] * (double)skr[th];
           const float lg = (float)(((double)S * coef) * (double)a.scale);
           xv = __fmul_rn(lg, kLog2e);
           if (a.qk_out) {
-            const int tq = rowS / a.G, g = rowS % a.G;
-            a.qk_out[((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq) * a.Tmax + t] = S;
+            const int tq = r / a.G, gq = r % a.G;
+            a.qk_out[((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq) * a.Tmax + t] = S;
           }
         }
-        x[nb][e] = xv;
+        x[th][e] = xv;
       }
     }
 
-    if (!mbar_wait(&full[2 + s], ph, abort_flag, a.status, 211)) {
+    if (!mbar_wait(&full[kStages + s], ph, abort_flag, a.status, 211)) {
       ok = false;
       break;
     }
 
-    // ---- online softmax (base 2), row rowS ----
-    float bm = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
-    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 1));
-    bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 2));
-    const float m_new = fmaxf(m_run, bm);
-    float alpha, pv[2][2];
-    if (m_new == -INFINITY) {
-      alpha = 1.0f;
-      pv[0][0] = pv[0][1] = pv[1][0] = pv[1][1] = 0.0f;
-    } else {
-      alpha = (m_run == -INFINITY) ? 0.0f : exp2f(m_run - m_new);
+    // ---- online softmax (base 2) of query rows qc, qc + 1 over this warp's tokens ----
+    float alpha[2], pv[2][2];
 #pragma unroll
-      for (int nb = 0; nb < 2; ++nb)
+    for (int e = 0; e < 2; ++e) {
+      float bm = fmaxf(x[0][e], x[1][e]);
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+      const float m_new = fmaxf(m_run[e], bm);
+      if (m_new == -INFINITY) {
+        alpha[e] = 1.0f;
+        pv[0][e] = pv[1][e] = 0.0f;
+      } else {
+        alpha[e] = (m_run[e] == -INFINITY) ? 0.0f : exp2f(m_run[e] - m_new);
 #pragma unroll
-        for (int e = 0; e < 2; ++e) pv[nb][e] = (x[nb][e] == -INFINITY) ? 0.0f : exp2f(x[nb][e] - m_new);
+        for (int th = 0; th < 2; ++th) pv[th][e] = (x[th][e] == -INFINITY) ? 0.0f : exp2f(x[th][e] - m_new);
+      }
+      l_run[e] = __fadd_rn(__fmul_rn(l_run[e], alpha[e]), __fadd_rn(pv[0][e], pv[1][e]));
+      m_run[e] = m_new;
     }
-    l_run = __fadd_rn(__fmul_rn(l_run, alpha), __fadd_rn(__fadd_rn(pv[0][0], pv[0][1]), __fadd_rn(pv[1][0], pv[1][1])));
-    m_run = m_new;
     // power of two for this block: the largest visible V scale times 2^E in [32, 64)
     float smax = 0.0f;
     {
@@ -432,40 +478,62 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
         E_run = E_blk;
       }
     }
-    // rescale O^T rows tokq, tokq+1: their alphas live in S-layout lanes 4*tokq, 4*(tokq+1)
-    const float a0 = __fmul_rn(__shfl_sync(0xffffffffu, alpha, 4 * tokq), escale);
-    const float a1 = __fmul_rn(__shfl_sync(0xffffffffu, alpha, 4 * (tokq + 1)), escale);
+    // rescale O^T columns qc, qc + 1 (this lane's own query rows)
+    const float a0 = __fmul_rn(alpha[0], escale);
+    const float a1 = __fmul_rn(alpha[1], escale);
     if (!__all_sync(0xffffffffu, a0 == 1.0f && a1 == 1.0f)) {
 #pragma unroll
-    for (int dt = 0; dt < D / 16; ++dt) {
-      om[dt][0] = __fmul_rn(om[dt][0], a0);
-      om[dt][1] = __fmul_rn(om[dt][1], a1);
-      om[dt][2] = __fmul_rn(om[dt][2], a0);
-      om[dt][3] = __fmul_rn(om[dt][3], a1);
-    }
+      for (int dt = 0; dt < D / 16; ++dt) {
+        om[dt][0] = __fmul_rn(om[dt][0], a0);
+        om[dt][1] = __fmul_rn(om[dt][1], a1);
+        om[dt][2] = __fmul_rn(om[dt][2], a0);
+        om[dt][3] = __fmul_rn(om[dt][3], a1);
+      }
     }
 
-    // ---- P' = P * s_v * 2^E as FP16 (P_hi, r = P' - P_hi): B fragments of PV ----
+    // ---- P' = P * s_v * 2^E (S^T layout), moved to the B layout of PV: lane (g8, c)
+    // needs tokens 2c, 2c + 1, 2c + 8, 2c + 9 of query row g8.  Token 2c + j lives in lane
+    // 4 * (2c + j) + g8 / 2 (halves th = 0 / 1 for +0 / +8), query row g8 in its slot g8 & 1.
     const float e2 = ldexpf(1.0f, E_run);
-    uint32_t ph_[2], pr_[2], ph256[2], pr256[2];
+    float pp[2][2];
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) {
-      float pp[2];
+    for (int th = 0; th < 2; ++th) {
+      const int t = t0 + tw + th * 8 + g8;
+      const float svt = svs[t - t0];
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const int t = t0 + tw + nb * 8 + tokq + e;
-        const float sv = (pv[nb][e] != 0.0f) ? __fmul_rn(svs[t - t0], e2) : 0.0f;
-        pp[e] = __fmul_rn(pv[nb][e], sv);
+        const float sv = (pv[th][e] != 0.0f) ? __fmul_rn(svt, e2) : 0.0f;
+        pp[th][e] = __fmul_rn(pv[th][e], sv);
       }
-      const __half2 h = __floats2half2_rn(pp[0], pp[1]);
+    }
+    float pt[2][2];                            // [token half][j]: P' of token 8*half + 2c + j, query g8
+    {
+      const int cq = lane & 3;
+      const bool odd = (g8 & 1) != 0;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int src = 4 * (2 * cq + j) + (g8 >> 1);
+#pragma unroll
+        for (int th = 0; th < 2; ++th) {
+          const float v0 = __shfl_sync(0xffffffffu, pp[th][0], src);
+          const float v1 = __shfl_sync(0xffffffffu, pp[th][1], src);
+          pt[th][j] = odd ? v1 : v0;
+        }
+      }
+    }
+    // FP16 P_hi and residual r = P' - P_hi: B fragments of PV
+    uint32_t ph_[2], pr_[2], ph256[2], pr256[2];
+#pragma unroll
+    for (int th = 0; th < 2; ++th) {
+      const __half2 h = __floats2half2_rn(pt[th][0], pt[th][1]);
       const float2 hf = __half22float2(h);
-      const __half2 r = __floats2half2_rn(__fsub_rn(pp[0], hf.x), __fsub_rn(pp[1], hf.y));
+      const __half2 rr = __floats2half2_rn(__fsub_rn(pt[th][0], hf.x), __fsub_rn(pt[th][1], hf.y));
       const __half2 k256 = __half2half2(__ushort_as_half(0x5C00));   // 256.0
-      const __half2 h256 = __hmul2(h, k256), r256 = __hmul2(r, k256); // exact: powers of two
-      ph_[nb] = *reinterpret_cast<const uint32_t*>(&h);
-      pr_[nb] = *reinterpret_cast<const uint32_t*>(&r);
-      ph256[nb] = *reinterpret_cast<const uint32_t*>(&h256);
-      pr256[nb] = *reinterpret_cast<const uint32_t*>(&r256);
+      const __half2 h256 = __hmul2(h, k256), r256 = __hmul2(rr, k256); // exact: powers of two
+      ph_[th] = *reinterpret_cast<const uint32_t*>(&h);
+      pr_[th] = *reinterpret_cast<const uint32_t*>(&rr);
+      ph256[th] = *reinterpret_cast<const uint32_t*>(&h256);
+      pr256[th] = *reinterpret_cast<const uint32_t*>(&r256);
     }
 
     // ---- O^T += V^T P'^T  (256*hi*P + lo*P with P = P_hi + r) ----
@@ -485,7 +553,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) heal_attn_decode_kernel(const
       mma16816(om[dt], l0, l1, l2, l3, pr_[0], pr_[1]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[2 + s]);
+    if (lane == 0) mbar_arrive(&empty[kStages + s]);
   }
   if (!ok) return;   // a wait gave up: the status word is set; leave without a partial
   if (cur_p >= 0) finalize(cur_p);
@@ -519,8 +587,8 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
 
 template <int D>
 constexpr int attn_smem_bytes() {
-  return 2 * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + (D / 16) * 32 * 16 + 2 * 2 * kBlk * 4 +
-         96 + 1024;
+  return kStages * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + (D / 32) * 32 * 16 +
+         kStages * 2 * kBlk * 4 + 2 * 2 * kStages * 8 + 32 + 1024;
 }
 
 }  // namespace

@@ -39,9 +39,19 @@ namespace heal {
 
 constexpr int kBM = 128;   // MMA M: rows of kernel-A per tile (= TMEM lanes)
 constexpr int kBK = 64;    // K per stage = one accumulation chunk
-constexpr int kThreads = 384;
-constexpr int kSplitWarp0 = 2, kNumSplitWarps = 6;
-constexpr int kEpiWarp0 = 8, kNumEpiWarps = 4;
+constexpr int kSplitWarp0 = 2, kNumEpiWarps = 4;
+
+// Warp roles per tile width: warp 0 TMA, warp 1 MMA, then the split warps, then four
+// epilogue warps (which must start at a multiple of 4 so that warp % 4 names the TMEM lane
+// quarter).  Six split warps for every tile width (ten measured no faster on the skinny
+// decode tiles, whose time goes elsewhere).
+template <int BN>
+struct Roles {
+  static constexpr int kSplitWarps = 6;
+  static constexpr int kEpiWarp0 = kSplitWarp0 + kSplitWarps;
+  static constexpr int kThreads = (kEpiWarp0 + kNumEpiWarps) * 32;
+  static_assert(kEpiWarp0 % 4 == 0, "epilogue warps must start at a lane-quarter boundary");
+};
 
 struct GemmArgs {
   int Mk, Nk, K;            // kernel-space rows of kernel-A, rows of kernel-B, reduction
@@ -158,17 +168,25 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
 // ---------------------------------------------------------------------------------
 __device__ __forceinline__ float pow2f(int e) { return __int_as_float((127 + e) << 23); }
 
-template <int FMT, bool MN>
-__device__ __forceinline__ void split_pair(uint8_t* src0, uint8_t* src1, int lane, const int8_t* chan_exp,
-                                           int exp_sign, int kb, int K) {
+// Load half: this lane's 16 FP32 values (two 16-byte pieces of each atom).
+__device__ __forceinline__ void split_load(const uint8_t* src0, const uint8_t* src1, int lane, float (&v)[16]) {
   const int row = lane & 7, q = lane >> 3;
-  uint8_t* r0 = src0 + row * 128;
-  uint8_t* r1 = src1 + row * 128;
-  float v[16];
+  const uint8_t* r0 = src0 + row * 128;
+  const uint8_t* r1 = src1 + row * 128;
   *reinterpret_cast<float4*>(&v[0]) = *reinterpret_cast<const float4*>(r0 + (((2 * q) ^ row) << 4));
   *reinterpret_cast<float4*>(&v[4]) = *reinterpret_cast<const float4*>(r0 + (((2 * q + 1) ^ row) << 4));
   *reinterpret_cast<float4*>(&v[8]) = *reinterpret_cast<const float4*>(r1 + (((2 * q) ^ row) << 4));
   *reinterpret_cast<float4*>(&v[12]) = *reinterpret_cast<const float4*>(r1 + (((2 * q + 1) ^ row) << 4));
+}
+
+// Store half: optional channel exponents, the split, and the hi / lo 16-byte pieces.  The
+// caller has synchronised the warp after every lane's split_load of this region.
+template <int FMT, bool MN>
+__device__ __forceinline__ void split_store(uint8_t* src0, uint8_t* src1, int lane, float (&v)[16],
+                                            const int8_t* chan_exp, int exp_sign, int kb, int K) {
+  const int row = lane & 7, q = lane >> 3;
+  uint8_t* r0 = src0 + row * 128;
+  uint8_t* r1 = src1 + row * 128;
   if (chan_exp != nullptr) {
     if constexpr (MN) {
       // every value of this lane has K index kb + row
@@ -185,7 +203,6 @@ __device__ __forceinline__ void split_pair(uint8_t* src0, uint8_t* src1, int lan
       }
     }
   }
-  __syncwarp();
   uint4 h0, h1, l0, l1;
   h0.x = split2<FMT>(v[0], v[1], l0.x);
   h0.y = split2<FMT>(v[2], v[3], l0.y);
@@ -199,6 +216,16 @@ __device__ __forceinline__ void split_pair(uint8_t* src0, uint8_t* src1, int lan
   *reinterpret_cast<uint4*>(r0 + (((4 + q) ^ row) << 4)) = h1;
   *reinterpret_cast<uint4*>(r1 + ((q ^ row) << 4)) = l0;
   *reinterpret_cast<uint4*>(r1 + (((4 + q) ^ row) << 4)) = l1;
+}
+
+// One warp splits one 2 KB region pair in place.
+template <int FMT, bool MN>
+__device__ __forceinline__ void split_pair(uint8_t* src0, uint8_t* src1, int lane, const int8_t* chan_exp,
+                                           int exp_sign, int kb, int K) {
+  float v[16];
+  split_load(src0, src1, lane, v);
+  __syncwarp();   // every lane has read the region before any lane overwrites it
+  split_store<FMT, MN>(src0, src1, lane, v, chan_exp, exp_sign, kb, K);
 }
 
 // Region pair t of an operand tile with R rows (t in [0, R/8)).
@@ -233,12 +260,14 @@ struct OperandDesc {
 // The kernel
 // ---------------------------------------------------------------------------------
 template <int BN, bool A_MN, bool B_MN, int FMT, bool CORR_SWAP, bool A_PRE, bool B_PRE>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
     heal_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA_lo,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB_lo,
                      const GemmArgs args) {
   using C = Cfg<BN>;
   constexpr int S = C::kStages;
+  constexpr int kNumSplitWarps = Roles<BN>::kSplitWarps;
+  constexpr int kEpiWarp0 = Roles<BN>::kEpiWarp0;
   constexpr int kLoShift = FMT == 0 ? 11 : 0;
   constexpr uint32_t kIdesc = idesc_f16(kBM, BN, FMT, A_MN ? 1 : 0, B_MN ? 1 : 0);
 
@@ -798,7 +827,7 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& alo, const C
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<grid, kThreads, smem, stream>>>(a, alo, b, blo, args);
+  kern<<<grid, Roles<BN>::kThreads, smem, stream>>>(a, alo, b, blo, args);
   return cudaGetLastError();
 }
 
@@ -807,6 +836,22 @@ cudaError_t launch_fmt(int fmt, const CUtensorMap& a, const CUtensorMap& alo, co
                        const CUtensorMap& blo, const GemmArgs& args, int grid, cudaStream_t stream) {
   if (fmt == 0) return launch_variant<BN, A_MN, B_MN, 0, CORR_SWAP, A_PRE, B_PRE>(a, alo, b, blo, args, grid, stream);
   return launch_variant<BN, A_MN, B_MN, 1, CORR_SWAP, A_PRE, B_PRE>(a, alo, b, blo, args, grid, stream);
+}
+
+// Swapped-operand skinny kernels: kernel-A = the weights (pre-split or FP32), kernel-B =
+// the M <= 64 activation rows padded to BN = 16 / 32 / 64.
+template <bool PRE>
+cudaError_t launch_skinny(int BNk, bool b_mn, int fmt, const CUtensorMap& a, const CUtensorMap& alo,
+                          const CUtensorMap& b, const CUtensorMap& blo, const GemmArgs& args, int grid,
+                          cudaStream_t stream) {
+  if (BNk == 16)
+    return b_mn ? launch_fmt<16, true, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream)
+                : launch_fmt<16, false, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream);
+  if (BNk == 32)
+    return b_mn ? launch_fmt<32, true, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream)
+                : launch_fmt<32, false, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream);
+  return b_mn ? launch_fmt<64, true, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream)
+              : launch_fmt<64, false, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream);
 }
 
 template <bool B_MN, int FMT, bool B_PRE>
@@ -840,8 +885,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
                           float* Cout, long long ldc, int fmt, const heal_gemm_opts_t& o, cudaStream_t stream) {
   int cfg = o.tile_config;
   if (cfg == HEAL_TILE_AUTO) {
-    if (M <= 64 && o.workspace != nullptr && o.workspace_bytes >= gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK) &&
-        !o.b_presplit)
+    if (M <= 64 && o.workspace != nullptr && o.workspace_bytes >= gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK))
       cfg = HEAL_TILE_SKINNY_SPLITK;
     else if (M >= 256 && N >= 256)
       cfg = HEAL_TILE_256x256_PAIR;
@@ -933,7 +977,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
 
   if (cfg == HEAL_TILE_SKINNY_SPLITK || cfg == HEAL_TILE_SKINNY_FULLK) {
     const bool split = (cfg == HEAL_TILE_SKINNY_SPLITK);
-    if (o.b_presplit) return HEAL_ERR_UNSUPPORTED;
+    const bool pre = o.b_presplit != 0;   // weights given as (hi, lo): kernel-A skips its split
     if (M > 64) return HEAL_ERR_UNSUPPORTED;
     if (split && (o.workspace == nullptr || o.workspace_bytes < gemm_workspace_bytes(M, N, K, cfg)))
       return HEAL_ERR_INVALID_ARGUMENT;
@@ -950,19 +994,13 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.expA_sign = +1;
     args.expB_sign = -1;
     const int BNk = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-    if (!operand_map(&ta, B, b_mn, false, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
+    if (!operand_map(&ta, B, b_mn, pre, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
+    if (pre && !operand_map(&talo, o.b_lo, b_mn, true, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (!operand_map(&tb, A, false, false, M, K, lda, BNk)) return HEAL_ERR_CUDA;
     const long long units = split ? (long long)args.tiles_m * nc : (long long)args.tiles_m;
     const int grid = (int)(units < sms ? units : sms);
-    if (BNk == 16)
-      err = b_mn ? launch_fmt<16, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
-                 : launch_fmt<16, false, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
-    else if (BNk == 32)
-      err = b_mn ? launch_fmt<32, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
-                 : launch_fmt<32, false, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
-    else
-      err = b_mn ? launch_fmt<64, true, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
-                 : launch_fmt<64, false, false, true, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
+    err = pre ? launch_skinny<true>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
+              : launch_skinny<false>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
     if (err != cudaSuccess) return HEAL_ERR_CUDA;
     if (!split) return HEAL_OK;
     const long long rblocks = (long long)((N + 31) / 32) * M;

@@ -93,6 +93,26 @@ def test_presplit_b_matches_in_kernel_split(fmt, b_layout):
     assert np.array_equal(c_in, c_pre)
 
 
+@pytest.mark.parametrize("M", [1, 8, 33, 64])
+@pytest.mark.parametrize("b_layout", [0, 1])
+@pytest.mark.parametrize("fmt", [heal.SPLIT_FP16_S11, heal.SPLIT_BF16])
+def test_skinny_presplit_weights_bitwise(M, b_layout, fmt):
+    """Decode shapes with the weights split once by heal_split: the swapped-operand
+    kernels (split-K and full-K) give the bits of the in-kernel split, ragged K and N."""
+    d = dev()
+    K, N = 1000, 648
+    X, W = synthetic.gemm_decode(M, K=K, N=N)
+    Bin = W if b_layout == 0 else W.T.contiguous()
+    B_d = Bin.to(d).contiguous()
+    hi = torch.empty(B_d.shape, dtype=torch.int16, device=d)
+    lo = torch.empty(B_d.shape, dtype=torch.int16, device=d)
+    heal.heal_split(B_d, hi, lo, fmt)
+    c_ref = gemm(X.numpy(), Bin.numpy(), fmt=fmt, b_layout=b_layout, tile=heal.TILE_128x128)
+    for tile in (heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK, heal.TILE_AUTO):
+        c_pre = gemm(X.numpy(), hi, fmt=fmt, b_layout=b_layout, tile=tile, b_lo=lo)
+        assert np.array_equal(c_pre, c_ref), tile
+
+
 def test_outlier_channel_rescale():
     rng = np.random.default_rng(3)
     A = rng.standard_normal((160, 320)).astype(np.float32)
