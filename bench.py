@@ -33,6 +33,7 @@ sys.path.insert(0, ROOT)
 METRIC = "compensated-GEMM effective TFLOP/s (% of 16-bit TC peak); INT16-KV attn GB/s"
 PREFILL = (4096, 4096, 14336)
 DECODE_M = (1, 8, 64)
+CHAIN = 8             # decode GEMMs issued back to back in the chain part
 KV = dict(B=8, T=8192, Hkv=8, Hq=32, D=128)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
@@ -132,6 +133,22 @@ class Workload:
                 wlo = torch.empty(Wd.shape, dtype=torch.int16, device=dev)
                 heal.heal_split(Wd, whi, wlo)
                 self.dec.append((m, Xd.to(dev), Wd, torch.empty(m, 4096, device=dev), ws, whi, wlo))
+            # a chain of CHAIN decode GEMMs with distinct weights, each one's output the next
+            # one's input, issued back to back as a decoder issues its projections
+            self.chain = []
+            for i in range(CHAIN):
+                Wc = synthetic.normal((4096, 4096), seed=500 + so + i, std=0.02).to(dev)
+                chi = torch.empty(Wc.shape, dtype=torch.int16, device=dev)
+                clo = torch.empty(Wc.shape, dtype=torch.int16, device=dev)
+                heal.heal_split(Wc, chi, clo)
+                self.chain.append((Wc, chi, clo, torch.empty(1, 4096, device=dev)))
+            # the same weights held as FP16 values (the two-product form: only activations split)
+            self.dec16 = [(m, Xd, chi16, Cd, ws) for (m, Xd, Wd, Cd, ws, whi, wlo), chi16 in
+                          zip(self.dec, [Wd.half() for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec])]
+            self.chain16 = [Wc.half() for (Wc, chi, clo, Cc) in self.chain]
+            self.chain_x = synthetic.normal((1, 4096), seed=600 + so).to(dev)
+            self.chain_ws = torch.empty(heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK) // 4,
+                                        device=dev)
         if need("kv_writer"):
             B, T, Hkv, Hq, D = KV["B"], KV["T"], KV["Hkv"], KV["Hq"], KV["D"]
             Qb, Kb, Vb = synthetic.kv_decode(B=B, T=T, Hkv=Hkv, Hq=Hq, D=D, seeds=(2 + so, 3 + so, 4 + so))
@@ -157,6 +174,9 @@ class Workload:
             "prefill_flop_eff": 2.0 * M * N * K,
             "prefill_flop_mma": 3 * 2.0 * M * N * K,
             "decode_bytes": {m: 4.0 * (4096 * 4096 + m * 4096 + m * 4096) for m in DECODE_M},
+            "chain_bytes": CHAIN * 4.0 * (4096 * 4096 + 2 * 4096),
+            "decode16_bytes": {m: 2.0 * 4096 * 4096 + 4.0 * (m * 4096 + m * 4096) for m in DECODE_M},
+            "chain16_bytes": CHAIN * (2.0 * 4096 * 4096 + 8.0 * 4096),
             "kv_writer_bytes": 2 * (2 * kv_elems + 2 * kv_elems + 4 * B * Hkv * T) + (2 + 2) * B * Hq * D + 4 * B * Hq,
             "attn_bytes": 2 * (2 * kv_elems + 4 * B * Hkv * T) + 2 * B * Hq * D + 4 * B * Hq + 4 * B * Hq * D,
         }
@@ -175,6 +195,12 @@ class Workload:
             for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
                 out.append((f"decode{m}_presplit", lambda Xd=Xd, whi=whi, wlo=wlo, Cd=Cd, ws=ws:
                             h.heal_gemm_compensated(Xd, whi, Cd, b_lo=wlo, workspace=ws)))
+            for (m, Xd, W16, Cd, ws) in self.dec16:
+                out.append((f"decode{m}_w16", lambda Xd=Xd, W16=W16, Cd=Cd, ws=ws: h.heal_gemm_compensated(
+                    Xd, W16, Cd, workspace=ws, b_16bit=True)))
+            out.append(("decode1_chain", lambda: self.run_chain(False)))
+            out.append(("decode1_chain_presplit", lambda: self.run_chain(True)))
+            out.append(("decode1_chain_w16", lambda: self.run_chain16()))
         if only in (None, "kv_writer", "attention"):
             out.append(("kv_writer", lambda: (h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs),
                                               h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks),
@@ -184,6 +210,21 @@ class Workload:
                 self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len, KV["D"] ** -0.5, self.out,
                 self.aws)))
         return out
+
+    def run_chain(self, presplit):
+        a = self.chain_x
+        for (Wc, chi, clo, Cc) in self.chain:
+            if presplit:
+                self.heal.heal_gemm_compensated(a, chi, Cc, b_lo=clo, workspace=self.chain_ws, b_static=True)
+            else:
+                self.heal.heal_gemm_compensated(a, Wc, Cc, workspace=self.chain_ws, b_static=True)
+            a = Cc
+
+    def run_chain16(self):
+        a = self.chain_x
+        for (Wc, chi, clo, Cc), W16 in zip(self.chain, self.chain16):
+            self.heal.heal_gemm_compensated(a, W16, Cc, workspace=self.chain_ws, b_static=True, b_16bit=True)
+            a = Cc
 
     def capture(self, stream):
         """One CUDA graph per part, captured from the library calls (replays launch the same
@@ -226,6 +267,17 @@ class Workload:
                 rec(f"decode{m}_presplit", 0)
                 h.heal_gemm_compensated(Xd, whi, Cd, b_lo=wlo, workspace=ws)
                 rec(f"decode{m}_presplit", 1)
+            for (m, Xd, W16, Cd, ws) in self.dec16:
+                rec(f"decode{m}_w16", 0)
+                h.heal_gemm_compensated(Xd, W16, Cd, workspace=ws, b_16bit=True)
+                rec(f"decode{m}_w16", 1)
+            for name, pre in (("decode1_chain", False), ("decode1_chain_presplit", True)):
+                rec(name, 0)
+                self.run_chain(pre)
+                rec(name, 1)
+            rec("decode1_chain_w16", 0)
+            self.run_chain16()
+            rec("decode1_chain_w16", 1)
         if only in (None, "kv_writer", "attention"):
             rec("kv_writer", 0)
             h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs)
@@ -238,7 +290,7 @@ class Workload:
                                    KV["D"] ** -0.5, self.out, self.aws)
             rec("attention", 1)
 
-    LAUNCHES_PER_STEP = 1 + 2 * 2 * len(DECODE_M) + 3 + 2
+    LAUNCHES_PER_STEP = 1 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
 
 
 def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=128):
@@ -384,7 +436,9 @@ def main():
     if st != heal.HEAL_OK:
         raise SystemExit(f"device status after warm-up: {heal.status_string(st)}")
 
-    dec_names = [f"decode{m}" for m in DECODE_M] + [f"decode{m}_presplit" for m in DECODE_M]
+    dec_names = ([f"decode{m}" for m in DECODE_M] + [f"decode{m}_presplit" for m in DECODE_M] +
+                 [f"decode{m}_w16" for m in DECODE_M] +
+                 ["decode1_chain", "decode1_chain_presplit", "decode1_chain_w16"])
     names = ["prefill"] + dec_names + ["kv_writer", "attention"]
     if args.only:
         keep = {"prefill": ["prefill"], "decode": dec_names,
@@ -443,6 +497,15 @@ def main():
             t = part_ms[f"decode{m}{suffix}"] / 1e3 / K
             dec[key] = {"gbs": u["decode_bytes"][m] / t / 1e9, "us": 1e6 * t,
                         "frac_hbm": u["decode_bytes"][m] / t / 1e9 / hbm}
+    for m in DECODE_M:
+        t = part_ms[f"decode{m}_w16"] / 1e3 / K
+        dec[f"M{m}_fp16_weights_two_products"] = {"gbs": u["decode16_bytes"][m] / t / 1e9, "us": 1e6 * t,
+                                                  "frac_hbm": u["decode16_bytes"][m] / t / 1e9 / hbm}
+    for suffix, key, nb in (("", "M1_chain", "chain_bytes"), ("_presplit", "M1_chain_presplit_weights", "chain_bytes"),
+                            ("_w16", "M1_chain_fp16_weights_two_products", "chain16_bytes")):
+        t = part_ms[f"decode1_chain{suffix}"] / 1e3 / K
+        dec[key] = {"gemms": CHAIN, "us_per_gemm": 1e6 * t / CHAIN, "gbs": u[nb] / t / 1e9,
+                    "frac_hbm": u[nb] / t / 1e9 / hbm}
 
     # end to end through the public API: pinned host inputs -> device -> GEMM -> host result
     M_, K_, N_ = PREFILL

@@ -27,7 +27,8 @@ class HealError(RuntimeError):
 class GemmOpts(ctypes.Structure):
     _fields_ = [("tile_config", ctypes.c_int), ("chan_exp", ctypes.c_void_p), ("b_layout", ctypes.c_int),
                 ("b_presplit", ctypes.c_int), ("b_lo", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_size_t), ("reserved", ctypes.c_int * 4)]
+                ("workspace_bytes", ctypes.c_size_t), ("b_static", ctypes.c_int),
+                ("reserved", ctypes.c_int * 3)]
 
 
 _lib = None
@@ -110,15 +111,19 @@ def heal_split(x, hi, lo, fmt=SPLIT_FP16_S11, stream=None):
     _check(lib().heal_split(_ptr(x), _ptr(hi), _ptr(lo), x.numel(), int(fmt), _stream(stream)), "heal_split")
 
 
-def gemm_opts(tile_config=TILE_AUTO, chan_exp=None, b_layout=0, b_lo=None, workspace=None):
+def gemm_opts(tile_config=TILE_AUTO, chan_exp=None, b_layout=0, b_lo=None, workspace=None, b_static=False,
+              b_16bit=False):
     o = GemmOpts()
     o.tile_config = int(tile_config)
     o.chan_exp = None if chan_exp is None else chan_exp.data_ptr()
     o.b_layout = int(b_layout)
-    o.b_presplit = 1 if b_lo is not None else 0
+    if b_16bit and b_lo is not None:
+        raise ValueError("a 16-bit B has no lo part")
+    o.b_presplit = 2 if b_16bit else (1 if b_lo is not None else 0)
     o.b_lo = None if b_lo is None else b_lo.data_ptr()
     o.workspace = None if workspace is None else workspace.data_ptr()
     o.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    o.b_static = 1 if b_static else 0
     return o
 
 
@@ -128,9 +133,10 @@ def heal_gemm_workspace_bytes(M, N, K, tile_config=TILE_AUTO):
 
 
 def heal_gemm_compensated(A, B, C, fmt=SPLIT_FP16_S11, tile_config=TILE_AUTO, chan_exp=None, b_layout=0,
-                          b_lo=None, workspace=None, stream=None):
+                          b_lo=None, workspace=None, b_static=False, b_16bit=False, stream=None):
     """C[M,N] = A[M,K] . B with B [K,N] (b_layout 0) or [N,K] (b_layout 1); B may be the
-    16-bit hi part with b_lo the lo part (pre-split weights)."""
+    16-bit hi part with b_lo the lo part (pre-split weights), or a 16-bit matrix with
+    b_16bit=True (two products: only A is split)."""
     _cuda(A, B, C, chan_exp, b_lo, workspace)
     if A.dim() != 2 or B.dim() != 2 or C.dim() != 2 or A.stride(1) != 1 or B.stride(1) != 1 or C.stride(1) != 1:
         raise ValueError("heal_gemm_compensated takes 2-D row-major tensors")
@@ -138,7 +144,7 @@ def heal_gemm_compensated(A, B, C, fmt=SPLIT_FP16_S11, tile_config=TILE_AUTO, ch
     N = C.shape[1]
     if C.shape[0] != M or (B.shape != ((K, N) if b_layout == 0 else (N, K))):
         raise ValueError("shape mismatch")
-    o = gemm_opts(tile_config, chan_exp, b_layout, b_lo, workspace)
+    o = gemm_opts(tile_config, chan_exp, b_layout, b_lo, workspace, b_static, b_16bit)
     st = lib().heal_gemm_compensated(M, N, K, _ptr(A), A.stride(0), _ptr(B), B.stride(0), _ptr(C), C.stride(0),
                                      int(fmt), ctypes.byref(o), _stream(stream))
     _check(st, "heal_gemm_compensated")

@@ -62,6 +62,8 @@ struct GemmArgs {
   float* ws;                // [num_chunks][Nk][Mk] chunk values (split-K mode)
   const int8_t* chan_exp;   // nullable, [K]
   int expA_sign, expB_sign; // +1 / -1: which operand gets 2^+e and which 2^-e
+  int static_op;            // 0: none; 1: kernel-A, 2: kernel-B is not written by the kernels
+                            // before this one (its first stages may be requested early)
   unsigned int* status;     // device status word
 };
 
@@ -130,12 +132,13 @@ __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, 
 //   K-major  (K contiguous) : two boxes {32 K, R rows} -> [0, R*128) and [R*128, R*256)
 //   MN-major (rows contiguous): R/32 boxes {32 rows, 64 K} -> b*8192
 //   16-bit pre-split input   : hi/lo boxes of 64 values that land exactly where the
-//                              in-place split would have written them.
+//                              in-place split would have written them (PRE = 1), or
+//                              the hi boxes alone for a 16-bit operand (PRE = 2).
 // ---------------------------------------------------------------------------------
-template <int R, bool MN, bool PRESPLIT>
+template <int R, bool MN, int PRE>
 __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* map, const CUtensorMap* map_lo,
                                              uint64_t* bar, int row0, int k0) {
-  if constexpr (!PRESPLIT) {
+  if constexpr (PRE == 0) {
     if constexpr (!MN) {
       tma_load_2d(dst, map, bar, k0, row0);
       tma_load_2d(dst + R * 128, map, bar, k0 + 32, row0);
@@ -145,13 +148,13 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
     }
   } else {
     if constexpr (!MN) {
-      tma_load_2d(dst, map, bar, k0, row0);              // hi: R rows x 64 values
-      tma_load_2d(dst + R * 128, map_lo, bar, k0, row0);  // lo
+      tma_load_2d(dst, map, bar, k0, row0);                                   // hi: R rows x 64 values
+      if constexpr (PRE == 1) tma_load_2d(dst + R * 128, map_lo, bar, k0, row0);  // lo
     } else {
 #pragma unroll
       for (int p = 0; p < R / 64; ++p) {
         tma_load_2d(dst + (2 * p) * 8192, map, bar, row0 + 64 * p, k0);
-        tma_load_2d(dst + (2 * p + 1) * 8192, map_lo, bar, row0 + 64 * p, k0);
+        if constexpr (PRE == 1) tma_load_2d(dst + (2 * p + 1) * 8192, map_lo, bar, row0 + 64 * p, k0);
       }
     }
   }
@@ -259,7 +262,9 @@ struct OperandDesc {
 // ---------------------------------------------------------------------------------
 // The kernel
 // ---------------------------------------------------------------------------------
-template <int BN, bool A_MN, bool B_MN, int FMT, bool CORR_SWAP, bool A_PRE, bool B_PRE>
+// A_PRE / B_PRE: 0 FP32 split in the kernel, 1 pre-split hi + lo, 2 a 16-bit operand with
+// no residual (its correction product is absent: the two-product form).
+template <int BN, bool A_MN, bool B_MN, int FMT, bool CORR_SWAP, int A_PRE, int B_PRE>
 __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
     heal_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmA_lo,
                      const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmB_lo,
@@ -268,6 +273,9 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   constexpr int S = C::kStages;
   constexpr int kNumSplitWarps = Roles<BN>::kSplitWarps;
   constexpr int kEpiWarp0 = Roles<BN>::kEpiWarp0;
+  // bytes that land in a stage (a 16-bit-only operand fills only its hi half)
+  constexpr uint32_t kStageTx = C::kStageBytes - (A_PRE == 2 ? C::kABytes / 2 : 0) - (B_PRE == 2 ? C::kBBytes / 2 : 0);
+  constexpr bool kHasALo = A_PRE != 2, kHasBLo = B_PRE != 2;
   constexpr int kLoShift = FMT == 0 ? 11 : 0;
   constexpr uint32_t kIdesc = idesc_f16(kBM, BN, FMT, A_MN ? 1 : 0, B_MN ? 1 : 0);
 
@@ -310,8 +318,8 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   if (warp == 1 && lane == 0) {
     tma_prefetch_desc(&tmA);
     tma_prefetch_desc(&tmB);
-    if (A_PRE) tma_prefetch_desc(&tmA_lo);
-    if (B_PRE) tma_prefetch_desc(&tmB_lo);
+    if (A_PRE == 1) tma_prefetch_desc(&tmA_lo);
+    if (B_PRE == 1) tma_prefetch_desc(&tmB_lo);
   }
   tc_fence_before();
   __syncthreads();
@@ -323,6 +331,22 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
     // ------------------------------ TMA producer ------------------------------
     if constexpr (kRegSplit) setmaxnreg_dec<96>();
     if (lane == 0) {
+      // Programmatic dependent launch: this grid may start while the kernel before it is
+      // still running.  An operand the caller declared static is requested for the first
+      // stages right away; everything else waits for the preceding grid to finish.
+      int pre = 0;
+      if (args.static_op != 0) {
+        for (WorkIter w(args); w.valid() && pre < S; w.advance(), ++pre) {
+          int tm, tn;
+          tile_coords(w.tile, args.tiles_m, args.tiles_n, tm, tn);
+          const int k0 = w.chunk * kBK;
+          uint8_t* st = stages + pre * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[pre], kStageTx);
+          if (args.static_op == 1) load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, &full[pre], tm * kBM, k0);
+          else load_operand<BN, B_MN, B_PRE>(st + C::kABytes, &tmB, &tmB_lo, &full[pre], tn * BN, k0);
+        }
+      }
+      pdl_wait_prerequisites();
       int it = 0;
       for (WorkIter w(args); w.valid(); w.advance(), ++it) {
         const int s = it % S;
@@ -332,9 +356,10 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
         tile_coords(w.tile, args.tiles_m, args.tiles_n, tm, tn);
         const int k0 = w.chunk * kBK;
         uint8_t* st = stages + s * C::kStageBytes;
-        mbar_arrive_expect_tx(&full[s], C::kStageBytes);
-        load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, &full[s], tm * kBM, k0);
-        load_operand<BN, B_MN, B_PRE>(st + C::kABytes, &tmB, &tmB_lo, &full[s], tn * BN, k0);
+        if (it >= pre) mbar_arrive_expect_tx(&full[s], kStageTx);
+        if (it >= pre || args.static_op != 1) load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, &full[s], tm * kBM, k0);
+        if (it >= pre || args.static_op != 2)
+          load_operand<BN, B_MN, B_PRE>(st + C::kABytes, &tmB, &tmB_lo, &full[s], tn * BN, k0);
       }
       // Do not leave the CTA with copies in flight: wait (bounded) for the last fill of
       // every stage that was issued.
@@ -363,15 +388,17 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
         const uint64_t b_hi = OperandDesc<BN, B_MN>::hi(sb), b_lo = OperandDesc<BN, B_MN>::lo(sb);
         constexpr uint64_t dA = OperandDesc<kBM, A_MN>::kStep, dB = OperandDesc<BN, B_MN>::kStep;
         const uint32_t d = tmem_base + (uint32_t)(b * BN);
-        // corrections first: Ah.Bl then Al.Bh in the caller's operand order
+        // corrections first: Ah.Bl then Al.Bh in the caller's operand order (a 16-bit
+        // operand has no residual, so its correction product is absent)
 #pragma unroll
         for (int j = 0; j < kBK / 16; ++j) {
+          uint32_t acc_in = j > 0 ? 1u : 0u;
           if constexpr (!CORR_SWAP) {
-            mma_f16(d, a_hi + j * dA, b_lo + j * dB, kIdesc, j > 0 ? 1u : 0u);
-            mma_f16(d, a_lo + j * dA, b_hi + j * dB, kIdesc, 1u);
+            if constexpr (kHasBLo) { mma_f16(d, a_hi + j * dA, b_lo + j * dB, kIdesc, acc_in); acc_in = 1u; }
+            if constexpr (kHasALo) mma_f16(d, a_lo + j * dA, b_hi + j * dB, kIdesc, acc_in);
           } else {
-            mma_f16(d, a_lo + j * dA, b_hi + j * dB, kIdesc, j > 0 ? 1u : 0u);
-            mma_f16(d, a_hi + j * dA, b_lo + j * dB, kIdesc, 1u);
+            if constexpr (kHasALo) { mma_f16(d, a_lo + j * dA, b_hi + j * dB, kIdesc, acc_in); acc_in = 1u; }
+            if constexpr (kHasBLo) mma_f16(d, a_hi + j * dA, b_lo + j * dB, kIdesc, acc_in);
           }
         }
         // main product; its first step scales the corrections by 2^-L
@@ -389,6 +416,7 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   } else if (warp < kEpiWarp0) {
     // ------------------------------ split warps ------------------------------
     if constexpr (kRegSplit) setmaxnreg_dec<96>();
+    pdl_wait_prerequisites();   // chan_exp may come from the preceding kernel
     const int sw = warp - kSplitWarp0;
     constexpr int kPairsA = kBM / 8, kPairsB = BN / 8;
     int it = 0;
@@ -417,6 +445,7 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   } else {
     // ------------------------------ epilogue ------------------------------
     if constexpr (kRegSplit) setmaxnreg_inc<240>();
+    pdl_wait_prerequisites();   // C and the workspace may still be read by the preceding kernel
     const int quarter = warp & 3;            // TMEM lanes this warp may access
     const int i_local = quarter * 32 + lane; // tile row
     float acc[BN];
@@ -519,7 +548,7 @@ constexpr int kPairStageBytes = 2 * kPairRows * kBK * 4;
 constexpr int kPairStages = 3;
 constexpr int kPairSmemBytes = kPairStages * kPairStageBytes + 1024 + 1024;
 
-template <bool B_MN, int FMT, bool B_PRE>
+template <bool B_MN, int FMT, int B_PRE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     heal_gemm_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmB_lo, const GemmArgs args) {
@@ -545,6 +574,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   const int cid = blockIdx.x >> 1, ncl = gridDim.x >> 1;
   const int ntiles = args.tiles_m * args.tiles_n, nc = args.num_chunks;
 
+  pdl_launch_dependents();   // a following kernel may be scheduled; it waits for this grid
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
@@ -575,7 +605,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
-      if (B_PRE) tma_prefetch_desc(&tmB_lo);
+      if (B_PRE == 1) tma_prefetch_desc(&tmB_lo);
+      pdl_wait_prerequisites();   // the operands may come from the preceding kernel
       int it = 0;
       bool ok = true;
       for (int tile = cid; tile < ntiles && ok; tile += ncl) {
@@ -589,9 +620,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
             break;
           }
           uint8_t* st = stages + s * kPairStageBytes;
-          mbar_arrive_expect_tx(&full[s], kPairStageBytes);
-          load_operand<kPairRows, false, false>(st, &tmA, &tmA, &full[s], tm * 256 + kPairRows * (int)rank,
-                                                ch * kBK);
+          mbar_arrive_expect_tx(&full[s], kPairStageBytes - (B_PRE == 2 ? kPairRows * kBK * 2 : 0));
+          load_operand<kPairRows, false, 0>(st, &tmA, &tmA, &full[s], tm * 256 + kPairRows * (int)rank, ch * kBK);
           load_operand<kPairRows, B_MN, B_PRE>(st + kPairRows * kBK * 4, &tmB, &tmB_lo, &full[s],
                                                tn * kPairN + kPairRows * (int)rank, ch * kBK);
         }
@@ -629,8 +659,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
           const uint32_t d = tmem_base + (uint32_t)(b * kPairN);
 #pragma unroll
           for (int j = 0; j < kBK / 16; ++j) {
-            mma_f16_pair(d, a_hi + j * dA, b_lo + j * dB, kIdesc, j > 0 ? 1u : 0u);
-            mma_f16_pair(d, a_lo + j * dA, b_hi + j * dB, kIdesc, 1u);
+            if constexpr (B_PRE != 2) {
+              mma_f16_pair(d, a_hi + j * dA, b_lo + j * dB, kIdesc, j > 0 ? 1u : 0u);
+              mma_f16_pair(d, a_lo + j * dA, b_hi + j * dB, kIdesc, 1u);
+            } else {
+              mma_f16_pair(d, a_lo + j * dA, b_hi + j * dB, kIdesc, j > 0 ? 1u : 0u);
+            }
           }
           mma_f16_pair_scale_d<kLoShift>(d, a_hi, b_hi, kIdesc);
 #pragma unroll
@@ -649,6 +683,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else if (warp < kPairEpiWarp0) {
     // ------------------------------ split warps (both CTAs) ------------------------------
     setmaxnreg_dec<88>();
+    pdl_wait_prerequisites();   // chan_exp may come from the preceding kernel
     const int sw = warp - 2;
     constexpr int kPairsA = kPairRows / 8, kPairsB = kPairRows / 8;
     const uint32_t sd_leader0 = mapa_shared(smem_u32(&split_done[0]), 0u);
@@ -684,6 +719,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   } else {
     // ------------------------------ epilogue (both CTAs) ------------------------------
     setmaxnreg_inc<168>();
+    pdl_wait_prerequisites();   // C may still be read by the preceding kernel
     const int quarter = warp & 3;
     const int half = (warp - kPairEpiWarp0) >> 2;
     const int i_local = quarter * 32 + lane;
@@ -754,7 +790,8 @@ constexpr int kRedChunks = 128;
 __global__ void __launch_bounds__(256) heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk,
                                                                 int Nk, float* out, long long si, long long sj) {
   __shared__ float tile[kRedChunks][33];
-  pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed
+  pdl_launch_dependents();   // the next kernel may be scheduled; it waits for this grid
+  pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed   // the GEMM kernel that wrote ws has completed
   const int tiles_i = (Mk + 31) / 32;
   const int ti = blockIdx.x % tiles_i, j = blockIdx.x / tiles_i;
   const int i0 = ti * 32;
@@ -813,7 +850,7 @@ bool operand_map(CUtensorMap* map, const void* base, bool mn, bool is16, int row
   return encode_2d(map, dt, eb, base, (uint64_t)rows, (uint64_t)K, (uint64_t)ld, inner_box, 64u);
 }
 
-template <int BN, bool A_MN, bool B_MN, int FMT, bool CORR_SWAP, bool A_PRE, bool B_PRE>
+template <int BN, bool A_MN, bool B_MN, int FMT, bool CORR_SWAP, int A_PRE, int B_PRE>
 cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& alo, const CUtensorMap& b,
                            const CUtensorMap& blo, const GemmArgs& args, int grid, cudaStream_t stream) {
   auto kern = heal_gemm_kernel<BN, A_MN, B_MN, FMT, CORR_SWAP, A_PRE, B_PRE>;
@@ -827,11 +864,12 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& alo, const C
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<grid, Roles<BN>::kThreads, smem, stream>>>(a, alo, b, blo, args);
-  return cudaGetLastError();
+  // programmatic dependent launch: the grid may start during the preceding kernel; every
+  // role waits for it (griddepcontrol.wait) before touching data it may produce or read
+  return launch_pdl(kern, dim3(grid), dim3(Roles<BN>::kThreads), (size_t)smem, stream, a, alo, b, blo, args);
 }
 
-template <int BN, bool A_MN, bool B_MN, bool CORR_SWAP, bool A_PRE, bool B_PRE>
+template <int BN, bool A_MN, bool B_MN, bool CORR_SWAP, int A_PRE, int B_PRE>
 cudaError_t launch_fmt(int fmt, const CUtensorMap& a, const CUtensorMap& alo, const CUtensorMap& b,
                        const CUtensorMap& blo, const GemmArgs& args, int grid, cudaStream_t stream) {
   if (fmt == 0) return launch_variant<BN, A_MN, B_MN, 0, CORR_SWAP, A_PRE, B_PRE>(a, alo, b, blo, args, grid, stream);
@@ -840,21 +878,21 @@ cudaError_t launch_fmt(int fmt, const CUtensorMap& a, const CUtensorMap& alo, co
 
 // Swapped-operand skinny kernels: kernel-A = the weights (pre-split or FP32), kernel-B =
 // the M <= 64 activation rows padded to BN = 16 / 32 / 64.
-template <bool PRE>
+template <int PRE>
 cudaError_t launch_skinny(int BNk, bool b_mn, int fmt, const CUtensorMap& a, const CUtensorMap& alo,
                           const CUtensorMap& b, const CUtensorMap& blo, const GemmArgs& args, int grid,
                           cudaStream_t stream) {
   if (BNk == 16)
-    return b_mn ? launch_fmt<16, true, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream)
-                : launch_fmt<16, false, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream);
+    return b_mn ? launch_fmt<16, true, false, true, PRE, 0>(fmt, a, alo, b, blo, args, grid, stream)
+                : launch_fmt<16, false, false, true, PRE, 0>(fmt, a, alo, b, blo, args, grid, stream);
   if (BNk == 32)
-    return b_mn ? launch_fmt<32, true, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream)
-                : launch_fmt<32, false, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream);
-  return b_mn ? launch_fmt<64, true, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream)
-              : launch_fmt<64, false, false, true, PRE, false>(fmt, a, alo, b, blo, args, grid, stream);
+    return b_mn ? launch_fmt<32, true, false, true, PRE, 0>(fmt, a, alo, b, blo, args, grid, stream)
+                : launch_fmt<32, false, false, true, PRE, 0>(fmt, a, alo, b, blo, args, grid, stream);
+  return b_mn ? launch_fmt<64, true, false, true, PRE, 0>(fmt, a, alo, b, blo, args, grid, stream)
+              : launch_fmt<64, false, false, true, PRE, 0>(fmt, a, alo, b, blo, args, grid, stream);
 }
 
-template <bool B_MN, int FMT, bool B_PRE>
+template <bool B_MN, int FMT, int B_PRE>
 cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& blo, const GemmArgs& args,
                         int grid, cudaStream_t stream) {
   auto kern = heal_gemm_pair_kernel<B_MN, FMT, B_PRE>;
@@ -867,8 +905,25 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtens
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
   }
-  kern<<<grid, kPairThreads, kPairSmemBytes, stream>>>(a, b, blo, args);
-  return cudaGetLastError();
+  return launch_pdl(kern, dim3(grid), dim3(kPairThreads), (size_t)kPairSmemBytes, stream, a, b, blo, args);
+}
+
+template <int PRE>
+cudaError_t launch_pair_fmt(bool b_mn, int fmt, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& blo,
+                            const GemmArgs& args, int grid, cudaStream_t stream) {
+  if (fmt == 0)
+    return b_mn ? launch_pair<true, 0, PRE>(a, b, blo, args, grid, stream)
+                : launch_pair<false, 0, PRE>(a, b, blo, args, grid, stream);
+  return b_mn ? launch_pair<true, 1, PRE>(a, b, blo, args, grid, stream)
+              : launch_pair<false, 1, PRE>(a, b, blo, args, grid, stream);
+}
+
+// 128 x 128 tiles in the caller's operand order
+template <int PRE>
+cudaError_t launch_wide(bool b_mn, int fmt, const CUtensorMap& a, const CUtensorMap& alo, const CUtensorMap& b,
+                        const CUtensorMap& blo, const GemmArgs& args, int grid, cudaStream_t stream) {
+  return b_mn ? launch_fmt<128, false, true, false, 0, PRE>(fmt, a, alo, b, blo, args, grid, stream)
+              : launch_fmt<128, false, false, false, 0, PRE>(fmt, a, alo, b, blo, args, grid, stream);
 }
 
 }  // namespace
@@ -901,6 +956,8 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
   args.K = K;
   args.num_chunks = nc;
   args.chan_exp = o.chan_exp;
+  args.static_op = 0;
+  const int pre = o.b_presplit;   // 0 FP32 B, 1 pre-split hi + lo, 2 16-bit B (two products)
   args.status = device_status_ptr();
   cudaError_t err = cudaSuccess;
 
@@ -916,31 +973,15 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.expA_sign = -1;
     args.expB_sign = +1;
     if (!operand_map(&ta, A, false, false, M, K, lda, kPairRows)) return HEAL_ERR_CUDA;
-    if (!o.b_presplit) {
-      if (!operand_map(&tb, B, b_mn, false, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
-    } else {
-      if (!operand_map(&tb, B, b_mn, true, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
-      if (!operand_map(&tblo, o.b_lo, b_mn, true, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
-    }
+    if (!operand_map(&tb, B, b_mn, pre != 0, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
+    if (pre == 1 && !operand_map(&tblo, o.b_lo, b_mn, true, N, K, ldb, kPairRows)) return HEAL_ERR_CUDA;
     const long long pairs = (long long)args.tiles_m * args.tiles_n;
     const int max_pairs = sms / 2;
     const int grid = 2 * (int)(pairs < max_pairs ? pairs : max_pairs);
     if (grid < 2) return HEAL_ERR_CUDA;
-    if (!o.b_presplit) {
-      if (fmt == 0)
-        err = b_mn ? launch_pair<true, 0, false>(ta, tb, tblo, args, grid, stream)
-                   : launch_pair<false, 0, false>(ta, tb, tblo, args, grid, stream);
-      else
-        err = b_mn ? launch_pair<true, 1, false>(ta, tb, tblo, args, grid, stream)
-                   : launch_pair<false, 1, false>(ta, tb, tblo, args, grid, stream);
-    } else {
-      if (fmt == 0)
-        err = b_mn ? launch_pair<true, 0, true>(ta, tb, tblo, args, grid, stream)
-                   : launch_pair<false, 0, true>(ta, tb, tblo, args, grid, stream);
-      else
-        err = b_mn ? launch_pair<true, 1, true>(ta, tb, tblo, args, grid, stream)
-                   : launch_pair<false, 1, true>(ta, tb, tblo, args, grid, stream);
-    }
+    err = pre == 0 ? launch_pair_fmt<0>(b_mn, fmt, ta, tb, tblo, args, grid, stream)
+        : pre == 1 ? launch_pair_fmt<1>(b_mn, fmt, ta, tb, tblo, args, grid, stream)
+                   : launch_pair_fmt<2>(b_mn, fmt, ta, tb, tblo, args, grid, stream);
     return err == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
   }
 
@@ -956,28 +997,20 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.out_sj = 1;
     args.expA_sign = -1;
     args.expB_sign = +1;
+    args.static_op = o.b_static ? 2 : 0;   // kernel-B = B
     if (!operand_map(&ta, A, false, false, M, K, lda, kBM)) return HEAL_ERR_CUDA;
-    if (!o.b_presplit) {
-      if (!operand_map(&tb, B, b_mn, false, N, K, ldb, BN)) return HEAL_ERR_CUDA;
-    } else {
-      if (!operand_map(&tb, B, b_mn, true, N, K, ldb, BN)) return HEAL_ERR_CUDA;
-      if (!operand_map(&tblo, o.b_lo, b_mn, true, N, K, ldb, BN)) return HEAL_ERR_CUDA;
-    }
+    if (!operand_map(&tb, B, b_mn, pre != 0, N, K, ldb, BN)) return HEAL_ERR_CUDA;
+    if (pre == 1 && !operand_map(&tblo, o.b_lo, b_mn, true, N, K, ldb, BN)) return HEAL_ERR_CUDA;
     const int ntiles = args.tiles_m * args.tiles_n;
     const int grid = ntiles < sms ? ntiles : sms;
-    if (!o.b_presplit) {
-      err = b_mn ? launch_fmt<BN, false, true, false, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream)
-                 : launch_fmt<BN, false, false, false, false, false>(fmt, ta, talo, tb, tblo, args, grid, stream);
-    } else {
-      err = b_mn ? launch_fmt<BN, false, true, false, false, true>(fmt, ta, talo, tb, tblo, args, grid, stream)
-                 : launch_fmt<BN, false, false, false, false, true>(fmt, ta, talo, tb, tblo, args, grid, stream);
-    }
+    err = pre == 0 ? launch_wide<0>(b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
+        : pre == 1 ? launch_wide<1>(b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
+                   : launch_wide<2>(b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
     return err == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
   }
 
   if (cfg == HEAL_TILE_SKINNY_SPLITK || cfg == HEAL_TILE_SKINNY_FULLK) {
     const bool split = (cfg == HEAL_TILE_SKINNY_SPLITK);
-    const bool pre = o.b_presplit != 0;   // weights given as (hi, lo): kernel-A skips its split
     if (M > 64) return HEAL_ERR_UNSUPPORTED;
     if (split && (o.workspace == nullptr || o.workspace_bytes < gemm_workspace_bytes(M, N, K, cfg)))
       return HEAL_ERR_INVALID_ARGUMENT;
@@ -993,14 +1026,16 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.out_sj = ldc;
     args.expA_sign = +1;
     args.expB_sign = -1;
+    args.static_op = o.b_static ? 1 : 0;   // kernel-A = B^T
     const int BNk = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-    if (!operand_map(&ta, B, b_mn, pre, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
-    if (pre && !operand_map(&talo, o.b_lo, b_mn, true, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
+    if (!operand_map(&ta, B, b_mn, pre != 0, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
+    if (pre == 1 && !operand_map(&talo, o.b_lo, b_mn, true, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (!operand_map(&tb, A, false, false, M, K, lda, BNk)) return HEAL_ERR_CUDA;
     const long long units = split ? (long long)args.tiles_m * nc : (long long)args.tiles_m;
     const int grid = (int)(units < sms ? units : sms);
-    err = pre ? launch_skinny<true>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
-              : launch_skinny<false>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
+    err = pre == 0 ? launch_skinny<0>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
+        : pre == 1 ? launch_skinny<1>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
+                   : launch_skinny<2>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
     if (err != cudaSuccess) return HEAL_ERR_CUDA;
     if (!split) return HEAL_OK;
     const long long rblocks = (long long)((N + 31) / 32) * M;

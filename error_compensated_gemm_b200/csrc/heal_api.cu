@@ -111,7 +111,8 @@ heal_status_t heal_gemm_compensated(int M, int N, int K, const float* A, int64_t
   if (!A || !B || !C) return HEAL_ERR_INVALID_ARGUMENT;
   if (fmt != HEAL_SPLIT_FP16_S11 && fmt != HEAL_SPLIT_BF16) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.b_layout != 0 && o.b_layout != 1) return HEAL_ERR_INVALID_ARGUMENT;
-  if (o.b_presplit != 0 && o.b_presplit != 1) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.b_presplit < 0 || o.b_presplit > 2) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.b_static != 0 && o.b_static != 1) return HEAL_ERR_INVALID_ARGUMENT;
   for (int r : o.reserved)
     if (r != 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.tile_config < HEAL_TILE_AUTO || o.tile_config > HEAL_TILE_SKINNY_FULLK) return HEAL_ERR_INVALID_ARGUMENT;
@@ -121,7 +122,8 @@ heal_status_t heal_gemm_compensated(int M, int N, int K, const float* A, int64_t
   const int64_t b_min = o.b_layout == 0 ? N : K;
   if (ldb < b_min || ldb % (o.b_presplit ? 8 : 4) != 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (ldc < N) return HEAL_ERR_INVALID_ARGUMENT;
-  if (o.b_presplit && (!o.b_lo || !aligned(o.b_lo, 16))) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.b_presplit == 1 && (!o.b_lo || !aligned(o.b_lo, 16))) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.b_presplit == 2 && o.b_lo) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.chan_exp && !aligned(o.chan_exp, 1)) return HEAL_ERR_INVALID_ARGUMENT;
   const heal_status_t st = gemm_launch(M, N, K, A, lda, B, ldb, C, ldc, (int)fmt, o, (cudaStream_t)stream);
   if (st == HEAL_ERR_CUDA) (void)cudaGetLastError();

@@ -73,13 +73,27 @@ typedef struct {
                                summary, section 2.B, "Overflow Handling").  |e_k| <= 64.   */
   int b_layout;             /* 0: B is K x N row-major (ldb >= N); 1: B is N x K row-major
                                (ldb >= K), the torch.nn.Linear weight layout                 */
-  int b_presplit;           /* 1: `B` holds the 16-bit hi part and `b_lo` the lo part, both
-                               written by heal_split in `fmt`, in b_layout.  The kernel then
-                               splits only A.                                               */
-  const void* b_lo;         /* lo part when b_presplit = 1                                   */
+  int b_presplit;           /* 0: B is FP32 and is split by the kernel.
+                               1: `B` holds the 16-bit hi part and `b_lo` the lo part, both
+                                  written by heal_split in `fmt`, in b_layout; the kernel
+                                  splits only A (same bits as 0).
+                               2: `B` is a 16-bit matrix in fmt's 16-bit type (FP16 for
+                                  HEAL_SPLIT_FP16_S11, BF16 for HEAL_SPLIT_BF16) with no
+                                  residual: only A is split and C = Ah.B + s.Al.B, the
+                                  two-product form of the technical summary, section 2.B
+                                  (16-bit weights, half the weight bytes); b_lo must be null.
+                               With 1 or 2 the kernel applies chan_exp to A only: B's rows
+                               must already carry the factor 2^e_k.                         */
+  const void* b_lo;         /* lo part when b_presplit = 1, else null                        */
   void* workspace;          /* device scratch for HEAL_TILE_SKINNY_SPLITK (nullable)        */
   size_t workspace_bytes;
-  int reserved[4];          /* must be zero                                                  */
+  int b_static;             /* 1: B (and b_lo) are not written by work queued before this call
+                               on the stream (weights).  GEMM kernels start with programmatic
+                               dependent launch and wait for the preceding kernel before they
+                               touch A, chan_exp, C or the workspace; with b_static they may
+                               request the first stages of B before that wait.  0: B is
+                               waited for like A.                                           */
+  int reserved[3];          /* must be zero                                                  */
 } heal_gemm_opts_t;
 
 /* K1. Hi/lo split of n FP32 values (technical summary, section 2.B, "Mechanism").

@@ -17,6 +17,10 @@ Functions:
                     in float64 from the oracle's own split -- the method's steps.
                     (three products; the lo*lo term is dropped.)
   truncation_term   closed form of C_emul - C_ref from the split residuals.
+  to_16bit          the 16-bit form of a weight matrix (FP16 or BF16 per the format).
+  gemm_two_product  C = Ah W16 + s Al W16: the section's own two-product form, in which
+                    only the activations are split and the weights are 16-bit values.
+  two_product_truncation  closed form of gemm_two_product - A @ W16.
   gemm_bf16_downcast  plain 16-bit GEMM with a BF16 store of the FP32 result: the
                     boundary-truncation negative control.
   rescale_channels  per-K-channel power-of-two rescale (exact).
@@ -76,6 +80,42 @@ def truncation_term(A, B, fmt=_split.FP16_S11, chan_exp=None):
     Ar = np.asarray(A, np.float64) - A1
     Br = np.asarray(B, np.float64) - B1
     return -(s * s * (Al @ Bl) + A1 @ Br + Ar @ np.asarray(B, np.float64))
+
+
+def to_16bit(B, fmt=_split.FP16_S11):
+    """B rounded to the format's 16-bit type (nearest even), returned as float64."""
+    B = np.asarray(B, np.float32)
+    if fmt == _split.FP16_S11:
+        with np.errstate(over="ignore"):
+            return _split.to_fp16(B).astype(np.float64)
+    return _split.to_bf16_as_f32(B).astype(np.float64)
+
+
+def gemm_two_product(A, W16, fmt=_split.FP16_S11, chan_exp=None):
+    """Two-product compensated GEMM in float64: C = Ah W16 + s Al W16.
+
+    The technical summary (section 2.B, "Mechanism") splits the input activations into a
+    16-bit value and a residual and runs two 16-bit products whose results are added;
+    the weights W16 are already 16-bit values (exactly representable), so they carry no
+    residual.  With chan_exp, column k of A is scaled by 2^-e_k and row k of W16 by 2^e_k.
+    """
+    A = np.asarray(A, np.float32)
+    W16 = np.asarray(W16, np.float64)
+    if chan_exp is not None:
+        e = np.asarray(chan_exp, np.int64)
+        A = np.ldexp(A.astype(np.float64), -e[None, :]).astype(np.float32)
+        W16 = np.ldexp(W16, e[:, None])
+    Ah, Al, _, _ = _split.split(A, fmt)
+    s = 1.0 / _split.LO_SCALE[fmt]
+    return Ah @ W16 + s * (Al @ W16)
+
+
+def two_product_truncation(A, W16, fmt=_split.FP16_S11):
+    """gemm_two_product - A @ W16 = -Ar @ W16 with Ar = A - (Ah + s Al)."""
+    Ah, Al, _, _ = _split.split(np.asarray(A, np.float32), fmt)
+    s = 1.0 / _split.LO_SCALE[fmt]
+    Ar = np.asarray(A, np.float32).astype(np.float64) - (Ah + s * Al)
+    return -(Ar @ np.asarray(W16, np.float64))
 
 
 def gemm_bf16_downcast(A, B):

@@ -13,7 +13,7 @@ import error_compensated_gemm_b200 as heal
 import synthetic
 from oracle import gemm as G
 from oracle import split as S
-from tests.gpu_helpers import dev, gemm, status_ok
+from tests.gpu_helpers import dev, gemm, status_ok, to_np
 
 pytestmark = pytest.mark.gpu
 TOL_FP16 = 1e-6
@@ -187,3 +187,89 @@ def test_cta_pair_presplit_and_bf16(fmt):
     c_in = gemm(X.numpy(), W.numpy(), fmt=fmt, tile=heal.TILE_256x256_PAIR)
     c_single = gemm(X.numpy(), W.numpy(), fmt=fmt, tile=heal.TILE_128x128)
     assert np.array_equal(c_pre, c_in) and np.array_equal(c_in, c_single)
+
+
+@pytest.mark.parametrize("M", [1, 8, 64, 300])
+@pytest.mark.parametrize("presplit", [False, True])
+def test_back_to_back_dependent_chain(M, presplit):
+    """Programmatic dependent launch: each call's A is the previous call's C and all calls
+    share one workspace, issued back to back with weights declared static.  The chain must
+    give the bits of the same calls separated by a device synchronisation."""
+    d = dev()
+    K = N = 1024
+    X = synthetic.normal((M, K), seed=21).to(d)
+    Ws = [(0.03 * synthetic.normal((K, N), seed=30 + i)).to(d) for i in range(4)]
+    pre = []
+    for W in Ws:
+        hi = torch.empty(W.shape, dtype=torch.int16, device=d)
+        lo = torch.empty(W.shape, dtype=torch.int16, device=d)
+        heal.heal_split(W, hi, lo)
+        pre.append((hi, lo))
+    ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(M, N, K, heal.TILE_SKINNY_SPLITK) // 4), device=d)
+    use_ws = ws if M <= 64 else None
+
+    def run(sync):
+        outs = []
+        a = X
+        for i, W in enumerate(Ws):
+            c = torch.full((M, N), float("nan"), device=d)
+            if presplit:
+                heal.heal_gemm_compensated(a, pre[i][0], c, b_lo=pre[i][1], workspace=use_ws, b_static=True)
+            else:
+                heal.heal_gemm_compensated(a, W, c, workspace=use_ws, b_static=True)
+            if sync:
+                torch.cuda.synchronize()
+            outs.append(c)
+            a = c
+        torch.cuda.synchronize()
+        return [to_np(o) for o in outs]
+
+    ref = run(True)
+    for _ in range(3):
+        got = run(False)
+        for r, g in zip(ref, got):
+            assert np.array_equal(r.view(np.uint32), g.view(np.uint32))
+    status_ok()
+    # the chain is the plain product of the inputs (first link against the oracle)
+    assert G.normwise_rel_err(ref[0].astype(np.float64), G.gemm_ref(to_np(X), to_np(Ws[0]))) <= TOL_FP16
+
+
+def _gemm16(X, W16, fmt, tile, b_layout=0):
+    """Two-product GEMM on device copies: X FP32 [M,K], W16 a 16-bit torch tensor ([K,N] or [N,K])."""
+    d = dev()
+    Xd = X.to(d).contiguous()
+    Wd = W16.to(d).contiguous()
+    M, K = Xd.shape
+    N = Wd.shape[1] if b_layout == 0 else Wd.shape[0]
+    C = torch.full((M, N), float("nan"), device=d)
+    ws = None
+    nbytes = heal.heal_gemm_workspace_bytes(M, N, K, tile)
+    if nbytes:
+        ws = torch.empty(nbytes // 4, dtype=torch.float32, device=d)
+    heal.heal_gemm_compensated(Xd, Wd, C, fmt=fmt, tile_config=tile, b_layout=b_layout, b_16bit=True, workspace=ws)
+    status_ok()
+    return to_np(C).astype(np.float64)
+
+
+@pytest.mark.parametrize("fmt", [heal.SPLIT_FP16_S11, heal.SPLIT_BF16])
+@pytest.mark.parametrize("b_layout", [0, 1])
+@pytest.mark.parametrize("M", [1, 8, 64, 300])
+def test_two_product_16bit_weights(fmt, b_layout, M):
+    """The pages' two-product form: 16-bit weights, only the activations split.  Against the
+    FP64 product with those 16-bit weights; identical bits in every tile configuration."""
+    K, N = 1000, 648
+    X, W = synthetic.gemm_decode(M, K=K, N=N)
+    W16 = W.half() if fmt == heal.SPLIT_FP16_S11 else W.bfloat16()
+    ref = G.gemm_ref(X.numpy(), W16.float().numpy())
+    Bin = W16 if b_layout == 0 else W16.t().contiguous()
+    tiles = [heal.TILE_128x128, heal.TILE_256x256_PAIR] + (
+        [heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK] if M <= 64 else [])
+    outs = [_gemm16(X, Bin, fmt, t, b_layout) for t in tiles]
+    for o in outs[1:]:
+        assert np.array_equal(o, outs[0])
+    tol = TOL_FP16 if fmt == heal.SPLIT_FP16_S11 else 2e-5
+    assert G.normwise_rel_err(outs[0], ref) <= tol
+    # and the oracle's own two-product emulation agrees to the accumulation level
+    emu = G.gemm_two_product(X.numpy(), W16.float().numpy().astype(np.float64),
+                             S.FP16_S11 if fmt == heal.SPLIT_FP16_S11 else S.BF16)
+    assert G.normwise_rel_err(outs[0], emu) <= (5e-7 if fmt == heal.SPLIT_FP16_S11 else 2e-5)

@@ -124,3 +124,46 @@ def test_gemm_ref_matches_scalar_loop():
         for j in range(3):
             exact = sum(Fraction(float(A[i, t])) * Fraction(float(B[t, j])) for t in range(37))
             assert abs(float(exact) - ref[i, j]) <= 1e-13 * max(1.0, abs(float(exact)))
+
+
+@pytest.mark.parametrize("shape", [(2, 3, 2), (4, 8, 3)])
+@pytest.mark.parametrize("fmt", [S.FP16_S11, S.BF16])
+def test_two_product_identity_exact(shape, fmt):
+    """Two-product form (technical summary 2.B): only A is split and the 16-bit weights carry
+    no residual.  Exact rational check of C_two - A @ W16 = -Ar @ W16 with Ar = A - Ah - s Al,
+    on random FP32 A (whose split leaves a nonzero Ar) and dyadic 16-bit weights."""
+    n, k, m = shape
+    rng = np.random.default_rng(7 * n + k)
+    A = rng.standard_normal((n, k)).astype(np.float32)
+    W16 = dyadic((k, m), rng)
+    two = G.gemm_two_product(A, W16, fmt)
+    Ah, Al, _, _ = S.split(A, fmt)
+    s = Fraction(1) / Fraction(int(S.LO_SCALE[fmt]))
+    exactA = [[Fraction(float(v)) for v in row] for row in A.astype(np.float64)]
+    emulA = [[Fraction(float(Ah[i, t])) + s * Fraction(float(Al[i, t])) for t in range(k)] for i in range(n)]
+    Wf = [[Fraction(float(v)) for v in row] for row in W16.astype(np.float64)]
+    assert any(exactA[i][t] != emulA[i][t] for i in range(n) for t in range(k)), "Ar must be nonzero somewhere"
+    trunc = G.two_product_truncation(A, W16, fmt)
+    for i in range(n):
+        for j in range(m):
+            c_emul = sum(emulA[i][t] * Wf[t][j] for t in range(k))
+            c_exact = sum(exactA[i][t] * Wf[t][j] for t in range(k))
+            # the float64 evaluation of the small dyadic products is exact
+            assert Fraction(float(two[i, j])) == c_emul
+            assert abs(float(trunc[i, j]) - float(c_emul - c_exact)) <= 1e-15 * max(1.0, abs(float(c_exact)))
+
+
+def test_two_product_error_levels():
+    """Against the product with the 16-bit weights, the two-product form is at the level of
+    the activation split (FP16: ~1e-7; BF16: ~1e-5); against the FP32 weights it is limited
+    by the 16-bit rounding of the weights themselves (~1e-4 for FP16)."""
+    X, W = synthetic.gemm_decode(16, K=512, N=256)
+    X, W = X.numpy(), W.numpy()
+    W16 = G.to_16bit(W, S.FP16_S11)
+    e16 = G.normwise_rel_err(G.gemm_two_product(X, W16, S.FP16_S11), G.gemm_ref(X, W16))
+    assert e16 < 2e-7
+    Wb = G.to_16bit(W, S.BF16)
+    eb = G.normwise_rel_err(G.gemm_two_product(X, Wb, S.BF16), G.gemm_ref(X, Wb))
+    assert 1e-7 < eb < 2e-5
+    e_w = G.normwise_rel_err(G.gemm_two_product(X, W16, S.FP16_S11), G.gemm_ref(X, W))
+    assert 1e-5 < e_w < 1e-3
