@@ -783,46 +783,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 }
 
 // Ordered sum of chunk values: out(i, j) = ((ws[0] + ws[1]) + ws[2]) + ...
-// One block per 32 consecutive i of one j: the block stages the chunk values of those 32
-// outputs (pieces of up to kRedChunks chunks, coalesced 128-byte rows) in shared memory,
-// then 32 threads add them in ascending chunk order, carrying the sum across pieces.
-constexpr int kRedChunks = 128;
+// One thread per output; a warp covers 32 consecutive i of one j, so every chunk row it
+// reads is one coalesced 128-byte line.  Each thread requests kRedBatch chunk values at once
+// (registers, no shared memory), then adds them in ascending chunk order.  Without shared
+// memory the blocks fit beside a resident GEMM CTA: launched with programmatic dependent
+// launch they are already on the SMs, waiting, when the GEMM grid finishes, and the next
+// GEMM's CTAs can start next to them.
+constexpr int kRedBatch = 32;
 __global__ void __launch_bounds__(256) heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk,
                                                                 int Nk, float* out, long long si, long long sj) {
-  __shared__ float tile[kRedChunks][33];
   pdl_launch_dependents();   // the next kernel may be scheduled; it waits for this grid
-  pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed   // the GEMM kernel that wrote ws has completed
-  const int tiles_i = (Mk + 31) / 32;
-  const int ti = blockIdx.x % tiles_i, j = blockIdx.x / tiles_i;
-  const int i0 = ti * 32;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed
+  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  if (idx >= (long long)Mk * Nk) return;
+  const int i = (int)(idx % Mk), j = (int)(idx / Mk);
   const size_t plane = (size_t)Mk * Nk;
-  const float* base = ws + (size_t)j * Mk + i0;
+  const float* p = ws + (size_t)j * Mk + i;
   float acc = 0.0f;
-  for (int c0 = 0; c0 < num_chunks; c0 += kRedChunks) {
-    const int cn = min(kRedChunks, num_chunks - c0);
-    __syncthreads();
-    for (int c = warp; c < cn; c += 8)
-      tile[c][lane] = (i0 + lane < Mk) ? __ldcs(base + (size_t)(c0 + c) * plane + lane) : 0.0f;
-    __syncthreads();
-    if (warp == 0) {
-      int c = 0;
-      if (c0 == 0) {
-        acc = tile[0][lane];
-        c = 1;
-      }
-      // 16 values at a time into registers, then added in ascending chunk order
-      for (; c + 16 <= cn; c += 16) {
-        float v[16];
+  for (int c0 = 0; c0 < num_chunks; c0 += kRedBatch) {
+    const int cn = min(kRedBatch, num_chunks - c0);
+    float v[kRedBatch];
 #pragma unroll
-        for (int t = 0; t < 16; ++t) v[t] = tile[c + t][lane];
+    for (int t = 0; t < kRedBatch; ++t) v[t] = t < cn ? __ldcs(p + (size_t)(c0 + t) * plane) : 0.0f;
 #pragma unroll
-        for (int t = 0; t < 16; ++t) acc = __fadd_rn(acc, v[t]);
-      }
-      for (; c < cn; ++c) acc = __fadd_rn(acc, tile[c][lane]);
-    }
+    for (int t = 0; t < kRedBatch; ++t)
+      if (t < cn) acc = (c0 + t == 0) ? v[t] : __fadd_rn(acc, v[t]);
   }
-  if (warp == 0 && i0 + lane < Mk) out[(size_t)(i0 + lane) * si + (size_t)j * sj] = acc;
+  out[(size_t)i * si + (size_t)j * sj] = acc;
 }
 
 // ---------------------------------------------------------------------------------
@@ -1038,7 +1025,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
                    : launch_skinny<2>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
     if (err != cudaSuccess) return HEAL_ERR_CUDA;
     if (!split) return HEAL_OK;
-    const long long rblocks = (long long)((N + 31) / 32) * M;
+    const long long rblocks = ((long long)N * M + 255) / 256;
     if (rblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
     const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(256), 0, stream,
                                      (const float*)args.ws, nc, N, M, Cout, 1LL, (long long)ldc);
