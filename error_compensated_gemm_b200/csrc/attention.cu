@@ -127,6 +127,13 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t&
                : "r"(addr));
 }
 
+// x * 2^e for |e| <= 252 in two exact power-of-two steps (a single factor 2^e would
+// overflow or underflow FP32 for |e| > 126, which extreme V scales can reach).
+__device__ __forceinline__ float mul_pow2(float x, int e) {
+  const int e1 = e / 2, e2 = e - e1;   // each in [-126, 126]
+  return __fmul_rn(__fmul_rn(x, __int_as_float((127 + e1) << 23)), __int_as_float((127 + e2) << 23));
+}
+
 __device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kCompute * 32) : "memory"); }
 
 __device__ __forceinline__ long long unit_begin(long long total, int grid, int c) {
@@ -268,11 +275,10 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
       f[h] = (mw == -INFINITY) ? 0.0f : exp2f(mw - mx);
     }
     // O of this warp, scaled to the CTA max, in true units (x 2^-E_run), in place
-    const float u = ldexpf(1.0f, -E_run);
 #pragma unroll
     for (int dt = 0; dt < D / 16; ++dt)
 #pragma unroll
-      for (int e = 0; e < 4; ++e) om[dt][e] = __fmul_rn(__fmul_rn(om[dt][e], u), f[e & 1]);
+      for (int e = 0; e < 4; ++e) om[dt][e] = __fmul_rn(mul_pow2(om[dt][e], -E_run), f[e & 1]);
     // sequential, fixed-order merge of the four warps through shared memory
     for (int w = 0; w < kCompute; ++w) {
       if (warp == w) {
@@ -374,7 +380,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
     const int tw = warp * 16;                 // this warp's first token inside the tile
 
     // ---- exact S^T = K Q^T on the byte-split operands (integer tensor cores) ----
-    int shh[4] = {0, 0, 0, 0}, sx[4] = {0, 0, 0, 0}, sll[4] = {0, 0, 0, 0};
+    // S_x in two accumulators (kh.ql and kl.qh) so no MMA chain is longer than the k32 steps
+    int shh[4] = {0, 0, 0, 0}, sxa[4] = {0, 0, 0, 0}, sxb[4] = {0, 0, 0, 0}, sll[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int s32 = 0; s32 < kKSteps32; ++s32) {
       const uint4 qf = qf_sm[s32 * 32 + lane];
@@ -392,8 +399,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
       const uint32_t al0 = lo_bytes(r[0][0], r[0][1]), al1 = lo_bytes(r[1][0], r[1][1]);
       const uint32_t al2 = lo_bytes(r[0][2], r[0][3]), al3 = lo_bytes(r[1][2], r[1][3]);
       imma16832<false, false>(shh, ah0, ah1, ah2, ah3, qf.x, qf.y);
-      imma16832<false, true>(sx, ah0, ah1, ah2, ah3, qf.z, qf.w);
-      imma16832<true, false>(sx, al0, al1, al2, al3, qf.x, qf.y);
+      imma16832<false, true>(sxa, ah0, ah1, ah2, ah3, qf.z, qf.w);
+      imma16832<true, false>(sxb, al0, al1, al2, al3, qf.x, qf.y);
       imma16832<true, true>(sll, al0, al1, al2, al3, qf.z, qf.w);
     }
     // every ldmatrix of the K tile has been consumed by the MMAs above and the K scales
@@ -412,7 +419,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
         const int i = 2 * th + e;
         const int t = t0 + tw + th * 8 + g8;
         const int r = qc + e;
-        const long long S = ((long long)shh[i] << 16) + ((long long)sx[i] << 8) + (long long)sll[i];
+        const long long S = ((long long)shh[i] << 16) + (((long long)sxa[i] + (long long)sxb[i]) << 8) +
+                            (long long)sll[i];
         const bool real = r < R;
         const bool vis = real && t < klen && (!a.causal || t <= pos[e]);
         float xv;
@@ -459,13 +467,15 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
       m_run[e] = m_new;
     }
     // power of two for this block: the largest visible V scale times 2^E in [32, 64)
-    float smax = 0.0f;
+    // (V scales are non-negative, so their bit patterns order like the floats: one
+    // warp-wide integer max gives the block maximum)
+    float smax;
     {
       const int ta = t0 + lane, tb = t0 + 32 + lane;
-      if (ta < klen) smax = svs[lane];
-      if (tb < klen) smax = fmaxf(smax, svs[32 + lane]);
-#pragma unroll
-      for (int o = 16; o >= 1; o >>= 1) smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, o));
+      unsigned int um = 0u;
+      if (ta < klen) um = __float_as_uint(svs[lane]);
+      if (tb < klen) um = max(um, __float_as_uint(svs[32 + lane]));
+      smax = __uint_as_float(__reduce_max_sync(0xffffffffu, um));
     }
     float escale = 1.0f;                       // 2^(E_new - E_run) applied to O
     if (smax > 0.0f) {
@@ -494,15 +504,14 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
     // ---- P' = P * s_v * 2^E (S^T layout), moved to the B layout of PV: lane (g8, c)
     // needs tokens 2c, 2c + 1, 2c + 8, 2c + 9 of query row g8.  Token 2c + j lives in lane
     // 4 * (2c + j) + g8 / 2 (halves th = 0 / 1 for +0 / +8), query row g8 in its slot g8 & 1.
-    const float e2 = ldexpf(1.0f, E_run);
     float pp[2][2];
 #pragma unroll
     for (int th = 0; th < 2; ++th) {
       const int t = t0 + tw + th * 8 + g8;
-      const float svt = svs[t - t0];
+      const float svt = mul_pow2(svs[t - t0], E_run);   // s_v * 2^E, in [0, 64)
 #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float sv = (pv[th][e] != 0.0f) ? __fmul_rn(svt, e2) : 0.0f;
+        const float sv = (pv[th][e] != 0.0f) ? svt : 0.0f;
         pp[th][e] = __fmul_rn(pv[th][e], sv);
       }
     }

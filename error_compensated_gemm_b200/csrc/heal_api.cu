@@ -125,6 +125,7 @@ heal_status_t heal_gemm_compensated(int M, int N, int K, const float* A, int64_t
   if (o.b_presplit == 1 && (!o.b_lo || !aligned(o.b_lo, 16))) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.b_presplit == 2 && o.b_lo) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.chan_exp && !aligned(o.chan_exp, 1)) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.workspace && !aligned(o.workspace, 16)) return HEAL_ERR_INVALID_ARGUMENT;
   const heal_status_t st = gemm_launch(M, N, K, A, lda, B, ldb, C, ldc, (int)fmt, o, (cudaStream_t)stream);
   if (st == HEAL_ERR_CUDA) (void)cudaGetLastError();
   return st;

@@ -29,7 +29,8 @@ def test_library_loads_and_exports_every_symbol():
 
 
 def test_workspace_queries_are_host_only():
-    assert heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK) == 64 * 4096 * 4
+    # chunk values [64][1][4096] FP32, then one 64-bit flag per CTA (room for 1024 CTAs)
+    assert heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK) == 64 * 4096 * 4 + 1024 * 8
     assert heal.heal_gemm_workspace_bytes(4096, 4096, 4096, heal.TILE_128x128) == 0
     assert heal.heal_attention_workspace_bytes(8, 32, 1, 8192) > 0
     assert heal.heal_attention_workspace_bytes(0, 32, 1, 8192) == 0
@@ -46,6 +47,21 @@ def test_invalid_arguments_rejected_before_launch():
     assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 4, fake, 4, 7, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
     o.reserved[0] = 1
     assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 4, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.reserved[0] = 0
+    o.b_static = 2                                   # only 0 / 1
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 8, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.b_static = 0
+    o.b_presplit = 3                                 # only 0 / 1 / 2
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 8, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.b_presplit = 1                                 # pre-split B needs its lo part
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 8, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.b_presplit = 2                                 # a 16-bit B has no lo part
+    o.b_lo = 1 << 20
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 8, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.b_lo = None
+    assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 4, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT  # ldb % 8
+    with pytest.raises(ValueError):
+        heal.gemm_opts(b_lo=object(), b_16bit=True)
     assert L.heal_split(fake, fake, fake, -1, 0, None) == heal.HEAL_ERR_INVALID_ARGUMENT
     assert L.heal_split(None, None, None, 0, 0, None) == heal.HEAL_OK       # n == 0 is a no-op
     assert L.heal_kv_quantize_int16(fake, 1, 1, 1, 1, 96, 96, 96, 96, fake, fake, 1, 0, None) == heal.HEAL_ERR_UNSUPPORTED

@@ -120,6 +120,19 @@ def test_extreme_int16_values_exact_dots():
     check(q, qs, kq, kss, vq, vss, [T], 0.5)
 
 
+def test_extreme_v_scales():
+    """V scales from 3e-38 up to 3e33: the per-block power of two 2^E that brings the largest
+    V scale into [32, 64) then lies outside FP32's normal range on both ends; the kernel applies
+    it in two exact steps.  Blocks of tiny and huge scales alternate, so E also moves down."""
+    B, Hq, Hkv, D, T = 1, 4, 1, 128, 320
+    q, qs, kq, kss, vq, vss = make_inputs(B=B, Hq=Hq, Hkv=Hkv, D=D, T=T)
+    vss = vss.copy()
+    vss[0, 0, :128] *= np.float32(3e-38 / float(vss[0, 0, :128].max()))   # first two blocks: tiny
+    vss[0, 0, 192:256] *= np.float32(3e33 / float(vss[0, 0, 192:256].max()))   # fourth block: huge
+    assert np.all(np.isfinite(vss))
+    check(q, qs, kq, kss, vq, vss, [T], D ** -0.5)
+
+
 def test_repeat_runs_bitwise_identical():
     q, qs, kq, kss, vq, vss = make_inputs(B=2, Hq=8, Hkv=2, D=128, T=1024)
     a, _ = run_gpu(q, qs, kq, kss, vq, vss, [1024, 900], 128 ** -0.5)
