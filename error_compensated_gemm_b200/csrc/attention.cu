@@ -569,6 +569,10 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
 }
 
 // out[b, hq, tq, :] = sum_c o_c 2^(m_c - M) / sum_c l_c 2^(m_c - M), c ascending.
+// The partials of kCombBatch CTAs are requested together (independent loads) and then
+// applied one by one in ascending CTA order, so the sums are the same as a one-at-a-time
+// loop while the number of dependent memory round trips drops by kCombBatch.
+constexpr int kCombBatch = 8;
 template <int D>
 __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) {
   pdl_wait_prerequisites();             // the decode kernel that wrote the partials has completed
@@ -578,15 +582,32 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
   const long long ufirst = (long long)p * a.nblk, ulast = ufirst + a.nblk - 1;
   const int c0 = cta_of(ufirst, a.total, a.grid), c1 = cta_of(ulast, a.total, a.grid);
   float M = -INFINITY;
-  for (int c = c0; c <= c1; ++c) M = fmaxf(M, slot_ptr(a.ws, c, p, a.R, D)[a.R * D + 2 * r]);
+  for (int cb = c0; cb <= c1; cb += kCombBatch) {
+    float m[kCombBatch];
+#pragma unroll
+    for (int t = 0; t < kCombBatch; ++t)
+      m[t] = (cb + t <= c1) ? slot_ptr(a.ws, cb + t, p, a.R, D)[a.R * D + 2 * r] : -INFINITY;
+#pragma unroll
+    for (int t = 0; t < kCombBatch; ++t) M = fmaxf(M, m[t]);
+  }
   float L = 0.0f, O = 0.0f;
-  for (int c = c0; c <= c1; ++c) {
-    const float* sl = slot_ptr(a.ws, c, p, a.R, D);
-    const float m = sl[a.R * D + 2 * r];
-    if (m == -INFINITY) continue;
-    const float f = exp2f(m - M);
-    L = __fadd_rn(L, __fmul_rn(sl[a.R * D + 2 * r + 1], f));
-    O = __fadd_rn(O, __fmul_rn(sl[r * D + d], f));
+  for (int cb = c0; cb <= c1; cb += kCombBatch) {
+    float m[kCombBatch], l[kCombBatch], o[kCombBatch];
+#pragma unroll
+    for (int t = 0; t < kCombBatch; ++t) {
+      const bool in = cb + t <= c1;
+      const float* sl = slot_ptr(a.ws, in ? cb + t : c0, p, a.R, D);
+      m[t] = in ? sl[a.R * D + 2 * r] : -INFINITY;
+      l[t] = in ? sl[a.R * D + 2 * r + 1] : 0.0f;
+      o[t] = in ? sl[r * D + d] : 0.0f;
+    }
+#pragma unroll
+    for (int t = 0; t < kCombBatch; ++t) {
+      if (m[t] == -INFINITY) continue;
+      const float f = exp2f(m[t] - M);
+      L = __fadd_rn(L, __fmul_rn(l[t], f));
+      O = __fadd_rn(O, __fmul_rn(o[t], f));
+    }
   }
   const int b = p / a.Hkv, hkv = p % a.Hkv;
   const int tq = r / a.G, g = r % a.G;

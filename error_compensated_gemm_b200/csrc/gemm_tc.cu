@@ -31,9 +31,6 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
-#include <atomic>
-#include <random>
-
 #include "heal_internal.h"
 #include "heal_ptx.cuh"
 #include "heal_split.cuh"
@@ -67,8 +64,6 @@ struct GemmArgs {
   int expA_sign, expB_sign; // +1 / -1: which operand gets 2^+e and which 2^-e
   int static_op;            // 0: none; 1: kernel-A, 2: kernel-B is not written by the kernels
                             // before this one (its first stages may be requested early)
-  unsigned long long* flags;  // split-K with the ordered sum in this kernel: one flag per CTA,
-  unsigned long long seq;     // set to seq once all of the CTA's chunk values are written
   unsigned int* status;     // device status word
 };
 
@@ -297,11 +292,10 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   uint64_t* mma_done = bars + 3 * S + 4; // MMA drain on exit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
-  uint64_t* epi_done = bars + 3 * S + 8;  // epilogue threads -> flag writer (128 arrivals)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  pdl_launch_dependents();   // a following kernel may be scheduled; it waits for us
+  pdl_launch_dependents();   // a following reduce kernel may be scheduled; it waits for us
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -313,7 +307,6 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kNumEpiWarps * 32);
     }
-    mbar_init(epi_done, kNumEpiWarps * 32);
     mbar_init(mma_done, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -525,75 +518,7 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
         }
       }
     }
-    if (ok && args.splitk && args.flags != nullptr) {
-      // Ordered sum of the chunk values in this kernel (small M).  First publish this CTA's
-      // chunk values: every epilogue thread fences its stores and arrives; one thread waits
-      // (bounded) for all of them and sets the CTA's flag to this call's tag.
-      __threadfence();
-      mbar_arrive(epi_done);
-      if (threadIdx.x == kEpiWarp0 * 32 && mbar_wait(epi_done, 0, abort_flag, args.status, 131))
-        st_release_gpu_u64(args.flags + blockIdx.x, args.seq);
-      // Then reduce a slice of the outputs, 32 consecutive i per warp: for each output tile
-      // the warp waits until every CTA whose unit range overlaps the tile has published
-      // (one lane per CTA, bounded), then adds the chunk values in ascending order, exactly
-      // as heal_chunk_reduce_kernel does.
-      const int ew = warp - kEpiWarp0;
-      const long long total = (long long)args.Mk * args.Nk;
-      const long long s0 = total * blockIdx.x / gridDim.x, s1 = total * (blockIdx.x + 1) / gridDim.x;
-      const size_t plane = (size_t)args.Mk * args.Nk;
-      const int nc = args.num_chunks;
-      const long long units = (long long)args.tiles_m * args.tiles_n * nc;
-      int ready_lo = 0, ready_hi = -1;         // tiles [ready_lo, ready_hi] verified
-      bool good = true;
-      for (long long base = s0 + (long long)ew * 32; base < s1 && good; base += kNumEpiWarps * 32) {
-        const long long idx = base + lane;
-        const bool mine = idx < s1;
-        const int i = mine ? (int)(idx % args.Mk) : 0, j = mine ? (int)(idx / args.Mk) : 0;
-        // tiles touched by this group of 32 outputs
-        const int t_lo = __reduce_min_sync(0xffffffffu, mine ? (unsigned)(i / kBM) : 0x7fffffffu);
-        const int t_hi = __reduce_max_sync(0xffffffffu, mine ? (unsigned)(i / kBM) : 0u);
-        if (t_lo < ready_lo || t_hi > ready_hi) {
-          // CTAs that hold units of tiles t_lo .. t_hi
-          const long long u_a = (long long)t_lo * nc, u_b = (long long)(t_hi + 1) * nc - 1;
-          int c_a = (int)((u_a * gridDim.x) / units), c_b = (int)((u_b * gridDim.x) / units);
-          while (c_a > 0 && units * c_a / gridDim.x > u_a) --c_a;
-          while (c_b + 1 < (int)gridDim.x && units * (c_b + 1) / gridDim.x <= u_b) ++c_b;
-          for (int c0 = c_a; c0 <= c_b && good; c0 += 32) {
-            const int cc = c0 + lane;
-            const bool need = cc <= c_b;
-            const uint64_t t0 = globaltimer();
-            while (true) {
-              const bool ready = !need || *reinterpret_cast<volatile unsigned long long*>(args.flags + cc) == args.seq;
-              if (__all_sync(0xffffffffu, ready)) break;
-              // the decision to give up is taken by the whole warp at once
-              if (__any_sync(0xffffffffu, *abort_flag != 0 || globaltimer() - t0 > kWaitLimitNs)) {
-                if (lane == 0 && !*abort_flag) {
-                  *abort_flag = 1;
-                  report_timeout(args.status, 132);
-                }
-                good = false;
-                break;
-              }
-            }
-          }
-          __threadfence();   // acquire: the chunk values published with the flags are visible
-          ready_lo = t_lo;
-          ready_hi = t_hi;
-        }
-        if (!good || !mine) continue;
-        const float* p = args.ws + (size_t)j * args.Mk + i;
-        float sum = 0.0f;
-        for (int c0 = 0; c0 < nc; c0 += 32) {
-          float v[32];
-#pragma unroll
-          for (int t = 0; t < 32; ++t) v[t] = (c0 + t < nc) ? __ldcg(p + (size_t)(c0 + t) * plane) : 0.0f;
-#pragma unroll
-          for (int t = 0; t < 32; ++t)
-            if (c0 + t < nc) sum = (c0 + t == 0) ? v[t] : __fadd_rn(sum, v[t]);
-        }
-        args.out[(size_t)i * args.out_si + (size_t)j * args.out_sj] = sum;
-      }
-    }
+    (void)ok;
   }
 
   tc_fence_before();
@@ -990,28 +915,12 @@ cudaError_t launch_wide(bool b_mn, int fmt, const CUtensorMap& a, const CUtensor
 
 }  // namespace
 
-// Split-K workspace: the chunk values [nc][M][N] FP32, then (8-byte aligned) one 64-bit
-// flag per CTA (at most kMaxFlagCtas) for the in-kernel ordered sum.
-static size_t partial_bytes(int M, int N, int K) {
-  const size_t nc = (size_t)((K + kBK - 1) / kBK);
-  return (nc * (size_t)M * (size_t)N * sizeof(float) + 7) & ~(size_t)7;
-}
-constexpr int kMaxFlagCtas = 1024;
-static size_t flag_count(int, int) { return (size_t)kMaxFlagCtas; }
-
 size_t gemm_workspace_bytes(int M, int N, int K, int tile_config) {
   if (tile_config != HEAL_TILE_SKINNY_SPLITK) return 0;
-  return partial_bytes(M, N, K) + flag_count(N, K) * sizeof(unsigned long long);
-}
-
-// Per-call tag for the unit flags: a random 64-bit start, then one step per call, so a flag
-// left in a workspace by an earlier call (or any earlier contents) never matches.
-static unsigned long long next_call_tag() {
-  static std::atomic<unsigned long long> tag{[] {
-    std::random_device rd;
-    return ((unsigned long long)rd() << 32) ^ (unsigned long long)rd() ^ 0x9E3779B97F4A7C15ull;
-  }()};
-  return tag.fetch_add(1, std::memory_order_relaxed);
+  const size_t nc = (size_t)((K + kBK - 1) / kBK);
+  const size_t mpad = (size_t)(M <= 16 ? 16 : M <= 32 ? 32 : 64);
+  (void)mpad;
+  return nc * (size_t)M * (size_t)N * sizeof(float);
 }
 
 heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, const void* B, long long ldb,
@@ -1035,8 +944,6 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
   args.num_chunks = nc;
   args.chan_exp = o.chan_exp;
   args.static_op = 0;
-  args.flags = nullptr;
-  args.seq = 0;
   const int pre = o.b_presplit;   // 0 FP32 B, 1 pre-split hi + lo, 2 16-bit B (two products)
   args.status = device_status_ptr();
   cudaError_t err = cudaSuccess;
@@ -1107,13 +1014,6 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.expA_sign = +1;
     args.expB_sign = -1;
     args.static_op = o.b_static ? 1 : 0;   // kernel-A = B^T
-    if (split && M <= 4 && sms <= kMaxFlagCtas) {
-      // M <= 4: the ordered chunk sum runs at the end of the same kernel (no reduce launch);
-      // from M = 8 on, the separate reduce kernel spreads the larger sum over more threads
-      // and measured faster
-      args.flags = reinterpret_cast<unsigned long long*>(static_cast<uint8_t*>(o.workspace) + partial_bytes(M, N, K));
-      args.seq = next_call_tag();
-    }
     const int BNk = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
     if (!operand_map(&ta, B, b_mn, pre != 0, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (pre == 1 && !operand_map(&talo, o.b_lo, b_mn, true, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
@@ -1124,7 +1024,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
         : pre == 1 ? launch_skinny<1>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
                    : launch_skinny<2>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
     if (err != cudaSuccess) return HEAL_ERR_CUDA;
-    if (!split || args.flags != nullptr) return HEAL_OK;   // ordered sum done in the kernel
+    if (!split) return HEAL_OK;
     const long long rblocks = ((long long)N * M + 255) / 256;
     if (rblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
     const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(256), 0, stream,

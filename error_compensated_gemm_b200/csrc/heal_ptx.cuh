@@ -84,37 +84,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // ---------------------------------------------------------------------------------
-// Flags in global memory between CTAs of one grid (release store / acquire load)
-// ---------------------------------------------------------------------------------
-__device__ __forceinline__ void st_release_gpu_u64(unsigned long long* p, unsigned long long v) {
-  asm volatile("st.release.gpu.global.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
-}
-__device__ __forceinline__ unsigned long long ld_acquire_gpu_u64(const unsigned long long* p) {
-  unsigned long long v;
-  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
-  return v;
-}
-
-// Wait until *flag == value.  Same bound and abort protocol as mbar_wait.
-__device__ __forceinline__ bool flag_wait(const unsigned long long* flag, unsigned long long value,
-                                          volatile int* abort_flag, unsigned int* status, int site,
-                                          unsigned long long limit_ns = kWaitLimitNs) {
-  if (ld_acquire_gpu_u64(flag) == value) return true;
-  const uint64_t t0 = globaltimer();
-  while (true) {
-#pragma unroll 1
-    for (int i = 0; i < 16; ++i)
-      if (ld_acquire_gpu_u64(flag) == value) return true;
-    if (*abort_flag) return false;
-    if (globaltimer() - t0 > limit_ns) {
-      *abort_flag = 1;
-      report_timeout(status, site);
-      return false;
-    }
-  }
-}
-
-// ---------------------------------------------------------------------------------
 // Proxy fences
 // ---------------------------------------------------------------------------------
 // Generic-proxy shared-memory writes -> visible to the async proxy (tensor cores, TMA).

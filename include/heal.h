@@ -86,11 +86,9 @@ typedef struct {
                                must already carry the factor 2^e_k.                         */
   const void* b_lo;         /* lo part when b_presplit = 1, else null                        */
   void* workspace;          /* device scratch for HEAL_TILE_SKINNY_SPLITK (nullable; 16-byte
-                               aligned): the per-chunk values, then one 64-bit flag per CTA
-                               through which CTAs publish their chunk values when M <= 4 (the
-                               ordered sum then runs in the same kernel).  Its contents need
-                               no initialisation; each call tags its flags with a fresh 64-bit
-                               value, so stale contents never match.                        */
+                               aligned): the per-chunk values [K/64][M][N] FP32, added in
+                               ascending chunk order by a second kernel.  Its contents need
+                               no initialisation.                                          */
   size_t workspace_bytes;
   int b_static;             /* 1: B (and b_lo) are not written by work queued before this call
                                on the stream (weights).  GEMM kernels start with programmatic

@@ -29,8 +29,8 @@ def test_library_loads_and_exports_every_symbol():
 
 
 def test_workspace_queries_are_host_only():
-    # chunk values [64][1][4096] FP32, then one 64-bit flag per CTA (room for 1024 CTAs)
-    assert heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK) == 64 * 4096 * 4 + 1024 * 8
+    # chunk values [64][1][4096] FP32
+    assert heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK) == 64 * 4096 * 4
     assert heal.heal_gemm_workspace_bytes(4096, 4096, 4096, heal.TILE_128x128) == 0
     assert heal.heal_attention_workspace_bytes(8, 32, 1, 8192) > 0
     assert heal.heal_attention_workspace_bytes(0, 32, 1, 8192) == 0

@@ -273,3 +273,34 @@ def test_two_product_16bit_weights(fmt, b_layout, M):
     emu = G.gemm_two_product(X.numpy(), W16.float().numpy().astype(np.float64),
                              S.FP16_S11 if fmt == heal.SPLIT_FP16_S11 else S.BF16)
     assert G.normwise_rel_err(outs[0], emu) <= (5e-7 if fmt == heal.SPLIT_FP16_S11 else 2e-5)
+
+
+@pytest.mark.parametrize("M", [1, 8, 64, 256])
+def test_graph_replay_with_new_inputs(M):
+    """A GEMM captured once in a CUDA graph and replayed after its input buffer was rewritten
+    gives, at every replay, the bits of an eager call on the new input (nothing of an earlier
+    launch may stand in for this one's data)."""
+    d = dev()
+    K, N = 1024, 768
+    W = (0.02 * synthetic.normal((K, N), seed=41)).to(d)
+    X = torch.empty(M, K, device=d)
+    C = torch.empty(M, N, device=d)
+    ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(M, N, K, heal.TILE_SKINNY_SPLITK) // 4), device=d)
+    use_ws = ws if M <= 64 else None
+    X.copy_(synthetic.normal((M, K), seed=50).to(d))
+    heal.heal_gemm_compensated(X, W, C, workspace=use_ws, b_static=True)
+    torch.cuda.synchronize()
+    s = torch.cuda.Stream()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=s):
+        heal.heal_gemm_compensated(X, W, C, workspace=use_ws, b_static=True)
+    for seed in (51, 52, 53):
+        X.copy_(synthetic.normal((M, K), seed=seed).to(d))
+        g.replay()
+        torch.cuda.synchronize()
+        got = to_np(C).copy()
+        ref = torch.empty(M, N, device=d)
+        heal.heal_gemm_compensated(X, W, ref, workspace=use_ws)
+        torch.cuda.synchronize()
+        assert np.array_equal(got.view(np.uint32), to_np(ref).view(np.uint32)), seed
+    status_ok()
