@@ -293,6 +293,135 @@ class Workload:
     LAUNCHES_PER_STEP = 1 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
 
 
+class TorchDecoder:
+    """The same random-init decoder block in plain torch ops at one precision: a comparison
+    pipeline for the reproducibility study, not the library.  Every op reads and writes
+    `dtype` tensors (for bf16 this is the plain 16-bit stack whose results are stored in 16
+    bits at every kernel boundary); K and V are cached in `dtype`; attention is torch's
+    scaled_dot_product_attention."""
+
+    def __init__(self, torch, cfg, w, dtype, dev, max_len):
+        self.t, self.cfg, self.dtype, self.dev = torch, cfg, dtype, dev
+        self.w = {k: v.to(dev, dtype) for k, v in w.items()}
+        half = cfg.head_dim // 2
+        inv = torch.tensor([cfg.rope_theta ** (-2.0 * i / cfg.head_dim) for i in range(half)], dtype=torch.float64)
+        ang = torch.arange(max_len, dtype=torch.float64)[:, None] * inv[None, :]
+        self.cos, self.sin = torch.cos(ang).to(dev, dtype), torch.sin(ang).to(dev, dtype)
+        self.k = [torch.zeros(max_len, cfg.kv_heads, cfg.head_dim, dtype=dtype, device=dev) for _ in range(cfg.layers)]
+        self.v = [torch.zeros(max_len, cfg.kv_heads, cfg.head_dim, dtype=dtype, device=dev) for _ in range(cfg.layers)]
+        self.pos = 0
+
+    def _rms(self, x):
+        t = self.t
+        return x * t.rsqrt((x * x).mean(-1, keepdim=True) + self.cfg.eps)
+
+    def _rope(self, x, p0):
+        n, half = x.shape[0], self.cfg.head_dim // 2
+        c, s = self.cos[p0:p0 + n, None, :], self.sin[p0:p0 + n, None, :]
+        a, b = x[..., :half], x[..., half:]
+        return self.t.cat([a * c - b * s, b * c + a * s], dim=-1)
+
+    def forward(self, ids):
+        t, c = self.t, self.cfg
+        F = t.nn.functional
+        n, p0 = ids.numel(), self.pos
+        h = self.w["embed"][ids.long()]
+        qd, kd = c.heads * c.head_dim, c.kv_heads * c.head_dim
+        G = c.heads // c.kv_heads
+        for l in range(c.layers):
+            x = self._rms(h)
+            qkv = x @ self.w[f"wqkv{l}"]
+            q = self._rope(qkv[:, :qd].view(n, c.heads, c.head_dim), p0)
+            k = self._rope(qkv[:, qd:qd + kd].view(n, c.kv_heads, c.head_dim), p0)
+            self.k[l][p0:p0 + n] = k
+            self.v[l][p0:p0 + n] = qkv[:, qd + kd:].view(n, c.kv_heads, c.head_dim)
+            K = self.k[l][:p0 + n].repeat_interleave(G, dim=1).transpose(0, 1)   # [heads, T, D]
+            V = self.v[l][:p0 + n].repeat_interleave(G, dim=1).transpose(0, 1)
+            o = F.scaled_dot_product_attention(q.transpose(0, 1), K, V, is_causal=(n > 1 and p0 == 0),
+                                               scale=c.head_dim ** -0.5)
+            h = h + o.transpose(0, 1).reshape(n, qd) @ self.w[f"wo{l}"]
+            x = self._rms(h)
+            gu = x @ self.w[f"wgu{l}"]
+            h = h + (F.silu(gu[:, :c.ffn]) * gu[:, c.ffn:]) @ self.w[f"wdown{l}"]
+        self.pos = p0 + n
+        self.last_hidden = self._rms(h[n - 1:n])
+        return self.last_hidden @ self.w["lm_head"]
+
+
+def reproducibility_study(torch, heal, synthetic, dev, prompt_len=512, steps=128):
+    """Reproducibility analogue on the random-init 2-layer stack: the FP64 pipeline decodes
+    greedily; the FP32, plain-BF16 and HEAL pipelines are teacher-forced on its tokens, and
+    each step's logits and final hidden state are compared with FP64 (flips = steps whose
+    argmax differs).  Each pipeline's own greedy decode is timed per output token."""
+    from error_compensated_gemm_b200.decoder import Decoder
+    torch.backends.cuda.matmul.allow_tf32 = False
+    torch.backends.cudnn.allow_tf32 = False
+    cfg = synthetic.DecoderConfig(max_pos=prompt_len + steps + 64)
+    w = synthetic.decoder_weights(cfg)
+    prompt = synthetic.prompt_ids(prompt_len, cfg.vocab).to(dev)
+    max_len = prompt_len + steps + 64
+
+    def run(fw, reset, tokens=None):
+        """Prefill, then `steps` decode steps (teacher-forced on `tokens` if given, else greedy).
+        Returns (logits list, hidden list, token list)."""
+        reset()
+        lg = fw(prompt)
+        L, Hs, toks = [], [], []
+        for s in range(steps):
+            L.append(lg.double().flatten())
+            Hs.append(fw.__self__.last_hidden.double().flatten())
+            nxt = int(torch.argmax(lg.float()).item()) if tokens is None else tokens[s]
+            toks.append(nxt)
+            if s + 1 < steps:
+                lg = fw(torch.tensor([nxt], dtype=torch.int32, device=dev))
+        return L, Hs, toks
+
+    ref = TorchDecoder(torch, cfg, w, torch.float64, dev, max_len)
+    L64, H64, T64 = run(ref.forward, lambda: setattr(ref, "pos", 0))
+    del ref
+    torch.cuda.empty_cache()
+    out = {"study": "reproducibility analogue (random-init 2-layer stack, teacher-forced on the FP64 "
+                    "greedy tokens)", "prompt": prompt_len, "steps": steps, "pipelines": {}}
+    pipes = [("fp32", None), ("bf16_downcast", None), ("heal", None)]
+    for name, _ in pipes:
+        if name == "heal":
+            dec = Decoder(cfg, w, dev, max_len=max_len)
+            fw, reset = dec.forward, (lambda d=dec: setattr(d, "pos_len", 0))
+        else:
+            dec = TorchDecoder(torch, cfg, w, torch.float32 if name == "fp32" else torch.bfloat16, dev, max_len)
+            fw, reset = dec.forward, (lambda d=dec: setattr(d, "pos", 0))
+        L, Hs, _ = run(fw, reset, T64)
+        rel = [float(torch.linalg.norm(a - b) / torch.linalg.norm(b)) for a, b in zip(L, L64)]
+        mse = [float(((a - b) ** 2).mean()) for a, b in zip(Hs, H64)]
+        flips = sum(int(torch.argmax(a).item() != torch.argmax(b).item()) for a, b in zip(L, L64))
+        # own greedy decode, timed per output token (eager launches, CUDA events)
+        reset()
+        lg = fw(prompt)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        own = []
+        e0.record()
+        for s in range(steps):
+            nxt = torch.argmax(lg.float()).to(torch.int32).view(1)
+            own.append(nxt)
+            if s + 1 < steps:
+                lg = fw(nxt)
+        e1.record()
+        torch.cuda.synchronize()
+        own = [int(x.item()) for x in own]
+        first_div = next((i for i, (a, b) in enumerate(zip(own, T64)) if a != b), None)
+        out["pipelines"][name] = {
+            "logits_rel_err_mean": sum(rel) / len(rel), "logits_rel_err_max": max(rel),
+            "final_hidden_mse_mean": sum(mse) / len(mse), "argmax_flips": flips,
+            "first_divergence_free_running": first_div, "tpot_ms": e0.elapsed_time(e1) / steps}
+        del dec
+        torch.cuda.empty_cache()
+    b = out["pipelines"]["bf16_downcast"]["tpot_ms"]
+    for name in out["pipelines"]:
+        out["pipelines"][name]["tpot_vs_bf16"] = out["pipelines"][name]["tpot_ms"] / b
+    return out
+
+
 def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=128):
     """2-layer random-init decoder (hidden 4096, 32q/8kv heads, FFN 14336, vocab 128256):
     time of the 512-token prefill and per greedy decode step, and a bitwise repeat check."""
@@ -444,6 +573,8 @@ def main():
     ap.add_argument("--prefill-shape", default=None, help="M,N,K of the prefill GEMM (profiling case)")
     ap.add_argument("--kv-batch", type=int, default=None, help="batch of the KV workload (profiling case)")
     ap.add_argument("--no-decoder", action="store_true", help="skip the 2-layer decoder measurement")
+    ap.add_argument("--study", action="store_true",
+                    help="reproducibility analogue: FP64 / FP32 / plain BF16 / HEAL pipelines on the decoder")
     args = ap.parse_args()
     if args.prefill_shape:
         global PREFILL
@@ -461,6 +592,10 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
     heal.lib()
+    if args.study:
+        if rank == 0:
+            print(json.dumps(reproducibility_study(torch, heal, synthetic, dev)), flush=True)
+        return 0
     peaks, peak_src = load_peaks()
     wl = Workload(torch, heal, synthetic, dev, seed_offset=1000 * rank, only=args.only)
     for _ in range(max(3, args.warmup)):

@@ -539,9 +539,22 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
 // Chunk arithmetic and the ascending FP32 chunk sum are those of heal_gemm_kernel, so C is
 // identical bit for bit.
 // ---------------------------------------------------------------------------------
-constexpr int kPairThreads = 512;
 constexpr int kPairSplitWarps = 6;
-constexpr int kPairEpiWarp0 = 8, kPairEpiWarps = 8;
+constexpr int kPairEpiWarp0 = 2 + kPairSplitWarps, kPairEpiWarps = 8;
+constexpr int kPairThreads = (kPairEpiWarp0 + kPairEpiWarps) * 32;
+// Register split: the epilogue keeps 128 FP32 sums per thread (168 registers); the other
+// warps give theirs back.  setmaxnreg.inc draws on the registers the block was launched
+// with, so the shares must add up to no more than threads x the compiled register count;
+// the host checks that count before the first launch (eight split warps, for instance,
+// compile to 96 registers per thread, too few for this split).
+constexpr int kPairEpiRegs = 168;
+constexpr int kPairLaunchRegs = (65536 / kPairThreads) / 8 * 8;
+constexpr int kPairOtherRegs =
+    ((kPairLaunchRegs * kPairThreads - kPairEpiRegs * kPairEpiWarps * 32) / (kPairEpiWarp0 * 32)) / 8 * 8 > 88
+        ? 88
+        : ((kPairLaunchRegs * kPairThreads - kPairEpiRegs * kPairEpiWarps * 32) / (kPairEpiWarp0 * 32)) / 8 * 8;
+static_assert(kPairEpiWarp0 * 32 * kPairOtherRegs + kPairEpiWarps * 32 * kPairEpiRegs <= kPairLaunchRegs * kPairThreads,
+              "register shares exceed the launch allocation");
 constexpr int kPairRows = 128;                      // rows of A and of B per CTA
 constexpr int kPairN = 256;                         // MMA N (= B columns per pair)
 constexpr int kPairStageBytes = 2 * kPairRows * kBK * 4;
@@ -601,7 +614,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 
   if (warp == 0) {
     // ------------------------------ TMA producer ------------------------------
-    setmaxnreg_dec<88>();
+    setmaxnreg_dec<kPairOtherRegs>();
     if (lane == 0) {
       tma_prefetch_desc(&tmA);
       tma_prefetch_desc(&tmB);
@@ -634,7 +647,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
   } else if (warp == 1) {
     // ------------------------------ MMA issuer (leader CTA) ------------------------------
-    setmaxnreg_dec<88>();
+    setmaxnreg_dec<kPairOtherRegs>();
     if (rank == 0 && lane == 0) {
       const uint32_t peer = 1u;
       int it = 0;
@@ -682,10 +695,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
   } else if (warp < kPairEpiWarp0) {
     // ------------------------------ split warps (both CTAs) ------------------------------
-    setmaxnreg_dec<88>();
+    setmaxnreg_dec<kPairOtherRegs>();
     pdl_wait_prerequisites();   // chan_exp may come from the preceding kernel
     const int sw = warp - 2;
     constexpr int kPairsA = kPairRows / 8, kPairsB = kPairRows / 8;
+    static_assert(kPairEpiWarp0 == 2 + kPairSplitWarps, "split warps are warps 2 .. kPairEpiWarp0 - 1");
     const uint32_t sd_leader0 = mapa_shared(smem_u32(&split_done[0]), 0u);
     int it = 0;
     bool ok = true;
@@ -718,7 +732,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     }
   } else {
     // ------------------------------ epilogue (both CTAs) ------------------------------
-    setmaxnreg_inc<168>();
+    setmaxnreg_inc<kPairEpiRegs>();
     pdl_wait_prerequisites();   // C may still be read by the preceding kernel
     const int quarter = warp & 3;
     const int half = (warp - kPairEpiWarp0) >> 2;
@@ -847,6 +861,13 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& alo, const C
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    if (BN == 128) {
+      // setmaxnreg shares (8 warps at 96, 4 epilogue warps at 240) must fit the launch allocation
+      cudaFuncAttributes fa{};
+      e = cudaFuncGetAttributes(&fa, kern);
+      if (e != cudaSuccess) return e;
+      if ((long long)fa.numRegs * Roles<BN>::kThreads < 8LL * 32 * 96 + 4LL * 32 * 240) return cudaErrorInvalidConfiguration;
+    }
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;
@@ -888,6 +909,13 @@ cudaError_t launch_pair(const CUtensorMap& a, const CUtensorMap& b, const CUtens
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 64 || !attr_set[dev]) {
+    // the warps' register shares must fit the registers the block is launched with
+    cudaFuncAttributes fa{};
+    e = cudaFuncGetAttributes(&fa, kern);
+    if (e != cudaSuccess) return e;
+    if ((long long)fa.numRegs * kPairThreads <
+        (long long)kPairEpiWarp0 * 32 * kPairOtherRegs + (long long)kPairEpiWarps * 32 * kPairEpiRegs)
+      return cudaErrorInvalidConfiguration;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kPairSmemBytes);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) attr_set[dev] = true;

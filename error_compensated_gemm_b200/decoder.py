@@ -109,6 +109,7 @@ class Decoder:
         self.pos_len = p0 + n
         x = torch.empty(1, c.hidden, device=self.dev)
         H.heal_rmsnorm(h[n - 1:n], self.rms_w, x, c.eps)
+        self.last_hidden = x                     # final normed hidden state of the last position
         logits = torch.empty(1, c.vocab, device=self.dev)
         self._linear(x, self.w["lm_head"], logits)
         return logits
