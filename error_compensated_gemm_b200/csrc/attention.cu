@@ -18,14 +18,18 @@
 // sum 256*hi*P + lo*P = v*P.  These are the two FP16 tensors the INT16 value is unpacked
 // into for the floating-point contraction.
 //
-// Work decomposition: a persistent grid; CTA c owns the contiguous slice
-// [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token block)
-// units.  Warp 4 streams 64-token K and V tiles with TMA (128-byte swizzle) into a
-// two-stage ring (the K half of a stage is released after QK^T, the V half after PV);
-// warps 0-3 each take 16 tokens of a tile with mma.sync (the decode GEMV shapes are far
-// below a tcgen05 tile; the kernel is HBM-bound).  Every (CTA, kv head) segment leaves one
-// partial (m, l, o) in the workspace; the combine kernel merges them in ascending token
-// order.  The order is fixed, so results are identical from run to run.
+// Work decomposition: a persistent grid (two CTAs per SM); CTA c owns the contiguous
+// slice [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token
+// block) units.  Warp roles: a TMA producer streams 64-token K and V tiles (128-byte
+// swizzle) into a three-stage ring; four QK warps take 16 tokens each (exact S^T on the
+// integer tensor cores, logits, the block's softmax step with the row maximum shared by
+// the four warps, P' split into FP16 parts and written in the PV operand layout); four PV
+// warps each own a quarter of the dims of O and add V^T P'^T over the block's 64 tokens.
+// The two groups work on consecutive blocks at the same time.  mma.sync rather than
+// tcgen05: the decode shapes (<= 8 query rows per KV head) are far below a tcgen05 tile
+// and the kernel is HBM-bound.  Every (CTA, kv head) segment leaves one partial (m, l, o)
+// in the workspace; the combine kernel merges them in ascending token order.  The order
+// is fixed, so results are identical from run to run.
 #include <cuda_fp16.h>
 
 #include <cmath>
@@ -38,13 +42,13 @@ namespace heal {
 namespace {
 
 constexpr int kBlk = 64;          // tokens per pipeline stage
-// K/V stages per CTA.  Two stages leave room for three CTAs (15 warps) per SM; on the
-// 8 x 8192 x 8 x 128 decode cache three stages (two CTAs per SM) measured 9% slower and
-// four or six (one CTA per SM) 44% slower: warps per SM matter more than ring depth here.
-constexpr int kStages = 2;
-constexpr int kMinBlocks = kStages <= 2 ? 3 : (kStages == 3 ? 2 : 1);   // CTAs per SM the ring allows
-constexpr int kCompute = 4;       // compute warps, 16 tokens each per stage
-constexpr int kAttnThreads = (kCompute + 1) * 32;
+// Warp roles per CTA: kQK warps for QK^T and the softmax step (16 tokens each), kPV warps
+// for PV (D/4 dims each), one TMA producer.  Three K/V stages per CTA, two CTAs per SM
+// (16 compute warps and six stages per SM).
+constexpr int kQK = 4, kPV = 4;
+constexpr int kStages = 3;
+constexpr int kMinBlocks = 2;
+constexpr int kAttnThreads = (kQK + kPV + 1) * 32;
 constexpr int kRows = 8;          // query rows per CTA: (Hq/Hkv) * Tq <= 8
 constexpr int kMaxGrid = 1024;
 constexpr float kLog2e = 1.4426950408889634f;
@@ -134,7 +138,6 @@ __device__ __forceinline__ float mul_pow2(float x, int e) {
   return __fmul_rn(__fmul_rn(x, __int_as_float((127 + e1) << 23)), __int_as_float((127 + e2) << 23));
 }
 
-__device__ __forceinline__ void compute_bar() { asm volatile("bar.sync 1, %0;" ::"n"(kCompute * 32) : "memory"); }
 
 __device__ __forceinline__ long long unit_begin(long long total, int grid, int c) {
   return (total * c) / grid;
@@ -161,16 +164,25 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
   constexpr int kTileBytes = kBlk * D * 2;          // one of K / V
   constexpr int kStageBytes = 2 * kTileBytes;
   constexpr int kKSteps32 = D / 32;                 // k32 steps of the integer MMA
+  constexpr int kDT = D / 16 / kPV;                 // 16-dim blocks of O per PV warp
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;                                                  // kStages x kStageBytes
-  float* o_sm = reinterpret_cast<float*>(smem + kStages * kStageBytes);    // [kRows][D]
-  float* ml_sm = o_sm + kRows * D;                                   // [kCompute][kRows][2]
-  uint4* qf_sm = reinterpret_cast<uint4*>(ml_sm + kCompute * kRows * 2); // [kKSteps32][32 lanes]
-  float* sc_sm = reinterpret_cast<float*>(qf_sm + kKSteps32 * 32);      // [kStages][K, V][kBlk]
-  uint64_t* full = reinterpret_cast<uint64_t*>(sc_sm + kStages * 2 * kBlk);  // [S] K tile, [S] V tile + scales
-  uint64_t* empty = full + 2 * kStages;                                // [S] K released, [S] V released
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(empty + 2 * kStages);
+  uint4* pb = reinterpret_cast<uint4*>(smem + kStages * kStageBytes);      // [2][kQK steps][2 parts][32 lanes]
+  uint4* qf_sm = pb + 2 * kQK * 2 * 32;                                    // [kKSteps32][32 lanes]
+  float* sc_sm = reinterpret_cast<float*>(qf_sm + kKSteps32 * 32);         // [kStages][K, V][kBlk]
+  float* meta = sc_sm + kStages * 2 * kBlk;                                // [2][16]: scale of O per row, E
+  float* red = meta + 2 * 16;                                              // [2][kQK][kRows] block maxima
+  float* lsum = red + 2 * kQK * kRows;                                     // [kQK][kRows] row sums
+  float* mq = lsum + kQK * kRows;                                          // [kRows] row maxima
+  uint64_t* full = reinterpret_cast<uint64_t*>(mq + kRows);                // [S] K tile, [S] V tile + scales
+  uint64_t* empty = full + 2 * kStages;                                    // [S] K released, [S] V released
+  uint64_t* pready = empty + 2 * kStages;                                  // [2] P' written (QK -> PV)
+  uint64_t* pfree = pready + 2;                                            // [2] P' consumed (PV -> QK)
+  uint64_t* mxbar = pfree + 2;                                             // [2] block maxima exchanged
+  uint64_t* finbar = mxbar + 2;                                            // row sums exchanged
+  uint64_t* qfbar = finbar + 1;                                            // Q table built
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(qfbar + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int c = blockIdx.x;
@@ -178,16 +190,25 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
   pdl_launch_dependents();   // the combine kernel may be scheduled; it waits for us
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < 2 * kStages; ++s) {
+    for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&empty[s], kCompute);
+      mbar_init(&full[kStages + s], 1);
+      mbar_init(&empty[s], kQK);
+      mbar_init(&empty[kStages + s], kPV);
     }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&pready[b], kQK);
+      mbar_init(&pfree[b], kPV);
+      mbar_init(&mxbar[b], kQK);
+    }
+    mbar_init(finbar, kQK);
+    mbar_init(qfbar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == kCompute) {
+  if (warp == kQK + kPV) {
     // ----------------------------- TMA producer -----------------------------
     if (lane == 0) {
       tma_prefetch_desc(&tmK);
@@ -202,7 +223,7 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
         const uint32_t ph = (uint32_t)(it / kStages) & 1u;
         uint8_t* st = stages + s * kStageBytes;
         const int row = p * a.Tmax + t0;
-        // K half: refilled as soon as the compute warps finish QK^T on the previous tile
+        // K half: refilled as soon as the QK warps finish QK^T on the previous tile
         if (!mbar_wait(&empty[s], ph ^ 1u, abort_flag, a.status, 200)) break;
         mbar_arrive_expect_tx(&full[s], kTileBytes + kBlk * 4);
         bulk_load_1d(sc_sm + (s * 2 + 0) * kBlk, a.ks + (size_t)row, kBlk * 4, &full[s]);
@@ -228,344 +249,393 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
     return;
   }
 
-  // ------------------------------- compute warps -------------------------------
-  // Fragment layouts (mma.sync, g = lane / 4, c = lane % 4):
-  //   S^T = K Q^T with m16n8k32 integer MMAs: rows = this warp's 16 tokens, columns = the
-  //   8 query rows.  C fragment of this lane: tokens g and g + 8, query rows 2c and 2c + 1.
-  //   O^T = V^T P'^T with m16n8k16 FP16 MMAs: rows = 16 dims, columns = query rows; the
-  //   lane holds dims g, g + 8 of query rows 2c, 2c + 1 (the same query rows as S^T).
-  // Byte order inside the K dimension of the integer MMA: slot 4c + j of a 16-slot half
-  // holds dim {2c, 2c + 1, 2c + 8, 2c + 9}[j] of that half; both operands use this order,
-  // and a dot product does not depend on the order of its terms.
   const int R = a.R;
   const int g8 = lane >> 2;                   // token row (S^T) / dim row (O^T) / query of B fragments
   const int qc = 2 * (lane & 3);              // this lane's query rows qc, qc + 1
-  float sq[2] = {0.0f, 0.0f};
-  int pos[2] = {0, 0};
-  float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};   // query rows qc + e
-  float om[D / 16][4];                        // O^T accumulator (units of 2^E_run)
-  int E_run = 0;                              // power of two folded into P (decreases only)
-  bool have_E = false;
-  int cur_p = -1, b = 0, hkv = 0, klen = 0;
-  int it = 0;
   bool ok = true;
 
-  auto finalize = [&](int p) {
-    // per query row: the warp's maximum (replicated over g8) and its sum over all lanes
+  if (warp < kQK) {
+    // ================================ QK warps ================================
+    // Fragment layouts (mma.sync, g8 = lane / 4, c = lane % 4): S^T = K Q^T with
+    // m16n8k32 integer MMAs, rows = this warp's 16 tokens, columns = the 8 query rows; the
+    // C fragment of this lane holds tokens g8, g8 + 8 of query rows qc, qc + 1.  Byte
+    // order in the K dimension: slot 4c + j of a 16-slot half holds dim
+    // {2c, 2c + 1, 2c + 8, 2c + 9}[j]; both operands use it (a dot product does not
+    // depend on the order of its terms).
+    const int w = warp;
+    const int tw = w * 16;                    // this warp's first token inside the tile
+    float sq[2] = {0.0f, 0.0f};
+    int pos[2] = {0, 0};
+    float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+    int E_run = 0;                            // power of two folded into P (decreases only)
+    bool have_E = false;
+    int cur_p = -1, b = 0, hkv = 0, klen = 0;
+    int j = 0, nfin = 0, nsetup = 0;
+
+    auto finalize = [&](int p) {
+      // row sums over this warp's lanes, then over the four QK warps in order
 #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float l = l_run[e];
-      l += __shfl_xor_sync(0xffffffffu, l, 4);
-      l += __shfl_xor_sync(0xffffffffu, l, 8);
-      l += __shfl_xor_sync(0xffffffffu, l, 16);
-      if (g8 == 0) {
-        ml_sm[(warp * kRows + qc + e) * 2 + 0] = m_run[e];
-        ml_sm[(warp * kRows + qc + e) * 2 + 1] = l;
+      for (int e = 0; e < 2; ++e) {
+        float l = l_run[e];
+        l += __shfl_xor_sync(0xffffffffu, l, 4);
+        l += __shfl_xor_sync(0xffffffffu, l, 8);
+        l += __shfl_xor_sync(0xffffffffu, l, 16);
+        if (g8 == 0) {
+          lsum[w * kRows + qc + e] = l;
+          if (w == 0) mq[qc + e] = m_run[e];
+        }
       }
-    }
-    compute_bar();
-    // query rows of this lane's O^T fragments: qc, qc + 1
-    float f[2];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(finbar);
+      if (!mbar_wait(finbar, (uint32_t)(nfin & 1), abort_flag, a.status, 215)) ok = false;
+      ++nfin;
+      if (ok && w == 0 && lane < R) {
+        float L = 0.0f;
+        for (int ww = 0; ww < kQK; ++ww) L = __fadd_rn(L, lsum[ww * kRows + lane]);
+        float* sl = slot_ptr(a.ws, c, p, R, D) + R * D;
+        sl[2 * lane] = mq[lane];
+        sl[2 * lane + 1] = L;
+      }
+    };
+
+    for (long long u = u0; u < u1 && ok; ++u) {
+      const int p = (int)(u / a.nblk), blk = (int)(u % a.nblk);
+      if (p != cur_p) {
+        if (cur_p >= 0) {
+          finalize(cur_p);
+          if (!ok) break;
+        }
+        cur_p = p;
+        b = p / a.Hkv;
+        hkv = p % a.Hkv;
+        klen = __ldg(a.kv_len + b);
+        // query row r = tq * G + g of this kv head  ->  head hkv*G + g, query tq
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int r = qc + h;
-      float mx = -INFINITY;
-      for (int w = 0; w < kCompute; ++w) mx = fmaxf(mx, ml_sm[(w * kRows + r) * 2]);
-      const float mw = ml_sm[(warp * kRows + r) * 2];
-      f[h] = (mw == -INFINITY) ? 0.0f : exp2f(mw - mx);
-    }
-    // O of this warp, scaled to the CTA max, in true units (x 2^-E_run), in place
+        for (int e = 0; e < 2; ++e) {
+          const int r = qc + e;
+          const bool real = r < R;
+          const int tq = real ? r / a.G : 0, gq = real ? r % a.G : 0;
+          sq[e] = real ? __ldg(a.qs + ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq)) : 0.0f;
+          pos[e] = klen - a.Tq + tq;
+        }
+        // B fragments of Q^T (query row g8), byte-split, one table per CTA:
+        // entry [s][lane] = (hi slots 0-15, hi slots 16-31, lo slots 0-15, lo slots 16-31).
+        // Warp 0 rebuilds it once every QK warp is past the previous pair (finalize).
+        if (w == 0) {
+          const int r = g8;
+          const bool real = r < R;
+          const int tq = real ? r / a.G : 0, gq = real ? r % a.G : 0;
+          const long long qrow = ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq);
 #pragma unroll
-    for (int dt = 0; dt < D / 16; ++dt)
+          for (int s32 = 0; s32 < kKSteps32; ++s32) {
+            uint32_t wq[4] = {0u, 0u, 0u, 0u};
+            if (real) {
+              const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow * D + s32 * 32 + qc);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) om[dt][e] = __fmul_rn(mul_pow2(om[dt][e], -E_run), f[e & 1]);
-    // sequential, fixed-order merge of the four warps through shared memory
-    for (int w = 0; w < kCompute; ++w) {
-      if (warp == w) {
+              for (int i = 0; i < 4; ++i) wq[i] = __ldg(qp + 4 * i);   // dims 32s + 8i + 2c, +1
+            }
+            qf_sm[s32 * 32 + lane] = make_uint4(hi_bytes(wq[0], wq[1]), hi_bytes(wq[2], wq[3]),
+                                                lo_bytes(wq[0], wq[1]), lo_bytes(wq[2], wq[3]));
+          }
+          __syncwarp();
+          if (lane == 0) mbar_arrive(qfbar);
+        }
+        if (!mbar_wait(qfbar, (uint32_t)(nsetup & 1), abort_flag, a.status, 216)) {
+          ok = false;
+          break;
+        }
+        ++nsetup;
 #pragma unroll
-        for (int dt = 0; dt < D / 16; ++dt)
+        for (int e = 0; e < 2; ++e) {
+          m_run[e] = -INFINITY;
+          l_run[e] = 0.0f;
+        }
+        E_run = 0;
+        have_E = false;
+      }
+      const int t0 = blk * kBlk;
+      if (t0 >= klen) continue;
+      const int s = j % kStages;
+      const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+      const int jb = j & 1;
+      const uint32_t jph = (uint32_t)(j >> 1) & 1u;
+      ++j;
+      if (!mbar_wait(&full[s], ph, abort_flag, a.status, 210)) {
+        ok = false;
+        break;
+      }
+      const uint32_t kst = smem_u32(stages + s * kStageBytes);
+      const float* sks = sc_sm + (s * 2 + 0) * kBlk;   // K scales of this block's 64 tokens
+      const float* svs = sc_sm + (s * 2 + 1) * kBlk;   // V scales
+
+      // ---- exact S^T = K Q^T on the byte-split operands (integer tensor cores) ----
+      // S_x in two accumulators (kh.ql and kl.qh) so no MMA chain is longer than the k32 steps
+      int shh[4] = {0, 0, 0, 0}, sxa[4] = {0, 0, 0, 0}, sxb[4] = {0, 0, 0, 0}, sll[4] = {0, 0, 0, 0};
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int d = dt * 16 + g8 + ((e >> 1) << 3);
-            const int r = qc + (e & 1);
-            float* dst = o_sm + r * D + d;
-            const float v = (w == 0) ? om[dt][e] : __fadd_rn(*dst, om[dt][e]);
-            if (w < kCompute - 1) {
-              *dst = v;
-            } else if (r < R) {
-              slot_ptr(a.ws, c, p, R, D)[r * D + d] = v;
+      for (int s32 = 0; s32 < kKSteps32; ++s32) {
+        const uint4 qf = qf_sm[s32 * 32 + lane];
+        uint32_t r[2][4];                       // [token half][16-byte chunk 4*s32 + i]
+#pragma unroll
+        for (int th = 0; th < 2; ++th) {
+          const int trow = tw + th * 8 + (lane & 7);
+          const int ch = 4 * s32 + (lane >> 3);   // 16-byte chunk of the K row
+          const uint32_t addr = kst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
+          ldsm_x4(addr, r[th][0], r[th][1], r[th][2], r[th][3]);
+        }
+        // A fragments: a0 token g8 slots 0-15, a1 token g8+8, a2 token g8 slots 16-31, a3 token g8+8
+        const uint32_t ah0 = hi_bytes(r[0][0], r[0][1]), ah1 = hi_bytes(r[1][0], r[1][1]);
+        const uint32_t ah2 = hi_bytes(r[0][2], r[0][3]), ah3 = hi_bytes(r[1][2], r[1][3]);
+        const uint32_t al0 = lo_bytes(r[0][0], r[0][1]), al1 = lo_bytes(r[1][0], r[1][1]);
+        const uint32_t al2 = lo_bytes(r[0][2], r[0][3]), al3 = lo_bytes(r[1][2], r[1][3]);
+        imma16832<false, false>(shh, ah0, ah1, ah2, ah3, qf.x, qf.y);
+        imma16832<false, true>(sxa, ah0, ah1, ah2, ah3, qf.z, qf.w);
+        imma16832<true, false>(sxb, al0, al1, al2, al3, qf.x, qf.y);
+        imma16832<true, true>(sll, al0, al1, al2, al3, qf.z, qf.w);
+      }
+      // every ldmatrix of the K tile has been consumed and the K scales this lane needs
+      // are in registers: release the K half before the logit arithmetic
+      float skr[2];
+#pragma unroll
+      for (int th = 0; th < 2; ++th) skr[th] = sks[tw + th * 8 + g8];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[s]);
+      float x[2][2];                            // [token half][query e]: logit * log2(e)
+#pragma unroll
+      for (int th = 0; th < 2; ++th) {
+#pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int i = 2 * th + e;
+          const int t = t0 + tw + th * 8 + g8;
+          const int r = qc + e;
+          const long long S = ((long long)shh[i] << 16) + (((long long)sxa[i] + (long long)sxb[i]) << 8) +
+                              (long long)sll[i];
+          const bool real = r < R;
+          const bool vis = real && t < klen && (!a.causal || t <= pos[e]);
+          float xv;
+          if (!real) {
+            xv = 0.0f;                          // padding query row: finite, never written
+          } else if (!vis) {
+            xv = -INFINITY;
+          } else {
+            const double coef = (double)sq[e] * (double)skr[th];
+            const float lg = (float)(((double)S * coef) * (double)a.scale);
+            xv = __fmul_rn(lg, kLog2e);
+            if (a.qk_out) {
+              const int tq = r / a.G, gq = r % a.G;
+              a.qk_out[((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq) * a.Tmax + t] = S;
             }
           }
+          x[th][e] = xv;
+        }
       }
-      compute_bar();
-    }
-    if (warp == 0 && lane < R) {
-      const int r = lane;
-      float mx = -INFINITY;
-      for (int w = 0; w < kCompute; ++w) mx = fmaxf(mx, ml_sm[(w * kRows + r) * 2]);
-      float L = 0.0f;
-      for (int w = 0; w < kCompute; ++w) {
-        const float mw = ml_sm[(w * kRows + r) * 2];
-        if (mw != -INFINITY) L = __fadd_rn(L, __fmul_rn(ml_sm[(w * kRows + r) * 2 + 1], exp2f(mw - mx)));
+
+      // ---- the block's maximum per query row, shared by the four QK warps ----
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float bm = fmaxf(x[0][e], x[1][e]);
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
+        bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
+        if (g8 == 0) red[(jb * kQK + w) * kRows + qc + e] = bm;
       }
-      float* sl = slot_ptr(a.ws, c, p, R, D) + R * D;
-      sl[2 * r] = mx;
-      sl[2 * r + 1] = L;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&mxbar[jb]);
+      // the V tile's scales arrive with it: wait for the stage without consuming it
+      if (!mbar_wait(&mxbar[jb], jph, abort_flag, a.status, 212) ||
+          !mbar_wait(&full[kStages + s], ph, abort_flag, a.status, 211)) {
+        ok = false;
+        break;
+      }
+      float alpha[2], pv[2][2];
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        float bm = -INFINITY;
+#pragma unroll
+        for (int ww = 0; ww < kQK; ++ww) bm = fmaxf(bm, red[(jb * kQK + ww) * kRows + qc + e]);
+        const float m_new = fmaxf(m_run[e], bm);
+        if (m_new == -INFINITY) {
+          alpha[e] = 1.0f;
+          pv[0][e] = pv[1][e] = 0.0f;
+        } else {
+          alpha[e] = (m_run[e] == -INFINITY) ? 0.0f : exp2f(m_run[e] - m_new);
+#pragma unroll
+          for (int th = 0; th < 2; ++th) pv[th][e] = (x[th][e] == -INFINITY) ? 0.0f : exp2f(x[th][e] - m_new);
+        }
+        l_run[e] = __fadd_rn(__fmul_rn(l_run[e], alpha[e]), __fadd_rn(pv[0][e], pv[1][e]));
+        m_run[e] = m_new;
+      }
+      // power of two for this block: the largest visible V scale times 2^E in [32, 64)
+      // (V scales are non-negative, so their bit patterns order like the floats)
+      float smax;
+      {
+        const int ta = t0 + lane, tb = t0 + 32 + lane;
+        unsigned int um = 0u;
+        if (ta < klen) um = __float_as_uint(svs[lane]);
+        if (tb < klen) um = max(um, __float_as_uint(svs[32 + lane]));
+        smax = __uint_as_float(__reduce_max_sync(0xffffffffu, um));
+      }
+      float escale = 1.0f;                       // 2^(E_new - E_run) applied to O
+      if (smax > 0.0f) {
+        const int E_blk = 5 - ilogbf(smax);
+        if (!have_E) {
+          E_run = E_blk;
+          have_E = true;
+        } else if (E_blk < E_run) {
+          escale = ldexpf(1.0f, E_blk - E_run);
+          E_run = E_blk;
+        }
+      }
+
+      // ---- P' = P * s_v * 2^E (S^T layout), moved to the B layout of PV: lane (g8, c)
+      // needs tokens 2c, 2c + 1, 2c + 8, 2c + 9 of query row g8.  Token 2c + jj lives in lane
+      // 4 * (2c + jj) + g8 / 2 (halves th = 0 / 1 for +0 / +8), query row g8 in slot g8 & 1.
+      float pp[2][2];
+#pragma unroll
+      for (int th = 0; th < 2; ++th) {
+        const int t = t0 + tw + th * 8 + g8;
+        const float svt = mul_pow2(svs[t - t0], E_run);   // s_v * 2^E, in [0, 64)
+#pragma unroll
+        for (int e = 0; e < 2; ++e) pp[th][e] = __fmul_rn(pv[th][e], (pv[th][e] != 0.0f) ? svt : 0.0f);
+      }
+      float pt[2][2];                            // [token half][jj]: P' of token 8*half + 2c + jj, query g8
+      {
+        const int cq = lane & 3;
+        const bool odd = (g8 & 1) != 0;
+#pragma unroll
+        for (int jj = 0; jj < 2; ++jj) {
+          const int src = 4 * (2 * cq + jj) + (g8 >> 1);
+#pragma unroll
+          for (int th = 0; th < 2; ++th) {
+            const float v0 = __shfl_sync(0xffffffffu, pp[th][0], src);
+            const float v1 = __shfl_sync(0xffffffffu, pp[th][1], src);
+            pt[th][jj] = odd ? v1 : v0;
+          }
+        }
+      }
+      // FP16 P_hi and residual r = P' - P_hi, and both times 256: the B fragments of PV
+      uint32_t ph_[2], pr_[2], ph256[2], pr256[2];
+#pragma unroll
+      for (int th = 0; th < 2; ++th) {
+        const __half2 h = __floats2half2_rn(pt[th][0], pt[th][1]);
+        const float2 hf = __half22float2(h);
+        const __half2 rr = __floats2half2_rn(__fsub_rn(pt[th][0], hf.x), __fsub_rn(pt[th][1], hf.y));
+        const __half2 k256 = __half2half2(__ushort_as_half(0x5C00));   // 256.0
+        const __half2 h256 = __hmul2(h, k256), r256 = __hmul2(rr, k256); // exact: powers of two
+        ph_[th] = *reinterpret_cast<const uint32_t*>(&h);
+        pr_[th] = *reinterpret_cast<const uint32_t*>(&rr);
+        ph256[th] = *reinterpret_cast<const uint32_t*>(&h256);
+        pr256[th] = *reinterpret_cast<const uint32_t*>(&r256);
+      }
+      // hand the block to the PV warps (the buffer is free once they finished block j - 2)
+      if (!mbar_wait(&pfree[jb], jph ^ 1u, abort_flag, a.status, 213)) {
+        ok = false;
+        break;
+      }
+      uint4* pbw = pb + ((jb * kQK + w) * 2) * 32;
+      pbw[lane] = make_uint4(ph256[0], ph256[1], ph_[0], ph_[1]);
+      pbw[32 + lane] = make_uint4(pr256[0], pr256[1], pr_[0], pr_[1]);
+      if (w == 0) {
+        if (g8 == 0) {
+          meta[jb * 16 + qc] = __fmul_rn(alpha[0], escale);
+          meta[jb * 16 + qc + 1] = __fmul_rn(alpha[1], escale);
+        }
+        if (lane == 0) meta[jb * 16 + 8] = __int_as_float(E_run);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&pready[jb]);
     }
-    compute_bar();
+    if (ok && cur_p >= 0) finalize(cur_p);
+    return;
+  }
+
+  // ================================ PV warps ================================
+  // O^T = V^T P'^T with m16n8k16 FP16 MMAs: rows = 16 dims, columns = the 8 query rows;
+  // this warp owns dims [v * D/4, (v + 1) * D/4) of every row over all 64 tokens.
+  const int v = warp - kQK;
+  float om[kDT][4];                           // O^T accumulator (units of 2^E_run)
+#pragma unroll
+  for (int dl = 0; dl < kDT; ++dl)
+#pragma unroll
+    for (int e = 0; e < 4; ++e) om[dl][e] = 0.0f;
+  int E_run = 0;
+  int cur_p = -1, klen = 0;
+  int j = 0;
+
+  auto finalize_o = [&](int p) {
+    float* sl = slot_ptr(a.ws, c, p, R, D);
+#pragma unroll
+    for (int dl = 0; dl < kDT; ++dl)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int d = (v * kDT + dl) * 16 + g8 + ((e >> 1) << 3);
+        const int r = qc + (e & 1);
+        if (r < R) sl[r * D + d] = mul_pow2(om[dl][e], -E_run);   // true units (x 2^-E_run)
+        om[dl][e] = 0.0f;
+      }
   };
 
   for (long long u = u0; u < u1 && ok; ++u) {
     const int p = (int)(u / a.nblk), blk = (int)(u % a.nblk);
     if (p != cur_p) {
-      if (cur_p >= 0) finalize(cur_p);
+      if (cur_p >= 0) finalize_o(cur_p);
       cur_p = p;
-      b = p / a.Hkv;
-      hkv = p % a.Hkv;
-      klen = __ldg(a.kv_len + b);
-      // query row r = tq * G + g of this kv head  ->  head hkv*G + g, query tq
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int r = qc + e;
-        const bool real = r < R;
-        const int tq = real ? r / a.G : 0, gq = real ? r % a.G : 0;
-        sq[e] = real ? __ldg(a.qs + ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq)) : 0.0f;
-        pos[e] = klen - a.Tq + tq;
-      }
-      // B fragments of Q^T (query row g8), byte-split, one table per CTA:
-      // entry [s][lane] = (hi slots 0-15, hi slots 16-31, lo slots 0-15, lo slots 16-31)
-      if (warp == 0) {
-        const int r = g8;
-        const bool real = r < R;
-        const int tq = real ? r / a.G : 0, gq = real ? r % a.G : 0;
-        const long long qrow = ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq);
-#pragma unroll
-        for (int s32 = 0; s32 < kKSteps32; ++s32) {
-          uint32_t w[4] = {0u, 0u, 0u, 0u};
-          if (real) {
-            const uint32_t* qp = reinterpret_cast<const uint32_t*>(a.q + qrow * D + s32 * 32 + qc);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) w[i] = __ldg(qp + 4 * i);   // dims 32s + 8i + 2c, +1
-          }
-          qf_sm[s32 * 32 + lane] = make_uint4(hi_bytes(w[0], w[1]), hi_bytes(w[2], w[3]), lo_bytes(w[0], w[1]),
-                                              lo_bytes(w[2], w[3]));
-        }
-      }
-      compute_bar();
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        m_run[e] = -INFINITY;
-        l_run[e] = 0.0f;
-      }
+      klen = __ldg(a.kv_len + p / a.Hkv);
       E_run = 0;
-      have_E = false;
-#pragma unroll
-      for (int dt = 0; dt < D / 16; ++dt)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) om[dt][e] = 0.0f;
     }
     const int t0 = blk * kBlk;
     if (t0 >= klen) continue;
-    const int s = it % kStages;
-    const uint32_t ph = (uint32_t)(it / kStages) & 1u;
-    ++it;
-    if (!mbar_wait(&full[s], ph, abort_flag, a.status, 210)) {
+    const int s = j % kStages;
+    const uint32_t ph = (uint32_t)(j / kStages) & 1u;
+    const int jb = j & 1;
+    const uint32_t jph = (uint32_t)(j >> 1) & 1u;
+    ++j;
+    if (!mbar_wait(&pready[jb], jph, abort_flag, a.status, 220) ||
+        !mbar_wait(&full[kStages + s], ph, abort_flag, a.status, 221)) {
       ok = false;
       break;
     }
-    const uint32_t kst = smem_u32(stages + s * kStageBytes);
-    const uint32_t vst = kst + kTileBytes;
-    const float* sks = sc_sm + (s * 2 + 0) * kBlk;   // K scales of this block's 64 tokens
-    const float* svs = sc_sm + (s * 2 + 1) * kBlk;   // V scales
-    const int tw = warp * 16;                 // this warp's first token inside the tile
-
-    // ---- exact S^T = K Q^T on the byte-split operands (integer tensor cores) ----
-    // S_x in two accumulators (kh.ql and kl.qh) so no MMA chain is longer than the k32 steps
-    int shh[4] = {0, 0, 0, 0}, sxa[4] = {0, 0, 0, 0}, sxb[4] = {0, 0, 0, 0}, sll[4] = {0, 0, 0, 0};
-#pragma unroll
-    for (int s32 = 0; s32 < kKSteps32; ++s32) {
-      const uint4 qf = qf_sm[s32 * 32 + lane];
-      uint32_t r[2][4];                       // [token half][16-byte chunk 4*s32 + i]
-#pragma unroll
-      for (int th = 0; th < 2; ++th) {
-        const int trow = tw + th * 8 + (lane & 7);
-        const int ch = 4 * s32 + (lane >> 3);   // 16-byte chunk of the K row
-        const uint32_t addr = kst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
-        ldsm_x4(addr, r[th][0], r[th][1], r[th][2], r[th][3]);
-      }
-      // A fragments: a0 token g8 slots 0-15, a1 token g8+8, a2 token g8 slots 16-31, a3 token g8+8
-      const uint32_t ah0 = hi_bytes(r[0][0], r[0][1]), ah1 = hi_bytes(r[1][0], r[1][1]);
-      const uint32_t ah2 = hi_bytes(r[0][2], r[0][3]), ah3 = hi_bytes(r[1][2], r[1][3]);
-      const uint32_t al0 = lo_bytes(r[0][0], r[0][1]), al1 = lo_bytes(r[1][0], r[1][1]);
-      const uint32_t al2 = lo_bytes(r[0][2], r[0][3]), al3 = lo_bytes(r[1][2], r[1][3]);
-      imma16832<false, false>(shh, ah0, ah1, ah2, ah3, qf.x, qf.y);
-      imma16832<false, true>(sxa, ah0, ah1, ah2, ah3, qf.z, qf.w);
-      imma16832<true, false>(sxb, al0, al1, al2, al3, qf.x, qf.y);
-      imma16832<true, true>(sll, al0, al1, al2, al3, qf.z, qf.w);
-    }
-    // every ldmatrix of the K tile has been consumed by the MMAs above and the K scales
-    // this lane needs are copied to registers: release the K half now, before the logit
-    // arithmetic, so the producer can refill it sooner
-    float skr[2];
-#pragma unroll
-    for (int th = 0; th < 2; ++th) skr[th] = sks[tw + th * 8 + g8];
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[s]);
-    float x[2][2];                            // [token half][query e]: logit * log2(e)
-#pragma unroll
-    for (int th = 0; th < 2; ++th) {
-#pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int i = 2 * th + e;
-        const int t = t0 + tw + th * 8 + g8;
-        const int r = qc + e;
-        const long long S = ((long long)shh[i] << 16) + (((long long)sxa[i] + (long long)sxb[i]) << 8) +
-                            (long long)sll[i];
-        const bool real = r < R;
-        const bool vis = real && t < klen && (!a.causal || t <= pos[e]);
-        float xv;
-        if (!real) {
-          xv = 0.0f;                          // padding query row: finite, never written
-        } else if (!vis) {
-          xv = -INFINITY;
-        } else {
-          const double coef = (double)sq[e] * (double)skr[th];
-          const float lg = (float)(((double)S * coef) * (double)a.scale);
-          xv = __fmul_rn(lg, kLog2e);
-          if (a.qk_out) {
-            const int tq = r / a.G, gq = r % a.G;
-            a.qk_out[((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq) * a.Tmax + t] = S;
-          }
-        }
-        x[th][e] = xv;
-      }
-    }
-
-    if (!mbar_wait(&full[kStages + s], ph, abort_flag, a.status, 211)) {
-      ok = false;
-      break;
-    }
-
-    // ---- online softmax (base 2) of query rows qc, qc + 1 over this warp's tokens ----
-    float alpha[2], pv[2][2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      float bm = fmaxf(x[0][e], x[1][e]);
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 4));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 8));
-      bm = fmaxf(bm, __shfl_xor_sync(0xffffffffu, bm, 16));
-      const float m_new = fmaxf(m_run[e], bm);
-      if (m_new == -INFINITY) {
-        alpha[e] = 1.0f;
-        pv[0][e] = pv[1][e] = 0.0f;
-      } else {
-        alpha[e] = (m_run[e] == -INFINITY) ? 0.0f : exp2f(m_run[e] - m_new);
-#pragma unroll
-        for (int th = 0; th < 2; ++th) pv[th][e] = (x[th][e] == -INFINITY) ? 0.0f : exp2f(x[th][e] - m_new);
-      }
-      l_run[e] = __fadd_rn(__fmul_rn(l_run[e], alpha[e]), __fadd_rn(pv[0][e], pv[1][e]));
-      m_run[e] = m_new;
-    }
-    // power of two for this block: the largest visible V scale times 2^E in [32, 64)
-    // (V scales are non-negative, so their bit patterns order like the floats: one
-    // warp-wide integer max gives the block maximum)
-    float smax;
-    {
-      const int ta = t0 + lane, tb = t0 + 32 + lane;
-      unsigned int um = 0u;
-      if (ta < klen) um = __float_as_uint(svs[lane]);
-      if (tb < klen) um = max(um, __float_as_uint(svs[32 + lane]));
-      smax = __uint_as_float(__reduce_max_sync(0xffffffffu, um));
-    }
-    float escale = 1.0f;                       // 2^(E_new - E_run) applied to O
-    if (smax > 0.0f) {
-      const int E_blk = 5 - ilogbf(smax);
-      if (!have_E) {
-        E_run = E_blk;
-        have_E = true;
-      } else if (E_blk < E_run) {
-        escale = ldexpf(1.0f, E_blk - E_run);
-        E_run = E_blk;
-      }
-    }
-    // rescale O^T columns qc, qc + 1 (this lane's own query rows)
-    const float a0 = __fmul_rn(alpha[0], escale);
-    const float a1 = __fmul_rn(alpha[1], escale);
+    const uint32_t vst = smem_u32(stages + s * kStageBytes) + kTileBytes;
+    // rescale O^T columns qc, qc + 1 by the block's softmax step and change of 2^E
+    const float a0 = meta[jb * 16 + qc], a1 = meta[jb * 16 + qc + 1];
+    E_run = __float_as_int(meta[jb * 16 + 8]);
     if (!__all_sync(0xffffffffu, a0 == 1.0f && a1 == 1.0f)) {
 #pragma unroll
-      for (int dt = 0; dt < D / 16; ++dt) {
-        om[dt][0] = __fmul_rn(om[dt][0], a0);
-        om[dt][1] = __fmul_rn(om[dt][1], a1);
-        om[dt][2] = __fmul_rn(om[dt][2], a0);
-        om[dt][3] = __fmul_rn(om[dt][3], a1);
+      for (int dl = 0; dl < kDT; ++dl) {
+        om[dl][0] = __fmul_rn(om[dl][0], a0);
+        om[dl][1] = __fmul_rn(om[dl][1], a1);
+        om[dl][2] = __fmul_rn(om[dl][2], a0);
+        om[dl][3] = __fmul_rn(om[dl][3], a1);
       }
     }
-
-    // ---- P' = P * s_v * 2^E (S^T layout), moved to the B layout of PV: lane (g8, c)
-    // needs tokens 2c, 2c + 1, 2c + 8, 2c + 9 of query row g8.  Token 2c + j lives in lane
-    // 4 * (2c + j) + g8 / 2 (halves th = 0 / 1 for +0 / +8), query row g8 in its slot g8 & 1.
-    float pp[2][2];
+    // ---- O^T += V^T P'^T  (256*hi*P + lo*P with P = P_hi + r), 16 tokens per step ----
 #pragma unroll
-    for (int th = 0; th < 2; ++th) {
-      const int t = t0 + tw + th * 8 + g8;
-      const float svt = mul_pow2(svs[t - t0], E_run);   // s_v * 2^E, in [0, 64)
+    for (int ts = 0; ts < kQK; ++ts) {
+      const uint4 fh = pb[((jb * kQK + ts) * 2) * 32 + lane];        // P_hi * 256, P_hi
+      const uint4 fr = pb[((jb * kQK + ts) * 2 + 1) * 32 + lane];    // r * 256, r
 #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float sv = (pv[th][e] != 0.0f) ? svt : 0.0f;
-        pp[th][e] = __fmul_rn(pv[th][e], sv);
+      for (int dl = 0; dl < kDT; ++dl) {
+        const int dt = v * kDT + dl;
+        const int mi = lane >> 3;
+        const int trow = ts * 16 + ((mi >> 1) << 3) + (lane & 7);
+        const int ch = 2 * dt + (mi & 1);
+        const uint32_t addr = vst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
+        uint32_t r0, r1, r2, r3;
+        ldsm_x4_t(addr, r0, r1, r2, r3);
+        const uint32_t h0 = hi_pair(r0), h1 = hi_pair(r1), h2 = hi_pair(r2), h3 = hi_pair(r3);
+        const uint32_t l0 = lo_pair(r0), l1 = lo_pair(r1), l2 = lo_pair(r2), l3 = lo_pair(r3);
+        mma16816(om[dl], h0, h1, h2, h3, fh.x, fh.y);
+        mma16816(om[dl], l0, l1, l2, l3, fh.z, fh.w);
+        mma16816(om[dl], h0, h1, h2, h3, fr.x, fr.y);
+        mma16816(om[dl], l0, l1, l2, l3, fr.z, fr.w);
       }
-    }
-    float pt[2][2];                            // [token half][j]: P' of token 8*half + 2c + j, query g8
-    {
-      const int cq = lane & 3;
-      const bool odd = (g8 & 1) != 0;
-#pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int src = 4 * (2 * cq + j) + (g8 >> 1);
-#pragma unroll
-        for (int th = 0; th < 2; ++th) {
-          const float v0 = __shfl_sync(0xffffffffu, pp[th][0], src);
-          const float v1 = __shfl_sync(0xffffffffu, pp[th][1], src);
-          pt[th][j] = odd ? v1 : v0;
-        }
-      }
-    }
-    // FP16 P_hi and residual r = P' - P_hi: B fragments of PV
-    uint32_t ph_[2], pr_[2], ph256[2], pr256[2];
-#pragma unroll
-    for (int th = 0; th < 2; ++th) {
-      const __half2 h = __floats2half2_rn(pt[th][0], pt[th][1]);
-      const float2 hf = __half22float2(h);
-      const __half2 rr = __floats2half2_rn(__fsub_rn(pt[th][0], hf.x), __fsub_rn(pt[th][1], hf.y));
-      const __half2 k256 = __half2half2(__ushort_as_half(0x5C00));   // 256.0
-      const __half2 h256 = __hmul2(h, k256), r256 = __hmul2(rr, k256); // exact: powers of two
-      ph_[th] = *reinterpret_cast<const uint32_t*>(&h);
-      pr_[th] = *reinterpret_cast<const uint32_t*>(&rr);
-      ph256[th] = *reinterpret_cast<const uint32_t*>(&h256);
-      pr256[th] = *reinterpret_cast<const uint32_t*>(&r256);
-    }
-
-    // ---- O^T += V^T P'^T  (256*hi*P + lo*P with P = P_hi + r) ----
-#pragma unroll
-    for (int dt = 0; dt < D / 16; ++dt) {
-      const int mi = lane >> 3;
-      const int trow = tw + ((mi >> 1) << 3) + (lane & 7);
-      const int ch = 2 * dt + (mi & 1);
-      const uint32_t addr = vst + (ch >> 3) * 8192 + trow * 128 + ((((ch & 7) ^ (trow & 7))) << 4);
-      uint32_t r0, r1, r2, r3;
-      ldsm_x4_t(addr, r0, r1, r2, r3);
-      const uint32_t h0 = hi_pair(r0), h1 = hi_pair(r1), h2 = hi_pair(r2), h3 = hi_pair(r3);
-      const uint32_t l0 = lo_pair(r0), l1 = lo_pair(r1), l2 = lo_pair(r2), l3 = lo_pair(r3);
-      mma16816(om[dt], h0, h1, h2, h3, ph256[0], ph256[1]);
-      mma16816(om[dt], l0, l1, l2, l3, ph_[0], ph_[1]);
-      mma16816(om[dt], h0, h1, h2, h3, pr256[0], pr256[1]);
-      mma16816(om[dt], l0, l1, l2, l3, pr_[0], pr_[1]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&empty[kStages + s]);
+    if (lane == 0) {
+      mbar_arrive(&empty[kStages + s]);   // V tile consumed
+      mbar_arrive(&pfree[jb]);            // P' buffer consumed
+    }
   }
-  if (!ok) return;   // a wait gave up: the status word is set; leave without a partial
-  if (cur_p >= 0) finalize(cur_p);
+  if (ok && cur_p >= 0) finalize_o(cur_p);
 }
 
 // out[b, hq, tq, :] = sum_c o_c 2^(m_c - M) / sum_c l_c 2^(m_c - M), c ascending.
@@ -617,8 +687,13 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
 
 template <int D>
 constexpr int attn_smem_bytes() {
-  return kStages * (2 * kBlk * D * 2) + kRows * D * 4 + kCompute * kRows * 2 * 4 + (D / 32) * 32 * 16 +
-         kStages * 2 * kBlk * 4 + 2 * 2 * kStages * 8 + 32 + 1024;
+  return kStages * (2 * kBlk * D * 2)          // K / V stages
+         + 2 * kQK * 2 * 32 * 16               // P' operand buffers
+         + (D / 32) * 32 * 16                  // Q table
+         + kStages * 2 * kBlk * 4              // K / V scales
+         + (2 * 16 + 2 * kQK * kRows + kQK * kRows + kRows) * 4   // meta, maxima, sums
+         + (4 * kStages + 8) * 8 + 16          // barriers, abort flag
+         + 1024;                               // alignment
 }
 
 }  // namespace
