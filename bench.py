@@ -121,6 +121,10 @@ class Workload:
             X, W = synthetic.gemm_prefill(M=M, K=K, N=N, seed_x=0 + so, seed_w=1 + so)
             self.X, self.W = X.to(dev), W.to(dev)
             self.C = torch.empty(M, N, device=dev)
+            # the same weights split once (static weights held as hi / lo)
+            self.Whi = torch.empty(self.W.shape, dtype=torch.int16, device=dev)
+            self.Wlo = torch.empty(self.W.shape, dtype=torch.int16, device=dev)
+            heal.heal_split(self.W, self.Whi, self.Wlo)
         self.dec = []
         if need("decode"):
             for i, m in enumerate(DECODE_M):
@@ -188,6 +192,7 @@ class Workload:
         only = self.only
         if only in (None, "prefill"):
             out.append(("prefill", lambda: h.heal_gemm_compensated(self.X, self.W, self.C)))
+            out.append(("prefill_presplit", lambda: h.heal_gemm_compensated(self.X, self.Whi, self.C, b_lo=self.Wlo)))
         if only in (None, "decode"):
             for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
                 out.append((f"decode{m}", lambda Xd=Xd, Wd=Wd, Cd=Cd, ws=ws: h.heal_gemm_compensated(
@@ -258,6 +263,9 @@ class Workload:
             rec("prefill", 0)
             h.heal_gemm_compensated(self.X, self.W, self.C)
             rec("prefill", 1)
+            rec("prefill_presplit", 0)
+            h.heal_gemm_compensated(self.X, self.Whi, self.C, b_lo=self.Wlo)
+            rec("prefill_presplit", 1)
         if only in (None, "decode"):
             for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
                 rec(f"decode{m}", 0)
@@ -290,7 +298,7 @@ class Workload:
                                    KV["D"] ** -0.5, self.out, self.aws)
             rec("attention", 1)
 
-    LAUNCHES_PER_STEP = 1 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
+    LAUNCHES_PER_STEP = 2 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
 
 
 class TorchDecoder:
@@ -614,9 +622,9 @@ def main():
     dec_names = ([f"decode{m}" for m in DECODE_M] + [f"decode{m}_presplit" for m in DECODE_M] +
                  [f"decode{m}_w16" for m in DECODE_M] +
                  ["decode1_chain", "decode1_chain_presplit", "decode1_chain_w16"])
-    names = ["prefill"] + dec_names + ["kv_writer", "attention"]
+    names = ["prefill", "prefill_presplit"] + dec_names + ["kv_writer", "attention"]
     if args.only:
-        keep = {"prefill": ["prefill"], "decode": dec_names,
+        keep = {"prefill": ["prefill", "prefill_presplit"], "decode": dec_names,
                 "kv_writer": ["kv_writer"], "attention": ["kv_writer", "attention"]}[args.only]
         names = keep
     evs = [{n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for n in names}
@@ -742,6 +750,11 @@ def main():
             "data": "synthetic",
             "config": arm_config(ws),
             "pct_of_16bit_peak": 100.0 * mma_tflops / peak_sus,
+            "prefill_presplit_weights": {
+                "tflops_effective": ws * u["prefill_flop_eff"] / (part_ms["prefill_presplit"] / 1e3 / K) / 1e12,
+                "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / (part_ms["prefill_presplit"] / 1e3 / K) / 1e12
+                                     / peak_sus,
+                "note": "the same product with W split once into hi/lo beforehand (static weights)"},
             "roofline": {"bound": "tensor", "achieved": mma_tflops, "peak": peak_sus, "unit": "TFLOP/s",
                          "frac": mma_tflops / peak_sus, "traffic": traffic,
                          "kernel": "heal_gemm_pair_kernel (prefill, 256x256 CTA pair)", "peak_source": f"bf16_tflops_sustained, {peak_src}",
