@@ -188,6 +188,7 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
   const int c = blockIdx.x;
   const long long u0 = unit_begin(a.total, a.grid, c), u1 = unit_begin(a.total, a.grid, c + 1);
   pdl_launch_dependents();   // the combine kernel may be scheduled; it waits for us
+  pdl_wait_prerequisites();  // Q, the caches and kv_len may come from the preceding kernel
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -778,11 +779,13 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
     return HEAL_ERR_CUDA;
   cudaError_t e;
   if (D == 128) {
-    heal_attn_decode_kernel<128><<<a.grid, kAttnThreads, attn_smem_bytes<128>(), stream>>>(tk, tv, a);
-    e = launch_pdl(heal_attn_combine_kernel<128>, dim3(B * Hkv * R), dim3(128), 0, stream, a);
+    e = launch_pdl(heal_attn_decode_kernel<128>, dim3(a.grid), dim3(kAttnThreads), (size_t)attn_smem_bytes<128>(), stream,
+                   tk, tv, a);
+    if (e == cudaSuccess) e = launch_pdl(heal_attn_combine_kernel<128>, dim3(B * Hkv * R), dim3(128), 0, stream, a);
   } else {
-    heal_attn_decode_kernel<64><<<a.grid, kAttnThreads, attn_smem_bytes<64>(), stream>>>(tk, tv, a);
-    e = launch_pdl(heal_attn_combine_kernel<64>, dim3(B * Hkv * R), dim3(64), 0, stream, a);
+    e = launch_pdl(heal_attn_decode_kernel<64>, dim3(a.grid), dim3(kAttnThreads), (size_t)attn_smem_bytes<64>(), stream,
+                   tk, tv, a);
+    if (e == cudaSuccess) e = launch_pdl(heal_attn_combine_kernel<64>, dim3(B * Hkv * R), dim3(64), 0, stream, a);
   }
   if (e != cudaSuccess) return HEAL_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;

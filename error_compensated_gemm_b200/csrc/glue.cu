@@ -12,6 +12,10 @@
 #include "heal_internal.h"
 #include "heal_ptx.cuh"
 
+// Every kernel here is launched with programmatic dependent launch: it lets the next
+// kernel of the stream be scheduled at once and waits for the preceding one before its
+// first global access, so only launch and setup overlap the neighbours.
+
 namespace heal {
 namespace {
 
@@ -26,6 +30,8 @@ __device__ __forceinline__ float warp_sum(float v) {
 // out[i, :] = table[ids[i], :]
 __global__ void embed_kernel(const float* __restrict__ table, const int32_t* __restrict__ ids, int n, int H,
                              int vocab, float* __restrict__ out, unsigned int* status) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   const int i = blockIdx.x;
   const int id = ids[i];
   if (id < 0 || id >= vocab) {   // invalid id: zero row and flag it (never read out of bounds)
@@ -41,6 +47,8 @@ __global__ void embed_kernel(const float* __restrict__ table, const int32_t* __r
 // then warp shuffles, then warps in index order)
 __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restrict__ w, int H, float eps,
                                float* __restrict__ y) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   __shared__ float part[kThreads / 32];
   const int i = blockIdx.x;
   const float* xr = x + (size_t)i * H;
@@ -61,6 +69,8 @@ __global__ void rmsnorm_kernel(const float* __restrict__ x, const float* __restr
 __global__ void rope_kernel(float* __restrict__ x, int n, int heads, int D, long long row_stride,
                             const int32_t* __restrict__ pos, const float* __restrict__ cos_t,
                             const float* __restrict__ sin_t) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   const int i = blockIdx.x / heads, h = blockIdx.x % heads;
   float* r = x + (size_t)i * row_stride + (size_t)h * D;
   const int p = pos[i];
@@ -75,6 +85,8 @@ __global__ void rope_kernel(float* __restrict__ x, int n, int heads, int D, long
 
 // out[i, j] = silu(g[i, j]) * u[i, j] with g = gu[i, j], u = gu[i, F + j]
 __global__ void swiglu_kernel(const float* __restrict__ gu, int n, int F, float* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   const long long total = (long long)n * F;
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < total;
        e += (long long)gridDim.x * blockDim.x) {
@@ -86,12 +98,16 @@ __global__ void swiglu_kernel(const float* __restrict__ gu, int n, int F, float*
 
 // x += y
 __global__ void add_kernel(float* __restrict__ x, const float* __restrict__ y, long long n) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   for (long long e = blockIdx.x * (long long)blockDim.x + threadIdx.x; e < n; e += (long long)gridDim.x * blockDim.x)
     x[e] += y[e];
 }
 
 // index of the largest value of each row (lowest index among equal maxima; NaN never wins)
 __global__ void argmax_kernel(const float* __restrict__ x, int rows, int n, int32_t* __restrict__ out) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   __shared__ float bv[kThreads];
   __shared__ int bi[kThreads];
   const int r = blockIdx.x;
@@ -130,7 +146,6 @@ int grid_for(long long n) {
   return (int)(g < 1 ? 1 : g);
 }
 
-heal_status_t done() { return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA; }
 
 }  // namespace
 }  // namespace heal
@@ -144,16 +159,16 @@ heal_status_t heal_embedding_gather(const float* table, int vocab, int H, const 
   if (n < 0 || H <= 0 || vocab <= 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (n == 0) return HEAL_OK;
   if (!table || !ids || !out) return HEAL_ERR_INVALID_ARGUMENT;
-  embed_kernel<<<n, kThreads, 0, (cudaStream_t)stream>>>(table, ids, n, H, vocab, out, device_status_ptr());
-  return done();
+  return launch_pdl(embed_kernel, dim3(n), dim3(kThreads), 0, (cudaStream_t)stream, table, ids, n, H, vocab, out,
+                    device_status_ptr()) == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 heal_status_t heal_rmsnorm(const float* x, const float* w, int n, int H, float eps, float* y, heal_stream_t stream) {
   if (n < 0 || H <= 0 || !(eps >= 0.0f)) return HEAL_ERR_INVALID_ARGUMENT;
   if (n == 0) return HEAL_OK;
   if (!x || !y) return HEAL_ERR_INVALID_ARGUMENT;
-  rmsnorm_kernel<<<n, kThreads, 0, (cudaStream_t)stream>>>(x, w, H, eps, y);
-  return done();
+  return launch_pdl(rmsnorm_kernel, dim3(n), dim3(kThreads), 0, (cudaStream_t)stream, x, w, H, eps, y) == cudaSuccess
+             ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 heal_status_t heal_rope(float* x, int n, int heads, int D, int64_t row_stride, const int32_t* pos,
@@ -161,32 +176,32 @@ heal_status_t heal_rope(float* x, int n, int heads, int D, int64_t row_stride, c
   if (n < 0 || heads <= 0 || D <= 0 || (D & 1) || row_stride < (int64_t)heads * D) return HEAL_ERR_INVALID_ARGUMENT;
   if (n == 0) return HEAL_OK;
   if (!x || !pos || !cos_t || !sin_t) return HEAL_ERR_INVALID_ARGUMENT;
-  rope_kernel<<<n * heads, 64, 0, (cudaStream_t)stream>>>(x, n, heads, D, row_stride, pos, cos_t, sin_t);
-  return done();
+  return launch_pdl(rope_kernel, dim3(n * heads), dim3(64), 0, (cudaStream_t)stream, x, n, heads, D,
+                    (long long)row_stride, pos, cos_t, sin_t) == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 heal_status_t heal_swiglu(const float* gate_up, int n, int F, float* out, heal_stream_t stream) {
   if (n < 0 || F <= 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (n == 0) return HEAL_OK;
   if (!gate_up || !out) return HEAL_ERR_INVALID_ARGUMENT;
-  swiglu_kernel<<<grid_for((long long)n * F), kThreads, 0, (cudaStream_t)stream>>>(gate_up, n, F, out);
-  return done();
+  return launch_pdl(swiglu_kernel, dim3(grid_for((long long)n * F)), dim3(kThreads), 0, (cudaStream_t)stream, gate_up,
+                    n, F, out) == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 heal_status_t heal_add(float* x, const float* y, int64_t n, heal_stream_t stream) {
   if (n < 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (n == 0) return HEAL_OK;
   if (!x || !y) return HEAL_ERR_INVALID_ARGUMENT;
-  add_kernel<<<grid_for(n), kThreads, 0, (cudaStream_t)stream>>>(x, y, n);
-  return done();
+  return launch_pdl(add_kernel, dim3(grid_for(n)), dim3(kThreads), 0, (cudaStream_t)stream, x, y, (long long)n) ==
+                 cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 heal_status_t heal_argmax(const float* x, int rows, int n, int32_t* out, heal_stream_t stream) {
   if (rows < 0 || n <= 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (rows == 0) return HEAL_OK;
   if (!x || !out) return HEAL_ERR_INVALID_ARGUMENT;
-  argmax_kernel<<<rows, kThreads, 0, (cudaStream_t)stream>>>(x, rows, n, out);
-  return done();
+  return launch_pdl(argmax_kernel, dim3(rows), dim3(kThreads), 0, (cudaStream_t)stream, x, rows, n, out) ==
+                 cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 }  // extern "C"

@@ -12,6 +12,7 @@
 #include <cuda_bf16.h>
 
 #include "heal_internal.h"
+#include "heal_ptx.cuh"
 
 namespace heal {
 
@@ -20,6 +21,10 @@ __global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restri
                                                             long long sb, long long st, long long sh,
                                                             int16_t* __restrict__ q, float* __restrict__ sc,
                                                             int Tmax, int t_off) {
+  // programmatic dependent launch: the next kernel may be scheduled now; the preceding one
+  // (which may write x or read the cache) finishes before the first global access here
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
   constexpr int D = 8 * L;
   constexpr int kRowsPerPass = 32 / L;      // (token, head) rows one warp covers per pass
   constexpr int kUnroll = 4;                // passes whose loads are in flight together
@@ -108,10 +113,10 @@ template <int L>
 static cudaError_t launch_L(const void* x, int bf16, int B, int T, int H, long long sb, long long st, long long sh,
                             int16_t* q, float* sc, int Tmax, int t_off, int grid, cudaStream_t s) {
   if (bf16)
-    heal_kv_quant_kernel<L, true><<<grid, 256, 0, s>>>(x, B, T, H, sb, st, sh, q, sc, Tmax, t_off);
-  else
-    heal_kv_quant_kernel<L, false><<<grid, 256, 0, s>>>(x, B, T, H, sb, st, sh, q, sc, Tmax, t_off);
-  return cudaGetLastError();
+    return launch_pdl(heal_kv_quant_kernel<L, true>, dim3(grid), dim3(256), 0, s, x, B, T, H, sb, st, sh, q, sc, Tmax,
+                      t_off);
+  return launch_pdl(heal_kv_quant_kernel<L, false>, dim3(grid), dim3(256), 0, s, x, B, T, H, sb, st, sh, q, sc, Tmax,
+                    t_off);
 }
 
 heal_status_t kv_quant_launch(const void* x, int is_bf16, int B, int T, int H, int D, long long sb, long long st,

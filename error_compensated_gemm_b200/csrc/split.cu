@@ -2,6 +2,7 @@
 // weights once, and to test the split in isolation).  HBM-bound: 4 bytes read and
 // 4 bytes written per value.
 #include "heal_internal.h"
+#include "heal_ptx.cuh"
 #include "heal_split.cuh"
 
 namespace heal {
@@ -9,6 +10,8 @@ namespace heal {
 template <int FMT>
 __global__ void __launch_bounds__(256) heal_split_kernel(const float* __restrict__ x, uint16_t* __restrict__ hi,
                                                          uint16_t* __restrict__ lo, long long n, int vec) {
+  pdl_launch_dependents();   // programmatic dependent launch: see the launch below
+  pdl_wait_prerequisites();  // x may come from the preceding kernel
   const long long stride = (long long)gridDim.x * blockDim.x;
   const long long gid = blockIdx.x * (long long)blockDim.x + threadIdx.x;
   long long tail = 0;
@@ -47,11 +50,15 @@ heal_status_t split_launch(const float* x, void* hi, void* lo, long long n, int 
   const long long cap = (long long)sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
-  if (fmt == HEAL_SPLIT_FP16_S11)
-    heal_split_kernel<0><<<(int)blocks, 256, 0, s>>>(x, (uint16_t*)hi, (uint16_t*)lo, n, vec ? 1 : 0);
-  else
-    heal_split_kernel<1><<<(int)blocks, 256, 0, s>>>(x, (uint16_t*)hi, (uint16_t*)lo, n, vec ? 1 : 0);
-  return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+  // programmatic dependent launch: scheduled during the preceding kernel, every access
+  // after griddepcontrol.wait
+  const cudaError_t e =
+      fmt == HEAL_SPLIT_FP16_S11
+          ? launch_pdl(heal_split_kernel<0>, dim3((unsigned)blocks), dim3(256), 0, s, x, (uint16_t*)hi, (uint16_t*)lo, n,
+                       vec ? 1 : 0)
+          : launch_pdl(heal_split_kernel<1>, dim3((unsigned)blocks), dim3(256), 0, s, x, (uint16_t*)hi, (uint16_t*)lo, n,
+                       vec ? 1 : 0);
+  return e == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 }  // namespace heal
