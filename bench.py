@@ -517,7 +517,11 @@ def dist_setup():
     if ws > 1:
         import datetime
         import torch.distributed as dist
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+        # bind this rank's GPU before NCCL starts, so the barrier and the max-over-ranks
+        # run on it
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
     return ws, rank, local
 
 
