@@ -486,6 +486,60 @@ def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=1
                     "(2 layers + the 128256-row LM head)"}
 
 
+# causal INT16 self-attention over a long prompt (the prefill kernel: 128-row query tiles on
+# the tcgen05 tensor cores), timed in its own loop after the step
+PREFILL_ATTN = {"B": 1, "T": 8192, "Hkv": 8, "Hq": 32, "D": 128}
+
+
+def prefill_attention_section(torch, heal, synthetic, dev, stream, cap_stream, reps, peaks):
+    c = PREFILL_ATTN
+    B, T, Hkv, Hq, D = c["B"], c["T"], c["Hkv"], c["Hq"], c["D"]
+    Qb, Kb, Vb = synthetic.kv_decode(B=B, T=T, Hkv=Hkv, Hq=Hq, D=D, Tq=T, seeds=(12, 13, 14))
+    i16, f32 = torch.int16, torch.float32
+    qc = torch.empty(B, Hq, T, D, dtype=i16, device=dev)
+    qs = torch.empty(B, Hq, T, dtype=f32, device=dev)
+    kc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
+    ks = torch.empty(B, Hkv, T, dtype=f32, device=dev)
+    vc = torch.empty(B, Hkv, T, D, dtype=i16, device=dev)
+    vs = torch.empty(B, Hkv, T, dtype=f32, device=dev)
+    heal.heal_kv_quantize_int16(Qb.to(dev), qc, qs)
+    heal.heal_kv_quantize_int16(Kb.to(dev), kc, ks)
+    heal.heal_kv_quantize_int16(Vb.to(dev), vc, vs)
+    kv_len = torch.full((B,), T, dtype=torch.int32, device=dev)
+    out = torch.empty(B, Hq, T, D, device=dev)
+    aws = torch.empty(heal.heal_attention_workspace_bytes_gqa(B, Hq, Hkv, T, T), dtype=torch.uint8, device=dev)
+    call = lambda: heal.heal_attention_int16(qc, qs, kc, ks, vc, vs, kv_len, D ** -0.5, out, aws, causal=True)
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=cap_stream):
+        call()
+    for _ in range(3):
+        g.replay()
+    torch.cuda.synchronize()
+    st = heal.heal_get_device_status()
+    if st != heal.HEAL_OK:
+        raise SystemExit(f"device status after prefill attention warm-up: {heal.status_string(st)}")
+    p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    p0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    p1.record(stream)
+    torch.cuda.synchronize()
+    t = p0.elapsed_time(p1) / 1e3 / reps
+    del g
+    pairs = B * Hq * T * (T + 1) / 2                     # visible (query, token) pairs
+    flop_eff = 4.0 * D * pairs                           # QK^T and PV, 2 flops per multiply-add
+    i8_ops = 4 * 2.0 * D * pairs                         # four 8-bit integer products (S_hh, S_x x2, S_ll)
+    f16_ops = 4 * 2.0 * D * pairs                        # four FP16 products (P_hi, r) x (256 V_hi, V_lo)
+    peak16 = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    ideal = i8_ops / (2 * peak16 * 1e12) + f16_ops / (peak16 * 1e12)
+    return {"config": dict(c, causal=True, Tq=T), "ms": 1e3 * t, "replays": reps,
+            "tflops_effective": flop_eff / t / 1e12,
+            "tensor_ops_per_s": (i8_ops + f16_ops) / t / 1e12,
+            "roofline": {"bound": "tensor", "ideal_ms": 1e3 * ideal, "frac": ideal / t,
+                         "peak": "bf16_tflops burst for the FP16 products, twice it for the 8-bit products"},
+            "note": "conversion pass + tcgen05 attention kernel per call; timed separately after the step"}
+
+
 def cpu_baseline_oracle(rows=4096):
     """The oracle's compensated GEMM (split + three FP64 products) on the prefill workload,
     restricted to `rows` rows of X; returns (TFLOP/s effective, seconds, threads)."""
@@ -576,10 +630,12 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "kv_writer", "attention"],
+    ap.add_argument("--only", choices=["prefill", "decode", "kv_writer", "attention", "attention_prefill"],
                     help="profiling case: run only this part of the step")
     ap.add_argument("--prefill-shape", default=None, help="M,N,K of the prefill GEMM (profiling case)")
     ap.add_argument("--kv-batch", type=int, default=None, help="batch of the KV workload (profiling case)")
+    ap.add_argument("--prompt-len", type=int, default=None,
+                    help="prompt length of the prefill attention workload (profiling case)")
     ap.add_argument("--no-decoder", action="store_true", help="skip the 2-layer decoder measurement")
     ap.add_argument("--study", action="store_true",
                     help="reproducibility analogue: FP64 / FP32 / plain BF16 / HEAL pipelines on the decoder")
@@ -605,6 +661,14 @@ def main():
             print(json.dumps(reproducibility_study(torch, heal, synthetic, dev)), flush=True)
         return 0
     peaks, peak_src = load_peaks()
+    if args.only == "attention_prefill":
+        if args.prompt_len:
+            PREFILL_ATTN["T"] = args.prompt_len
+        res = prefill_attention_section(torch, heal, synthetic, dev, torch.cuda.current_stream(),
+                                        torch.cuda.Stream(), max(1, args.steps), peaks)
+        if rank == 0:
+            print(json.dumps({"profiling_case": args.only, "result": res}), flush=True)
+        return 0
     wl = Workload(torch, heal, synthetic, dev, seed_offset=1000 * rank, only=args.only)
     for _ in range(max(3, args.warmup)):
         wl.run()
@@ -717,6 +781,20 @@ def main():
                             "timed separately after the step"}
         del g
 
+    attn_prefill = None
+    if args.only is None:
+        try:
+            attn_prefill = prefill_attention_section(torch, heal, synthetic, dev, stream, cap_stream,
+                                                     max(5, min(K, 20)), peaks)
+        except SystemExit:
+            raise
+        except Exception as exc:  # report, do not hide
+            attn_prefill = {"error": repr(exc)}
+        if ws > 1:   # every rank takes this collective, failed or not
+            mx = max_over_ranks([attn_prefill.get("ms", -1.0)], device=dev)[0]
+            if "ms" in attn_prefill:
+                attn_prefill["ms"] = mx
+
     # end to end through the public API: pinned host inputs -> device -> GEMM -> host result
     M_, K_, N_ = PREFILL
     e2e = None
@@ -778,6 +856,7 @@ def main():
             "config": arm_config(ws),
             "pct_of_16bit_peak": 100.0 * mma_tflops / peak_sus,
             "prefill_presplit_weights": presplit,
+            "attention_prefill": attn_prefill,
             "roofline": {"bound": "tensor", "achieved": mma_tflops, "peak": peak_sus, "unit": "TFLOP/s",
                          "frac": mma_tflops / peak_sus, "traffic": traffic,
                          "kernel": "heal_gemm_pair_kernel (prefill, 256x256 CTA pair)", "peak_source": f"bf16_tflops_sustained, {peak_src}",

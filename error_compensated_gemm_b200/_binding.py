@@ -13,9 +13,11 @@ TILE_AUTO, TILE_128x128, TILE_256x256_PAIR, TILE_SKINNY_SPLITK, TILE_SKINNY_FULL
 
 # every symbol the public header declares
 EXPORTED = ("heal_split", "heal_gemm_compensated", "heal_gemm_workspace_bytes", "heal_kv_quantize_int16",
-            "heal_attention_int16", "heal_attention_workspace_bytes", "heal_get_device_status",
+            "heal_attention_int16", "heal_attention_workspace_bytes", "heal_attention_workspace_bytes_gqa",
+            "heal_get_device_status",
             "heal_status_string", "heal_version", "heal_attention_int16_noalloc", "heal_embedding_gather",
-            "heal_rmsnorm", "heal_rope", "heal_swiglu", "heal_add", "heal_argmax", "heal_probe_wait_timeout")
+            "heal_rmsnorm", "heal_rope", "heal_swiglu", "heal_add", "heal_argmax", "heal_probe_wait_timeout",
+            "heal_heads_to_rows")
 
 
 class HealError(RuntimeError):
@@ -52,6 +54,7 @@ def lib():
         "heal_attention_int16": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _f, _i, _vp, _vp, _sz,
                                   _vp, _vp], _i),
         "heal_attention_workspace_bytes": ([_i, _i, _i, _i], _sz),
+        "heal_attention_workspace_bytes_gqa": ([_i, _i, _i, _i, _i], _sz),
         "heal_attention_int16_noalloc": ([_vp, _vp, _vp, _vp, _vp, _vp, _i, _i, _i, _i, _i, _vp, _i, _f, _i, _vp,
                                           _vp, _vp], _i),
         "heal_get_device_status": ([_vp], _i),
@@ -62,6 +65,7 @@ def lib():
         "heal_swiglu": ([_vp, _i, _i, _vp, _vp], _i),
         "heal_add": ([_vp, _vp, _i64, _vp], _i),
         "heal_argmax": ([_vp, _i, _i, _vp, _vp], _i),
+        "heal_heads_to_rows": ([_vp, _i, _i, _i, _i, _vp, _vp], _i),
         "heal_status_string": ([_i], ctypes.c_char_p),
         "heal_version": ([], ctypes.c_char_p),
     }
@@ -177,6 +181,10 @@ def heal_attention_workspace_bytes(B, Hq, Tq, Tmax):
     return int(lib().heal_attention_workspace_bytes(int(B), int(Hq), int(Tq), int(Tmax)))
 
 
+def heal_attention_workspace_bytes_gqa(B, Hq, Hkv, Tq, Tmax):
+    return int(lib().heal_attention_workspace_bytes_gqa(int(B), int(Hq), int(Hkv), int(Tq), int(Tmax)))
+
+
 def heal_attention_int16(q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len, softmax_scale, out, workspace,
                          causal=False, qk_int_out=None, stream=None):
     _cuda(q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len, out, workspace, qk_int_out)
@@ -245,6 +253,17 @@ def heal_argmax(x, out, stream=None):
     _cuda(x, out)
     rows, n = x.shape
     _check(lib().heal_argmax(_ptr(x), rows, n, _ptr(out), _stream(stream)), "heal_argmax")
+
+
+def heal_heads_to_rows(x, y, stream=None):
+    """y [B, T, H, D] <- x [B, H, T, D] (both contiguous)."""
+    _cuda(x, y)
+    if not (x.is_contiguous() and y.is_contiguous()):
+        raise ValueError("heal_heads_to_rows needs contiguous tensors")
+    B, H, T, D = x.shape
+    if tuple(y.shape) != (B, T, H, D):
+        raise ValueError("y must be [B, T, H, D]")
+    _check(lib().heal_heads_to_rows(_ptr(x), B, H, T, D, _ptr(y), _stream(stream)), "heal_heads_to_rows")
 
 
 def heal_probe_wait_timeout(limit_ms=200, stream=None):

@@ -53,7 +53,8 @@ extern "C" heal_status_t heal_attention_int16_noalloc(const int16_t* q, const fl
                                                       int64_t* qk_int_out, heal_stream_t stream) {
   // size check first, on the host: the scratch the workspace variant asks for must fit
   if (B <= 0 || Hq <= 0 || Tq <= 0 || Tmax <= 0) return HEAL_ERR_INVALID_ARGUMENT;
-  if (heal_attention_workspace_bytes(B, Hq, Tq, Tmax) > (size_t)HEAL_ATTN_STATIC_SCRATCH_BYTES)
+  if (Hkv <= 0 || Hq % Hkv != 0) return HEAL_ERR_INVALID_ARGUMENT;
+  if (heal_attention_workspace_bytes_gqa(B, Hq, Hkv, Tq, Tmax) > (size_t)HEAL_ATTN_STATIC_SCRATCH_BYTES)
     return HEAL_ERR_UNSUPPORTED;
   void* scratch = nullptr;
   const heal_status_t st = heal::scratch_address(&scratch);

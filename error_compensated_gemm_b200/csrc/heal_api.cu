@@ -149,9 +149,19 @@ heal_status_t heal_kv_quantize_int16(const void* x, int x_is_bf16, int B, int T,
   return st;
 }
 
+size_t heal_attention_workspace_bytes_gqa(int B, int Hq, int Hkv, int Tq, int Tmax) {
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tmax <= 0 || Hq % Hkv != 0) return 0;
+  if ((long long)(Hq / Hkv) * Tq <= 8) return attention_workspace_bytes(B, Hq, Tq, Tmax);
+  return attention_prefill_workspace_bytes(B, Hq, Hkv, Tq, Tmax);
+}
+
 size_t heal_attention_workspace_bytes(int B, int Hq, int Tq, int Tmax) {
   if (B <= 0 || Hq <= 0 || Tq <= 0 || Tmax <= 0) return 0;
-  return attention_workspace_bytes(B, Hq, Tq, Tmax);
+  const size_t dec = attention_workspace_bytes(B, Hq, Tq, Tmax);
+  if (Tq == 1) return dec;
+  // enough for every Hkv that divides Hq (the prefill planes grow with Hkv <= Hq)
+  const size_t pre = attention_prefill_workspace_bytes(B, Hq, Hq, Tq, Tmax);
+  return pre > dec ? pre : dec;
 }
 
 heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale, const int16_t* k_cache,
@@ -162,7 +172,8 @@ heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale, const
   if (B <= 0 || Hq <= 0 || Hkv <= 0 || Tq <= 0 || Tmax <= 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (Hq % Hkv != 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (D != 64 && D != 128) return HEAL_ERR_UNSUPPORTED;
-  if ((Hq / Hkv) * Tq > 8) return HEAL_ERR_UNSUPPORTED;
+  const bool prefill = (long long)(Hq / Hkv) * Tq > 8;   // more query rows per KV head than the decode kernel takes
+  if (prefill && D != 128) return HEAL_ERR_UNSUPPORTED;
   if (Tmax % 64 != 0) return HEAL_ERR_UNSUPPORTED;
   if (causal != 0 && causal != 1) return HEAL_ERR_INVALID_ARGUMENT;
   if (!(softmax_scale > 0.0f) || softmax_scale != softmax_scale) return HEAL_ERR_INVALID_ARGUMENT;
@@ -174,7 +185,14 @@ heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale, const
   if (!aligned(q_scale, 4) || !aligned(k_scale, 16) || !aligned(v_scale, 16) || !aligned(kv_len, 4))
     return HEAL_ERR_INVALID_ARGUMENT;
   if (qk_int_out && !aligned(qk_int_out, 8)) return HEAL_ERR_INVALID_ARGUMENT;
-  if (workspace_bytes < attention_workspace_bytes(B, Hq, Tq, Tmax)) return HEAL_ERR_INVALID_ARGUMENT;
+  if (workspace_bytes < heal_attention_workspace_bytes_gqa(B, Hq, Hkv, Tq, Tmax)) return HEAL_ERR_INVALID_ARGUMENT;
+  if (prefill) {
+    const heal_status_t st =
+        attention_prefill_launch(q, q_scale, k_cache, k_scale, v_cache, v_scale, B, Hq, Hkv, Tq, kv_len, Tmax,
+                                 softmax_scale, causal, out, workspace, workspace_bytes, qk_int_out, (cudaStream_t)stream);
+    if (st == HEAL_ERR_CUDA) (void)cudaGetLastError();
+    return st;
+  }
   const heal_status_t st = attention_launch(q, q_scale, k_cache, k_scale, v_cache, v_scale, B, Hq, Hkv, D, Tq, kv_len,
                                             Tmax, softmax_scale, causal, out, workspace, workspace_bytes,
                                             qk_int_out, (cudaStream_t)stream);

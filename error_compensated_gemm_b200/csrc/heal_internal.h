@@ -53,4 +53,11 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
                                const int32_t* kv_len, int Tmax, float scale, int causal, float* out,
                                void* ws, size_t ws_bytes, int64_t* qk_out, cudaStream_t s);
 
+// Many query rows per KV head ((Hq/Hkv) * Tq > 8, D = 128): the tcgen05 kernel.
+size_t attention_prefill_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tmax);
+heal_status_t attention_prefill_launch(const int16_t* q, const float* qs, const int16_t* k, const float* ks,
+                                       const int16_t* v, const float* vs, int B, int Hq, int Hkv, int Tq,
+                                       const int32_t* kv_len, int Tmax, float scale, int causal, float* out,
+                                       void* ws, size_t ws_bytes, int64_t* qk_out, cudaStream_t s);
+
 }  // namespace heal

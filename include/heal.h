@@ -158,14 +158,22 @@ heal_status_t heal_kv_quantize_int16(const void* x, int x_is_bf16,
  *   out        : device float32 [B, Hq, Tq, D]
  * Query head h reads KV head h / (Hq/Hkv).  Query i sits at position kv_len - Tq + i;
  * with causal = 1 it sees tokens t <= its position.  QK^T is the exact integer dot
- * product (each INT16 value byte-split into two FP16 values, three FP16 tensor-core
- * products, combined in int64); logit = fp32(S_int * (s_q * s_k) * softmax_scale)
- * evaluated in double; FP32 online softmax; PV with P split into two FP16 parts and V
- * byte-split.  The context is cut into chunks whose partial results are merged in
- * ascending chunk order.
- * Limits: D in {64, 128}; Hq % Hkv == 0; (Hq/Hkv) * Tq <= 8; Tmax % 64 == 0;
+ * product (each INT16 value byte-split into a signed high byte and an unsigned low byte,
+ * four 8-bit integer tensor-core products, combined in int64); FP32 online softmax; PV
+ * with P split into two FP16 parts and V byte-split into two exact FP16 values.
+ * Two kernels, chosen by the number of query rows per KV head, R = (Hq/Hkv) * Tq:
+ *   R <= 8 (decode): logit = fp32(S_int * (s_q * s_k) * softmax_scale) evaluated in
+ *     double; the context is cut into chunks whose partial results are merged in
+ *     ascending chunk order.
+ *   R > 8 (prefill, D = 128 only): 128 query rows per tile on the tcgen05 tensor cores;
+ *     logit * log2(e) = fp32(fp32(S_int) * s_k) * fp32(s_q * softmax_scale * log2(e))
+ *     in FP32; a conversion pass first writes the byte planes of Q, K and V into the
+ *     workspace.
+ * Both are deterministic (identical results from run to run).
+ * Limits: D in {64, 128} (128 when R > 8); Hq % Hkv == 0; Tmax % 64 == 0;
  * q, the caches, k_scale, v_scale, out and workspace 16-byte aligned.
- * workspace  : device, >= heal_attention_workspace_bytes(B, Hq, Tq, Tmax) bytes
+ * workspace  : device, >= heal_attention_workspace_bytes_gqa(B, Hq, Hkv, Tq, Tmax) bytes
+ *              (heal_attention_workspace_bytes(B, Hq, Tq, Tmax) is an upper bound)
  * qk_int_out : nullable test hook, int64 [B, Hq, Tq, Tmax]; when given, the exact
  *              S_int of every visible (query, token) pair is written there.          */
 heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale,
@@ -177,7 +185,10 @@ heal_status_t heal_attention_int16(const int16_t* q, const float* q_scale,
                                    void* workspace, size_t workspace_bytes,
                                    int64_t* qk_int_out, heal_stream_t stream);
 
-/* Scratch bytes for heal_attention_int16 (host-only, no CUDA call).                   */
+/* Scratch bytes for heal_attention_int16 (host-only, no CUDA call).  The _gqa form is
+ * exact for the given Hkv; the short form is an upper bound valid for every Hkv that
+ * divides Hq (for Tq = 1: every Hkv with Hq/Hkv <= 8).  0 for invalid sizes.         */
+size_t heal_attention_workspace_bytes_gqa(int B, int Hq, int Hkv, int Tq, int Tmax);
 size_t heal_attention_workspace_bytes(int B, int Hq, int Tq, int Tmax);
 
 /* Fixed-scratch variant of heal_attention_int16.  The paper has no counterpart to this
@@ -197,9 +208,11 @@ size_t heal_attention_workspace_bytes(int B, int Hq, int Tq, int Tmax);
  *     needs to start at zero: every partial result a call reads was written earlier in the
  *     same call.  Calls whose kernels overlap on the GPU (other streams, other host
  *     threads) race on the array and corrupt each other's results: serialise them.
- *   - Size limit: B * Hq * Tq <= 7939 (the scratch the workspace variant would need,
- *     heal_attention_workspace_bytes(B, Hq, Tq, Tmax), must fit the array).  Larger
- *     problems return HEAL_ERR_UNSUPPORTED and launch nothing.                            */
+ *   - Size limit: the scratch the workspace variant would need,
+ *     heal_attention_workspace_bytes_gqa(B, Hq, Hkv, Tq, Tmax), must fit the array (for
+ *     decode shapes: B * Hq * Tq <= 7939; the prefill kernel's byte planes need
+ *     6 * B * Hkv * Tmax * 128 + 2 * B * Hq * Tq * 128 bytes).  Larger problems return
+ *     HEAL_ERR_UNSUPPORTED and launch nothing.                                            */
 #define HEAL_ATTN_STATIC_SCRATCH_BYTES (8u << 20)
 heal_status_t heal_attention_int16_noalloc(const int16_t* q, const float* q_scale,
                                            const int16_t* k_cache, const float* k_scale,
@@ -222,7 +235,10 @@ heal_status_t heal_attention_int16_noalloc(const int16_t* q, const float* q_scal
  *     FP32 tables [max_pos, D/2] made by the caller.
  *   heal_swiglu: out[i, j] = silu(gu[i, j]) * gu[i, F + j], gu [n, 2F], out [n, F].
  *   heal_add: x[e] += y[e] for e < n.
- *   heal_argmax: out[r] = index of the largest x[r, :] (lowest index on ties), x [rows, n]. */
+ *   heal_argmax: out[r] = index of the largest x[r, :] (lowest index on ties), x [rows, n].
+ *   heal_heads_to_rows: y[b, t, h, :] = x[b, h, t, :] for x [B, H, T, D] (an attention
+ *     output) and y [B, T, H, D]; D a multiple of 4 up to 1024, x and y 16-byte aligned
+ *     and distinct. */
 heal_status_t heal_embedding_gather(const float* table, int vocab, int H, const int32_t* ids,
                                     int n, float* out, heal_stream_t stream);
 heal_status_t heal_rmsnorm(const float* x, const float* w, int n, int H, float eps, float* y,
@@ -233,6 +249,7 @@ heal_status_t heal_rope(float* x, int n, int heads, int D, int64_t row_stride,
 heal_status_t heal_swiglu(const float* gate_up, int n, int F, float* out, heal_stream_t stream);
 heal_status_t heal_add(float* x, const float* y, int64_t n, heal_stream_t stream);
 heal_status_t heal_argmax(const float* x, int rows, int n, int32_t* out, heal_stream_t stream);
+heal_status_t heal_heads_to_rows(const float* x, int B, int H, int T, int D, float* y, heal_stream_t stream);
 
 /* Synchronises `stream`, returns HEAL_ERR_TIMEOUT if any kernel of this library gave up
  * on a bounded wait since the last call, HEAL_ERR_INVALID_ARGUMENT if a kernel met an
