@@ -839,13 +839,13 @@ def main():
             dec_res["prefill_ms"], dec_res["decode_ms_per_token"] = max_over_ranks(
                 [dec_res["prefill_ms"], dec_res["decode_ms_per_token"]], device=dev)
 
+    # DRAM bytes of one prefill launch from the committed ncu summary (a full-size capture)
     traffic = None
-    prof = os.path.join(ROOT, "profiles", "traffic.json")
-    if os.path.exists(prof):
-        try:
-            traffic = json.load(open(prof)).get("heal_gemm_prefill_bytes_per_launch")
-        except Exception:
-            traffic = None
+    prof = os.path.join(ROOT, "profiles", "heal_gemm_pair_kernel_prefill_traffic.md")
+    if os.path.exists(prof) and PREFILL == (4096, 4096, 14336):
+        for ln in open(prof):
+            if ln.startswith("bytes_per_launch:"):
+                traffic = int(ln.split(":")[1])
 
     if rank == 0:
         line = {

@@ -41,6 +41,7 @@
 #include <cuda_fp16.h>
 
 #include <cmath>
+#include <type_traits>
 
 #include "heal_internal.h"
 #include "heal_ptx.cuh"
@@ -55,7 +56,15 @@ constexpr int kPN = 64;             // tokens per key block
 constexpr int kKSt = 2;             // K plane stages
 constexpr int kVSt = 2;             // V plane stages
 constexpr int kScSt = 4;            // scale stages
-constexpr int kPThreads = 320;      // 10 warps
+#ifndef HEAL_PREFILL_SM_WARPS
+#define HEAL_PREFILL_SM_WARPS 8
+#endif
+constexpr int kSmWarps = HEAL_PREFILL_SM_WARPS;   // softmax warps: 8 or 16
+constexpr int kGroups = kSmWarps / 4;             // warps sharing one TMEM lane quarter
+constexpr int kTokPer = kPN / kGroups;            // tokens of a block per softmax thread
+constexpr int kOCols = kPD / kGroups;             // columns of O per softmax thread
+static_assert(kSmWarps == 8 || kSmWarps == 16, "8 or 16 softmax warps");
+constexpr int kPThreads = (2 + kSmWarps) * 32;
 constexpr int kSmWarp0 = 2;         // first softmax warp
 constexpr float kLog2eP = 1.4426950408889634f;
 
@@ -70,9 +79,9 @@ constexpr int kOffP = kOffV + kVSt * kVStage;                // per buffer: Phi 
 constexpr int kPBuf = 2 * kPM * kPN * 2;
 constexpr int kOffSc = kOffP + 2 * kPBuf;                    // per stage: 64 K scales, 64 V scales
 constexpr int kScStage = 2 * kPN * 4;
-constexpr int kOffRed = kOffSc + kScSt * kScStage;           // [2 buffers][2 halves][128] block maxima
-constexpr int kOffL = kOffRed + 2 * 2 * kPM * 4;             // [2 halves][128] row sums
-constexpr int kOffBar = kOffL + 2 * kPM * 4;
+constexpr int kOffRed = kOffSc + kScSt * kScStage;           // [2 buffers][kGroups][128] block maxima
+constexpr int kOffL = kOffRed + 2 * kGroups * kPM * 4;       // [kGroups][128] row sums
+constexpr int kOffBar = kOffL + kGroups * kPM * 4;
 // barriers: qfull, kfull[kKSt], kfree[kKSt], vfull[kVSt], vfree[kVSt], scfull[kScSt],
 // scfree[kScSt], sfull[2], sfree[2], pready[2], pfree[2], odone, drain, mx[2][4] (block
 // maxima exchanged by the two warps of a lane quarter), fin[4] (their row sums), ofree
@@ -87,6 +96,7 @@ struct PrefillArgs {
   const float* vs;        // [B, Hkv, Tmax]
   const int32_t* kv_len;  // [B]
   const int* E;           // [B, Hkv] (conversion pass output)
+  const float* cv;        // [B, Hkv, Tmax] s_v * 2^E, 0 past kv_len (conversion pass output)
   long long* qk_out;      // nullable [B, Hq, Tq, Tmax]
   float* out;             // [B, Hq, Tq, 128]
   int B, Hq, Hkv, G, Tq, Tmax, nqt, causal;
@@ -107,10 +117,17 @@ struct PlanesArgs {
   uint8_t* qhi;           // [B*Hq*Tq, 128]
   uint8_t* qlo;
   int* E;                 // [B, Hkv]
+  float* cv;              // [B, Hkv, Tmax]
   long long nk8;          // K/V elements / 8
   long long nq8;          // Q elements / 8
   int B, Hkv, Tmax;
 };
+
+// x * 2^e exactly for |e| <= 252 (two steps, each a normal power of two).
+__device__ __forceinline__ float mul_pow2_p(float x, int e) {
+  const int e1 = e / 2, e2 = e - e1;
+  return __fmul_rn(__fmul_rn(x, __int_as_float((127 + e1) << 23)), __int_as_float((127 + e2) << 23));
+}
 
 // Eight int16 values (a uint4) -> their high bytes and low bytes (two uint2).
 __device__ __forceinline__ void bytes8(const uint4 w, uint2& hi, uint2& lo) {
@@ -173,7 +190,9 @@ __global__ void __launch_bounds__(256) heal_attn_planes_kernel(const PlanesArgs 
   } else {
     // E of (b, hkv) = blockIdx.x: the largest V scale of the visible tokens times 2^E in
     // [32, 64).  V scales are non-negative, so their bit patterns order like the floats.
+    // Then cv = s_v * 2^E for the visible tokens and 0 for the rest of the cache rows.
     __shared__ unsigned int wmax[8];
+    __shared__ int e_sh;
     const int p = blockIdx.x;
     if (p >= a.B * a.Hkv) return;
     const int b = p / a.Hkv;
@@ -188,16 +207,29 @@ __global__ void __launch_bounds__(256) heal_attn_planes_kernel(const PlanesArgs 
       unsigned int m = 0u;
       for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, wmax[w]);
       const float smax = __uint_as_float(m);
-      a.E[p] = (smax > 0.0f) ? 5 - ilogbf(smax) : 0;
+      e_sh = (smax > 0.0f) ? 5 - ilogbf(smax) : 0;
+      a.E[p] = e_sh;
     }
+    __syncthreads();
+    const int E = e_sh;
+    float* cv = a.cv + (long long)p * a.Tmax;
+    for (int t = threadIdx.x; t < a.Tmax; t += blockDim.x) cv[t] = t < klen ? mul_pow2_p(__ldg(s + t), E) : 0.0f;
   }
 }
 
-// x * 2^e exactly for |e| <= 252 (two steps, each a normal power of two).
-__device__ __forceinline__ float mul_pow2_p(float x, int e) {
-  const int e1 = e / 2, e2 = e - e1;
-  return __fmul_rn(__fmul_rn(x, __int_as_float((127 + e1) << 23)), __int_as_float((127 + e2) << 23));
+// n as a float for |n| < 2^22, exactly: the bits of 1.5 * 2^23 + n, minus 1.5 * 2^23.
+__device__ __forceinline__ float small_int_to_float(int n) {
+  return __fsub_rn(__int_as_float(0x4B400000 + n), 12582912.0f);
 }
+
+// 2^x with the hardware approximation (ex2.approx, relative error about 2^-22; results
+// below 2^-126 flush to zero); 2^-inf = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) { return smem_desc_sw128(addr, 16, 1024); }
 __device__ __forceinline__ uint64_t vdesc(uint32_t addr) { return smem_desc_sw128(addr, 8192, 1024); }
@@ -254,19 +286,19 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
     for (int i = 0; i < kScSt; ++i) {
       mbar_init(&scfull[i], 1);
-      mbar_init(&scfree[i], 8);
+      mbar_init(&scfree[i], kSmWarps);
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sfull[i], 1);
-      mbar_init(&sfree[i], 8);
-      mbar_init(&pready[i], 8);
+      mbar_init(&sfree[i], kSmWarps);
+      mbar_init(&pready[i], kSmWarps);
       mbar_init(&pfree[i], 1);
     }
     mbar_init(odone, 1);
     mbar_init(drain, 1);
-    for (int i = 0; i < 8; ++i) mbar_init(&mx[i], 2);
-    for (int i = 0; i < 4; ++i) mbar_init(&fin[i], 2);
-    mbar_init(ofree, 8);
+    for (int i = 0; i < 8; ++i) mbar_init(&mx[i], kGroups);
+    for (int i = 0; i < 4; ++i) mbar_init(&fin[i], kGroups);
+    mbar_init(ofree, kSmWarps);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -296,7 +328,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
       tma_prefetch_desc(&tv_h);
       const int kvrow0 = (b * a.Hkv + hkv) * a.Tmax;
       const float* ksrc = a.ks + (long long)(b * a.Hkv + hkv) * a.Tmax;
-      const float* vsrc = a.vs + (long long)(b * a.Hkv + hkv) * a.Tmax;
+      const float* vsrc = a.cv + (long long)(b * a.Hkv + hkv) * a.Tmax;
       mbar_arrive_expect_tx(qfull, 2 * kPM * kPD);
       tma_load_3d(sm + kOffQhi, &tq_hi, qfull, 0, row0, bh);
       tma_load_3d(sm + kOffQlo, &tq_lo, qfull, 0, row0, bh);
@@ -396,37 +428,48 @@ __global__ void __launch_bounds__(kPThreads, 1)
     }
   } else {
     // ------------------------------ softmax warps ------------------------------
-    const int sw = warp - kSmWarp0;          // 0..7
+    const int sw = warp - kSmWarp0;          // 0 .. kSmWarps-1
     const int qd = warp & 3;                 // TMEM lane quarter this warp may access
-    const int hf = sw >> 2;                  // token half of each block, column half of O
+    const int hf = sw >> 2;                  // token group of each block, column group of O
     const int r = qd * 32 + lane;            // query row within the tile
     const int tq = row0 + r;
     const bool real = tq < a.Tq;
     const int pos = klen - a.Tq + tq;
     const uint32_t tl_addr = tbase + ((uint32_t)(qd * 32) << 16);
-    const float qcoef = real ? __fmul_rn(__fmul_rn(__ldg(a.qs + (long long)bh * a.Tq + tq), a.scale), kLog2eP) : 0.0f;
+    // logit * log2(e) = fp32(S) * s_k * qcoef; the scores are kept as x' = fp32(S) * s_k and
+    // qcoef enters through the row maximum and one FMA per exponent.  qcoef = 0 (an all-zero
+    // query row, whose S is 0) or a padding row uses 1 instead: x' is then 0 (or -inf when
+    // masked) either way, and no 0 * inf can occur.
+    float qcoef = real ? __fmul_rn(__fmul_rn(__ldg(a.qs + (long long)bh * a.Tq + tq), a.scale), kLog2eP) : 1.0f;
+    if (!(qcoef > 0.0f)) qcoef = 1.0f;
     const int E = __ldg(a.E + b * a.Hkv + hkv);
     long long* qk_row = (a.qk_out != nullptr && real) ? a.qk_out + ((long long)bh * a.Tq + tq) * a.Tmax : nullptr;
     float* red = reinterpret_cast<float*>(sm + kOffRed);
     float* lsm = reinterpret_cast<float*>(sm + kOffL);
     float m_ref = -INFINITY, l = 0.0f;
-    float o_acc[64];                         // this thread's 64 columns of O (FP32, round-to-nearest)
+    float o_acc[kOCols];                     // this thread's columns of O (FP32, round-to-nearest)
 #pragma unroll
-    for (int i = 0; i < 64; ++i) o_acc[i] = 0.0f;
+    for (int i = 0; i < kOCols; ++i) o_acc[i] = 0.0f;
     float alpha_j = 1.0f;                    // rescale applied at the current block
-    const uint32_t ob = tl_addr + 384 + hf * 64;
+    const uint32_t ob = tl_addr + 384 + hf * kOCols;
     // O += the product of block jj (complete once PV(jj) has committed), then * alpha
     auto take_block = [&](int jj, float alpha) -> bool {
       if (!mbar_wait(odone, (uint32_t)jj & 1u, abort_flag, a.status, 323)) return false;
       tc_fence_after();
+      const bool scaled = __any_sync(0xffffffffu, alpha != 1.0f);
 #pragma unroll
-      for (int c16 = 0; c16 < 4; ++c16) {
+      for (int c16 = 0; c16 < kOCols / 16; ++c16) {
         uint32_t o[16];
         tmem_ld16(ob + c16 * 16, o);
         tmem_ld_wait();
+        if (scaled) {
 #pragma unroll
-        for (int i = 0; i < 16; ++i)
-          o_acc[c16 * 16 + i] = __fmul_rn(__fadd_rn(o_acc[c16 * 16 + i], __uint_as_float(o[i])), alpha);
+          for (int i = 0; i < 16; ++i)
+            o_acc[c16 * 16 + i] = __fmul_rn(__fadd_rn(o_acc[c16 * 16 + i], __uint_as_float(o[i])), alpha);
+        } else {
+#pragma unroll
+          for (int i = 0; i < 16; ++i) o_acc[c16 * 16 + i] = __fadd_rn(o_acc[c16 * 16 + i], __uint_as_float(o[i]));
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -443,45 +486,79 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       tc_fence_after();
       const float* scs = reinterpret_cast<const float*>(sm + kOffSc + c * kScStage);   // K scales, then V scales
-      float x[32];
-      const uint32_t sbase = tl_addr + sb * 192 + hf * 32;
+      float x[kTokPer];
+      const uint32_t sbase = tl_addr + sb * 192 + hf * kTokPer;
+      // every token of this block visible to every row of the tile: no per-element mask
+      const int tlast = j * kPN + kPN - 1;
+      const bool full = tlast < klen && (!a.causal || tlast <= klen - a.Tq + row0);
+      auto logits = [&](auto mask_c, auto hook_c) {
+        constexpr bool kMask = decltype(mask_c)::value, kHook = decltype(hook_c)::value;
 #pragma unroll
-      for (int q16 = 0; q16 < 2; ++q16) {
-        uint32_t rh[16], rx[16], rl[16];
-        tmem_ld16(sbase + q16 * 16, rh);
-        tmem_ld16(sbase + 64 + q16 * 16, rx);
-        tmem_ld16(sbase + 128 + q16 * 16, rl);
-        tmem_ld_wait();
+        for (int q8 = 0; q8 < kTokPer / 8; ++q8) {
+          uint32_t rh[8], rx[8], rl[8];
+          tmem_ld8(sbase + q8 * 8, rh);
+          tmem_ld8(sbase + 64 + q8 * 8, rx);
+          tmem_ld8(sbase + 128 + q8 * 8, rl);
+          // K scales of these 8 tokens (broadcast shared-memory loads)
+          const float4 k0 = *reinterpret_cast<const float4*>(scs + hf * kTokPer + q8 * 8);
+          const float4 k1 = *reinterpret_cast<const float4*>(scs + hf * kTokPer + q8 * 8 + 4);
+          const float ksv[8] = {k0.x, k0.y, k0.z, k0.w, k1.x, k1.y, k1.z, k1.w};
+          tmem_ld_wait();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int tb = hf * 32 + q16 * 16 + i;   // token within the block
-          const int t = j * kPN + tb;
-          const long long S = ((long long)(int)rh[i] << 16) + ((long long)(int)rx[i] << 8) + (long long)(int)rl[i];
-          const bool vis = real && t < klen && (!a.causal || t <= pos);
-          float xv = -INFINITY;
-          if (vis) {
-            xv = __fmul_rn(__fmul_rn(__ll2float_rn(S), scs[tb]), qcoef);
-            if (qk_row) qk_row[t] = S;
+          for (int i = 0; i < 8; ++i) {
+            const int tb = hf * kTokPer + q8 * 8 + i;   // token within the block
+            const int t = j * kPN + tb;
+            // S = 65536*S_hh + 256*S_x + S_ll = 65536*A + L with |A| < 2^22, 0 <= L < 2^16
+            const int low = (int)rx[i] * 256 + (int)rl[i];   // |low| < 2^31 for head_dim 128
+            const int A = (int)rh[i] + (low >> 16);
+            const int L = low & 0xFFFF;
+            const float sf = __fmaf_rn(small_int_to_float(A), 65536.0f, small_int_to_float(L));   // fp32_rn(S)
+            float xv = __fmul_rn(sf, ksv[i]);
+            bool vis = true;
+            if constexpr (kMask) {
+              vis = real && t < klen && (!a.causal || t <= pos);
+              if (!vis) xv = -INFINITY;
+            }
+            if constexpr (kHook) {
+              if (vis && qk_row) qk_row[t] = (long long)A * 65536LL + (long long)L;
+            }
+            x[q8 * 8 + i] = xv;
           }
-          x[q16 * 16 + i] = xv;
         }
+      };
+      if (a.qk_out == nullptr) {
+        if (full) logits(std::false_type{}, std::false_type{});
+        else logits(std::true_type{}, std::false_type{});
+      } else {
+        logits(std::true_type{}, std::true_type{});
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&sfree[sb]);   // this half of the S buffer is in registers
 
       // the block's row maximum over both token halves
-      float bm = x[0];
+      float bm;
+      {
+        float m16[16];
 #pragma unroll
-      for (int i = 1; i < 32; ++i) bm = fmaxf(bm, x[i]);
-      red[(sb * 2 + hf) * kPM + r] = bm;
+        for (int i = 0; i < 16; ++i) m16[i] = (kTokPer == 32) ? fmaxf(x[i], x[(i + 16) % kTokPer]) : x[i];
+#pragma unroll
+        for (int w = 8; w >= 1; w >>= 1)
+#pragma unroll
+          for (int i = 0; i < w; ++i) m16[i] = fmaxf(m16[i], m16[i + w]);
+        bm = m16[0];
+      }
+      red[(sb * kGroups + hf) * kPM + r] = bm;
       __syncwarp();
       if (lane == 0) mbar_arrive(&mx[sb * 4 + qd]);
       if (!mbar_wait(&mx[sb * 4 + qd], (uint32_t)(j >> 1) & 1u, abort_flag, a.status, 322)) {
         ok = false;
         break;
       }
-      const float m_blk = fmaxf(red[(sb * 2) * kPM + r], red[(sb * 2 + 1) * kPM + r]);
+      float m_blk = red[(sb * kGroups) * kPM + r];
+#pragma unroll
+      for (int gi = 1; gi < kGroups; ++gi) m_blk = fmaxf(m_blk, red[(sb * kGroups + gi) * kPM + r]);
+      m_blk = __fmul_rn(m_blk, qcoef);          // qcoef > 0: the maximum of fp32(x' * qcoef)
       // lazy maximum: move the reference only when this block exceeds it by more than 2^8
       const bool need = m_blk > m_ref + 8.0f;
       alpha_j = 1.0f;
@@ -491,26 +568,28 @@ __global__ void __launch_bounds__(kPThreads, 1)
       }
       l = __fmul_rn(l, alpha_j);
 
-      // P = 2^(x - m_ref) <= 2^8; P' = P * s_v * 2^E; FP16 P_hi and residual, two tokens a word
-      uint32_t phi[16], prr[16];
-      const float* svs = scs + kPN;
+      // P = 2^(x - m_ref) <= 2^8; P' = P * (s_v * 2^E); FP16 P_hi and residual, two tokens a word
+      uint32_t phi[kTokPer / 2], prr[kTokPer / 2];
+      const float* cvs = scs + kPN;             // s_v * 2^E of the block's tokens (0 past kv_len)
+      // a row with no visible token so far keeps m_ref = -inf: subtract 0 instead (P = 0)
+      const float msub = (m_ref == -INFINITY) ? 0.0f : m_ref;
+      const float nsub = -msub;
+      float ls[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-      for (int i = 0; i < 32; i += 2) {
-        float p0 = 0.0f, p1 = 0.0f;
-        if (m_ref != -INFINITY) {
-          p0 = exp2f(x[i] - m_ref);
-          p1 = exp2f(x[i + 1] - m_ref);
-        }
-        l = __fadd_rn(__fadd_rn(l, p0), p1);
-        const int tb = hf * 32 + i;
-        const float q0 = (p0 != 0.0f) ? __fmul_rn(p0, mul_pow2_p(svs[tb], E)) : 0.0f;
-        const float q1 = (p1 != 0.0f) ? __fmul_rn(p1, mul_pow2_p(svs[tb + 1], E)) : 0.0f;
+      for (int i = 0; i < kTokPer; i += 2) {
+        const float p0 = fast_exp2(__fmaf_rn(x[i], qcoef, nsub));
+        const float p1 = fast_exp2(__fmaf_rn(x[i + 1], qcoef, nsub));
+        ls[(i >> 1) & 3] = __fadd_rn(ls[(i >> 1) & 3], __fadd_rn(p0, p1));
+        const float2 c2 = *reinterpret_cast<const float2*>(cvs + hf * kTokPer + i);
+        const float q0 = __fmul_rn(p0, c2.x);
+        const float q1 = __fmul_rn(p1, c2.y);
         const __half2 hh = __floats2half2_rn(q0, q1);
         const float2 hv = __half22float2(hh);
         const __half2 rr = __floats2half2_rn(__fsub_rn(q0, hv.x), __fsub_rn(q1, hv.y));
         phi[i >> 1] = *reinterpret_cast<const uint32_t*>(&hh);
         prr[i >> 1] = *reinterpret_cast<const uint32_t*>(&rr);
       }
+      l = __fadd_rn(l, __fadd_rn(__fadd_rn(ls[0], ls[1]), __fadd_rn(ls[2], ls[3])));
       __syncwarp();
       if (lane == 0) mbar_arrive(&scfree[c]);
       // the P buffer was last read by PV(j-2)
@@ -521,8 +600,8 @@ __global__ void __launch_bounds__(kPThreads, 1)
       // K-major A operand, 128-byte swizzle: row r, 16-byte chunk k at k ^ (r & 7)
       uint8_t* pb = sm + kOffP + sb * kPBuf + r * 128;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int phys = ((hf * 4 + cc) ^ (r & 7)) * 16;
+      for (int cc = 0; cc < kTokPer / 8; ++cc) {
+        const int phys = ((hf * (kTokPer / 8) + cc) ^ (r & 7)) * 16;
         *reinterpret_cast<uint4*>(pb + phys) = make_uint4(phi[4 * cc], phi[4 * cc + 1], phi[4 * cc + 2], phi[4 * cc + 3]);
         *reinterpret_cast<uint4*>(pb + kPM * kPN * 2 + phys) =
             make_uint4(prr[4 * cc], prr[4 * cc + 1], prr[4 * cc + 2], prr[4 * cc + 3]);
@@ -544,13 +623,15 @@ __global__ void __launch_bounds__(kPThreads, 1)
     if (lane == 0) mbar_arrive(&fin[qd]);
     if (!mbar_wait(&fin[qd], 0u, abort_flag, a.status, 326)) ok = false;
     ok = __all_sync(0xffffffffu, ok);
-    const float L = __fadd_rn(lsm[r], lsm[kPM + r]);
-    float* dst = real ? a.out + ((long long)bh * a.Tq + tq) * kPD + hf * 64 : nullptr;
+    float L = lsm[r];
+#pragma unroll
+    for (int gi = 1; gi < kGroups; ++gi) L = __fadd_rn(L, lsm[gi * kPM + r]);
+    float* dst = real ? a.out + ((long long)bh * a.Tq + tq) * kPD + hf * kOCols : nullptr;
     if (ok && nb > 0) {
       if (dst) {
         float4* d4 = reinterpret_cast<float4*>(dst);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
+        for (int i = 0; i < kOCols / 4; ++i) {
           float v[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u)
@@ -561,7 +642,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
     } else if (ok && dst) {
       // no visible token for this tile (causal with kv_len < Tq): zeros
       float4* d4 = reinterpret_cast<float4*>(dst);
-      for (int i = 0; i < 16; ++i) d4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int i = 0; i < kOCols / 4; ++i) d4[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
     }
   }
 
@@ -578,7 +659,7 @@ __global__ void __launch_bounds__(kPThreads, 1)
 size_t attention_prefill_workspace_bytes(int B, int Hq, int Hkv, int Tq, int Tmax) {
   const size_t nk = (size_t)B * Hkv * Tmax * kPD;
   const size_t nq = (size_t)B * Hq * Tq * kPD;
-  return 6 * nk + 2 * nq + (((size_t)B * Hkv * sizeof(int) + 127) & ~(size_t)127);
+  return 6 * nk + 2 * nq + (size_t)B * Hkv * Tmax * sizeof(float) + (((size_t)B * Hkv * sizeof(int) + 127) & ~(size_t)127);
 }
 
 heal_status_t attention_prefill_launch(const int16_t* q, const float* qs, const int16_t* k, const float* ks,
@@ -608,7 +689,8 @@ heal_status_t attention_prefill_launch(const int16_t* q, const float* qs, const 
   pa.vl = reinterpret_cast<__half*>(w + 4 * nk);
   pa.qhi = w + 6 * nk;
   pa.qlo = w + 6 * nk + nq;
-  pa.E = reinterpret_cast<int*>(w + 6 * nk + 2 * nq);
+  pa.cv = reinterpret_cast<float*>(w + 6 * nk + 2 * nq);
+  pa.E = reinterpret_cast<int*>(w + 6 * nk + 2 * nq + (size_t)kv_rows * sizeof(float));
   pa.nk8 = (long long)(nk / 8);
   pa.nq8 = (long long)(nq / 8);
   pa.B = B;
@@ -621,6 +703,7 @@ heal_status_t attention_prefill_launch(const int16_t* q, const float* qs, const 
   a.vs = vs;
   a.kv_len = kv_len;
   a.E = pa.E;
+  a.cv = pa.cv;
   a.qk_out = reinterpret_cast<long long*>(qk_out);
   a.out = out;
   a.B = B;

@@ -147,6 +147,19 @@ int grid_for(long long n) {
 }
 
 
+// y[b, t, h, :] = x[b, h, t, :]: attention output [B, H, T, D] to token rows [B*T, H*D]
+__global__ void heads_to_rows_kernel(const float4* __restrict__ x, float4* __restrict__ y, int H, int T, int D4,
+                                     long long rows) {
+  pdl_launch_dependents();
+  pdl_wait_prerequisites();
+  const long long r = (long long)blockIdx.x * (blockDim.x / D4) + threadIdx.x / D4;   // source row (b, h, t)
+  const int e = threadIdx.x % D4;
+  if (r >= rows || threadIdx.x >= (blockDim.x / D4) * D4) return;
+  const long long t = r % T, bh = r / T;
+  const long long h = bh % H, b = bh / H;
+  y[((b * T + t) * H + h) * D4 + e] = x[r * D4 + e];
+}
+
 }  // namespace
 }  // namespace heal
 
@@ -194,6 +207,21 @@ heal_status_t heal_add(float* x, const float* y, int64_t n, heal_stream_t stream
   if (!x || !y) return HEAL_ERR_INVALID_ARGUMENT;
   return launch_pdl(add_kernel, dim3(grid_for(n)), dim3(kThreads), 0, (cudaStream_t)stream, x, y, (long long)n) ==
                  cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+}
+
+heal_status_t heal_heads_to_rows(const float* x, int B, int H, int T, int D, float* y, heal_stream_t stream) {
+  if (B < 0 || H < 0 || T < 0 || D <= 0 || D % 4 != 0 || D > 1024) return HEAL_ERR_INVALID_ARGUMENT;
+  const long long rows = (long long)B * H * T;
+  if (rows == 0) return HEAL_OK;
+  if (!x || !y || x == y) return HEAL_ERR_INVALID_ARGUMENT;
+  if ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(y)) & 15u) return HEAL_ERR_INVALID_ARGUMENT;
+  const int D4 = D / 4;
+  const int per = kThreads / D4 > 0 ? kThreads / D4 : 1;   // source rows per block
+  const long long blocks = (rows + per - 1) / per;
+  if (blocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
+  return launch_pdl(heads_to_rows_kernel, dim3((unsigned)blocks), dim3(per * D4), 0, (cudaStream_t)stream,
+                    reinterpret_cast<const float4*>(x), reinterpret_cast<float4*>(y), H, T, D4, rows) == cudaSuccess
+             ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
 heal_status_t heal_argmax(const float* x, int rows, int n, int32_t* out, heal_stream_t stream) {

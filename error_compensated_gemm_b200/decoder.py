@@ -6,8 +6,10 @@ glue (embedding, RMSNorm, RoPE, SwiGLU, residual, argmax) is the library's FP32 
 the "HEAL-Full" pipeline of the gist.science technical summary (Results), on synthetic
 weights.  PyTorch only allocates buffers and supplies the stream.
 
-Prefill runs the projections and MLP on all prompt rows at once (M = prompt length) and
-attention one query position at a time with the decode kernel (kv_len = position + 1).
+Prefill runs the projections, the MLP and causal attention on all prompt rows at once
+(M = prompt length; attention through the library's prefill kernel, queries at positions
+p0 .. p0+n-1 of a context of p0+n tokens).  That kernel is built for head_dim 128; other
+head sizes run prefill attention one query position at a time with the decode kernel.
 """
 import math
 
@@ -43,8 +45,8 @@ class Decoder:
                   (1, c.hidden, c.ffn), (1, c.vocab, c.hidden)]
         ws = max(H.heal_gemm_workspace_bytes(m, n, k) for (m, n, k) in shapes)
         self.gemm_ws = torch.empty(max(1, ws // 4), dtype=f32, device=device)
-        self.attn_ws = torch.empty(H.heal_attention_workspace_bytes(1, c.heads, 1, Tmax) // 4, dtype=f32,
-                                   device=device)
+        self.attn_ws = torch.empty(max(H.heal_attention_workspace_bytes_gqa(1, c.heads, c.kv_heads, q, Tmax)
+                                       for q in (1, self.max_len)) // 4, dtype=f32, device=device)
         self.kv_len = torch.arange(1, Tmax + 1, dtype=torch.int32, device=device)   # kv_len for position t: t + 1
         self.positions = torch.arange(0, Tmax, dtype=torch.int32, device=device)
         self.pos_len = 0
@@ -65,24 +67,44 @@ class Decoder:
         qd = c.heads * c.head_dim
         H.heal_rope(qkv, c.heads, c.head_dim, pos, self.cos, self.sin)                 # q heads
         H.heal_rope(qkv[:, qd:], c.kv_heads, c.head_dim, pos, self.cos, self.sin)      # k heads (in place)
-        # INT16 Q rows [n, Hq, 1, D], K/V into the layer's cache at positions p0 .. p0+n-1
-        q16 = torch.empty(n, c.heads, 1, c.head_dim, dtype=torch.int16, device=d)
-        qsc = torch.empty(n, c.heads, 1, device=d)
+        # INT16 Q (all rows in one call: [1, Hq, n, D]; one position a call: [n, Hq, 1, D]),
+        # K/V into the layer's cache at positions p0 .. p0+n-1
+        one_call = n == 1 or c.head_dim == 128
         R, D = c.qkv_dim, c.head_dim
         kd = c.kv_heads * D
-        H.heal_kv_quantize_int16(qkv.as_strided((n, 1, c.heads, D), (R, R, D, 1), qkv.storage_offset()), q16, qsc)
+        if one_call:
+            q16 = torch.empty(1, c.heads, n, D, dtype=torch.int16, device=d)
+            qsc = torch.empty(1, c.heads, n, device=d)
+            H.heal_kv_quantize_int16(qkv.as_strided((1, n, c.heads, D), (n * R, R, D, 1), qkv.storage_offset()),
+                                     q16, qsc)
+        else:
+            q16 = torch.empty(n, c.heads, 1, D, dtype=torch.int16, device=d)
+            qsc = torch.empty(n, c.heads, 1, device=d)
+            H.heal_kv_quantize_int16(qkv.as_strided((n, 1, c.heads, D), (R, R, D, 1), qkv.storage_offset()),
+                                     q16, qsc)
         H.heal_kv_quantize_int16(qkv.as_strided((1, n, c.kv_heads, D), (n * R, R, D, 1), qkv.storage_offset() + qd),
                                  self.kc[l], self.ks[l], t_offset=p0)
         H.heal_kv_quantize_int16(qkv.as_strided((1, n, c.kv_heads, D), (n * R, R, D, 1),
                                                 qkv.storage_offset() + qd + kd),
                                  self.vc[l], self.vs[l], t_offset=p0)
-        attn = torch.empty(n, c.heads * c.head_dim, device=d)
         scale = 1.0 / math.sqrt(c.head_dim)
-        for i in range(n):
-            t = p0 + i
-            H.heal_attention_int16(q16[i:i + 1], qsc[i:i + 1], self.kc[l], self.ks[l], self.vc[l], self.vs[l],
-                                   self.kv_len[t:t + 1], scale, attn[i:i + 1].view(1, c.heads, 1, c.head_dim),
-                                   self.attn_ws)
+        if not one_call:
+            attn = torch.empty(n, c.heads * D, device=d)
+            for i in range(n):
+                t = p0 + i
+                H.heal_attention_int16(q16[i:i + 1], qsc[i:i + 1], self.kc[l], self.ks[l], self.vc[l], self.vs[l],
+                                       self.kv_len[t:t + 1], scale, attn[i:i + 1].view(1, c.heads, 1, D),
+                                       self.attn_ws)
+        elif n == 1:
+            attn = torch.empty(1, c.heads * D, device=d)
+            H.heal_attention_int16(q16, qsc, self.kc[l], self.ks[l], self.vc[l], self.vs[l],
+                                   self.kv_len[p0:p0 + 1], scale, attn.view(1, c.heads, 1, D), self.attn_ws)
+        else:
+            attn_h = torch.empty(1, c.heads, n, D, device=d)
+            H.heal_attention_int16(q16, qsc, self.kc[l], self.ks[l], self.vc[l], self.vs[l],
+                                   self.kv_len[p0 + n - 1:p0 + n], scale, attn_h, self.attn_ws, causal=True)
+            attn = torch.empty(n, c.heads * D, device=d)
+            H.heal_heads_to_rows(attn_h, attn.view(1, n, c.heads, D))
         o = torch.empty(n, c.hidden, device=d)
         self._linear(attn, self.w[f"wo{l}"], o)
         H.heal_add(h, o)

@@ -8,10 +8,11 @@ no expected value comes from the CUDA path.
   * O is compared with the FP64 definition under the decode tests' bound,
         ||O - O_ref|| / ||O_ref||  <=  4 * (x_max + 8) * 2^-23 + 1e-6.
     The prefill kernel forms logit * log2(e) from fp32(S_int) with two FP32 products
-    (relative error <= 3 * 2^-24 of |x|), evaluates exp2 in FP32 with a reference maximum
-    that may trail the row maximum by up to 8 (P <= 2^8, the same relative precision), and
+    (relative error <= 3 * 2^-24 of |x|), evaluates 2^x with the hardware approximation
+    (relative error about 2^-22) against a reference maximum that may trail the row maximum
+    by up to 8 (P <= 2^8, the same relative precision), and
     adds each 64-token block's tensor-core PV product into FP32 with round-to-nearest, so
-    each weight carries about (1.5 |x| + 8) * 2^-23 of relative error: inside the bound.
+    each weight carries about (1.5 |x| + 10) * 2^-23 of relative error: inside the bound.
 """
 import math
 
@@ -124,7 +125,7 @@ def test_prefill_full_size_sampled_rows():
 
 def test_prefill_workspace_sizes():
     exact = heal.heal_attention_workspace_bytes_gqa(1, 32, 8, 8192, 8192)
-    assert exact == 6 * 8 * 8192 * 128 + 2 * 32 * 8192 * 128 + 128
+    assert exact == 6 * 8 * 8192 * 128 + 2 * 32 * 8192 * 128 + 4 * 8 * 8192 + 128
     assert heal.heal_attention_workspace_bytes(1, 32, 8192, 8192) >= exact
     # a workspace one byte short is refused before any launch
     d = dev()

@@ -118,3 +118,18 @@ def test_config5_decoder_bitwise_and_oracle():
         assert torch.equal(a, b)
     errs = _check_against_oracle(cfg, w, prompt, list(to_np(t1)), l1, check=[511, 512, 513])
     print("config-5 logit errors", errs)
+
+
+def test_heads_to_rows_is_an_exact_transpose():
+    d = dev()
+    g = torch.Generator().manual_seed(21)
+    for (B, Hh, T, D) in ((1, 32, 515, 128), (2, 3, 7, 64), (1, 1, 1, 4)):
+        x = torch.randn(B, Hh, T, D, generator=g)
+        y = torch.full((B, T, Hh, D), float("nan"), device=d)
+        heal.heal_heads_to_rows(x.to(d), y)
+        status_ok()
+        assert torch.equal(to_np_t(y), x.permute(0, 2, 1, 3))
+
+
+def to_np_t(t):
+    return t.detach().cpu()
