@@ -9,9 +9,10 @@
 // four tcgen05.mma.kind::i8 products per 32-wide slice of the head dimension, each exact in
 // its 32-bit TMEM accumulator (for head_dim 128 no partial sum reaches 2^24), combined in
 // int64 by the softmax threads.
-//   logit * log2(e) = fp32 products of fp32(S_int), s_k and (s_q * scale * log2 e)
-// (three FP32 roundings; the decode kernel forms the same value through FP64, the two agree
-// to a few units in the last place).  Online softmax in base 2 with a lazy maximum: the
+//   logit * log2(e) = fp32(fp32(S_int) * s_k) * (s_q * scale * log2 e), the last factor
+// applied inside the exponent's FMA; fp32(S_int) is 65536*S_hh + fp32(256*S_x + S_ll)
+// rounded once more (the decode kernel forms the logit through FP64; the two agree to a
+// few units in the last place).  Online softmax in base 2 with a lazy maximum: the
 // reference maximum of a row moves only when a block's maximum exceeds it by more than 8,
 // so P <= 2^8 and the running O is rescaled only on those blocks.
 //   P' = P * s_v * 2^E, E per (batch, kv head) such that max s_v * 2^E lies in [32, 64);
@@ -241,6 +242,9 @@ __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity, unsig
   (void)mbar_wait(bar, parity, &never, status, site);
 }
 
+// HOOK: also write the exact S_int of every visible pair to qk_out (the test hook); a
+// separate instantiation keeps that path out of the production kernel.
+template <bool HOOK>
 __global__ void __launch_bounds__(kPThreads, 1)
     heal_attn_prefill_kernel(const __grid_constant__ CUtensorMap tq_hi, const __grid_constant__ CUtensorMap tq_lo,
                              const __grid_constant__ CUtensorMap tk_hi, const __grid_constant__ CUtensorMap tk_lo,
@@ -508,11 +512,10 @@ __global__ void __launch_bounds__(kPThreads, 1)
           for (int i = 0; i < 8; ++i) {
             const int tb = hf * kTokPer + q8 * 8 + i;   // token within the block
             const int t = j * kPN + tb;
-            // S = 65536*S_hh + 256*S_x + S_ll = 65536*A + L with |A| < 2^22, 0 <= L < 2^16
-            const int low = (int)rx[i] * 256 + (int)rl[i];   // |low| < 2^31 for head_dim 128
-            const int A = (int)rh[i] + (low >> 16);
-            const int L = low & 0xFFFF;
-            const float sf = __fmaf_rn(small_int_to_float(A), 65536.0f, small_int_to_float(L));   // fp32_rn(S)
+            // S = 65536*S_hh + low, low = 256*S_x + S_ll (|low| < 2^31 for head_dim 128);
+            // fp32(S) with two roundings: fp32(low), then the FMA (S_hh is exact in fp32)
+            const int low = (int)rx[i] * 256 + (int)rl[i];
+            const float sf = __fmaf_rn(small_int_to_float((int)rh[i]), 65536.0f, __int2float_rn(low));
             float xv = __fmul_rn(sf, ksv[i]);
             bool vis = true;
             if constexpr (kMask) {
@@ -520,17 +523,17 @@ __global__ void __launch_bounds__(kPThreads, 1)
               if (!vis) xv = -INFINITY;
             }
             if constexpr (kHook) {
-              if (vis && qk_row) qk_row[t] = (long long)A * 65536LL + (long long)L;
+              if (vis && qk_row) qk_row[t] = (long long)(int)rh[i] * 65536LL + (long long)low;
             }
             x[q8 * 8 + i] = xv;
           }
         }
       };
-      if (a.qk_out == nullptr) {
+      if constexpr (HOOK) {
+        logits(std::true_type{}, std::true_type{});
+      } else {
         if (full) logits(std::false_type{}, std::false_type{});
         else logits(std::true_type{}, std::false_type{});
-      } else {
-        logits(std::true_type{}, std::true_type{});
       }
       tc_fence_before();
       __syncwarp();
@@ -756,8 +759,10 @@ heal_status_t attention_prefill_launch(const int16_t* q, const float* qs, const 
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return HEAL_ERR_CUDA;
   if (!attr_set[dev]) {
-    if (cudaFuncSetAttribute(heal_attn_prefill_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem) !=
-        cudaSuccess)
+    if (cudaFuncSetAttribute(heal_attn_prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(heal_attn_prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, kPSmem) !=
+            cudaSuccess)
       return HEAL_ERR_CUDA;
     attr_set[dev] = true;
   }
@@ -767,8 +772,12 @@ heal_status_t attention_prefill_launch(const int16_t* q, const float* qs, const 
   if (gx < (long long)B * Hkv) gx = (long long)B * Hkv;
   cudaError_t e = launch_pdl(heal_attn_planes_kernel, dim3((unsigned)gx, 4), dim3(256), 0, stream, pa);
   if (e != cudaSuccess) return HEAL_ERR_CUDA;
-  e = launch_pdl(heal_attn_prefill_kernel, dim3((unsigned)(B * Hq * nqt)), dim3(kPThreads), (size_t)kPSmem, stream,
-                 mq_hi, mq_lo, mk_hi, mk_lo, mv_h, mv_l, a);
+  if (qk_out)
+    e = launch_pdl(heal_attn_prefill_kernel<true>, dim3((unsigned)(B * Hq * nqt)), dim3(kPThreads), (size_t)kPSmem,
+                   stream, mq_hi, mq_lo, mk_hi, mk_lo, mv_h, mv_l, a);
+  else
+    e = launch_pdl(heal_attn_prefill_kernel<false>, dim3((unsigned)(B * Hq * nqt)), dim3(kPThreads), (size_t)kPSmem,
+                   stream, mq_hi, mq_lo, mk_hi, mk_lo, mv_h, mv_l, a);
   if (e != cudaSuccess) return HEAL_ERR_CUDA;
   return cudaGetLastError() == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
