@@ -121,6 +121,10 @@ class Workload:
             X, W = synthetic.gemm_prefill(M=M, K=K, N=N, seed_x=0 + so, seed_w=1 + so)
             self.X, self.W = X.to(dev), W.to(dev)
             self.C = torch.empty(M, N, device=dev)
+            # scratch for B's hi and lo parts: the product splits B in one streaming pass,
+            # then runs on the 16-bit parts (the same bits as splitting B inside every tile)
+            self.wsp = torch.empty(heal.heal_gemm_workspace_bytes(M, N, K, b_split_pass=True), dtype=torch.uint8,
+                                   device=dev)
             # the same weights split once (static weights held as hi / lo)
             self.Whi = torch.empty(self.W.shape, dtype=torch.int16, device=dev)
             self.Wlo = torch.empty(self.W.shape, dtype=torch.int16, device=dev)
@@ -191,7 +195,7 @@ class Workload:
         out = []
         only = self.only
         if only in (None, "prefill"):
-            out.append(("prefill", lambda: h.heal_gemm_compensated(self.X, self.W, self.C)))
+            out.append(("prefill", lambda: self.prefill()))
         if only in (None, "decode"):
             for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
                 out.append((f"decode{m}", lambda Xd=Xd, Wd=Wd, Cd=Cd, ws=ws: h.heal_gemm_compensated(
@@ -214,6 +218,9 @@ class Workload:
                 self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len, KV["D"] ** -0.5, self.out,
                 self.aws)))
         return out
+
+    def prefill(self):
+        self.heal.heal_gemm_compensated(self.X, self.W, self.C, workspace=self.wsp, b_split_pass=True)
 
     def run_chain(self, presplit):
         a = self.chain_x
@@ -260,7 +267,7 @@ class Workload:
         only = self.only
         if only in (None, "prefill"):
             rec("prefill", 0)
-            h.heal_gemm_compensated(self.X, self.W, self.C)
+            self.prefill()
             rec("prefill", 1)
         if only in (None, "decode"):
             for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
@@ -294,7 +301,7 @@ class Workload:
                                    KV["D"] ** -0.5, self.out, self.aws)
             rec("attention", 1)
 
-    LAUNCHES_PER_STEP = 1 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
+    LAUNCHES_PER_STEP = 2 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
 
 
 class TorchDecoder:
@@ -756,30 +763,39 @@ def main():
 
     # the prefill product with W split once into hi/lo beforehand (static weights), timed in
     # its own loop after the step so that it does not change the step's power and clocks
-    presplit = None
+    presplit = inkernel = None
     if args.only is None and hasattr(wl, "Whi"):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=cap_stream):
-            heal.heal_gemm_compensated(wl.X, wl.Whi, wl.C, b_lo=wl.Wlo)
-        for _ in range(3):
-            g.replay()
-        reps = max(10, min(K, 50))
-        p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        torch.cuda.synchronize()
-        p0.record(stream)
-        for _ in range(reps):
-            g.replay()
-        p1.record(stream)
-        torch.cuda.synchronize()
-        t_pre = p0.elapsed_time(p1) / 1e3 / reps
-        if ws > 1:
-            t_pre = max_over_ranks([t_pre], device=dev)[0]
+        def time_call(fn):
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cap_stream):
+                fn()
+            for _ in range(3):
+                g.replay()
+            reps = max(10, min(K, 50))
+            p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            torch.cuda.synchronize()
+            p0.record(stream)
+            for _ in range(reps):
+                g.replay()
+            p1.record(stream)
+            torch.cuda.synchronize()
+            t = p0.elapsed_time(p1) / 1e3 / reps
+            if ws > 1:
+                t = max_over_ranks([t], device=dev)[0]
+            del g
+            return t, reps
+        t_pre, reps = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.Whi, wl.C, b_lo=wl.Wlo))
         presplit = {"tflops_effective": ws * u["prefill_flop_eff"] / t_pre / 1e12,
                     "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_pre / 1e12 / peak_sus,
                     "ms": 1e3 * t_pre, "replays": reps,
                     "note": "the same product with W split once into hi/lo beforehand (static weights); "
                             "timed separately after the step"}
-        del g
+        t_ik, reps = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.W, wl.C))
+        inkernel = {"tflops_effective": ws * u["prefill_flop_eff"] / t_ik / 1e12,
+                    "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_ik / 1e12 / peak_sus,
+                    "ms": 1e3 * t_ik, "replays": reps,
+                    "note": "the same product with both operands split inside every tile (no split pass, "
+                            "no workspace); timed separately after the step"}
 
     attn_prefill = None
     if args.only is None:
@@ -806,14 +822,14 @@ def main():
         reps = max(2, min(args.steps, 5))
         for _ in range(2):
             dX.copy_(hX, non_blocking=True); dW.copy_(hW, non_blocking=True)
-            heal.heal_gemm_compensated(dX, dW, dC)
+            heal.heal_gemm_compensated(dX, dW, dC, workspace=wl.wsp, b_split_pass=True)
             hC.copy_(dC, non_blocking=True)
         torch.cuda.synchronize()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
         for _ in range(reps):
             dX.copy_(hX, non_blocking=True); dW.copy_(hW, non_blocking=True)
-            heal.heal_gemm_compensated(dX, dW, dC)
+            heal.heal_gemm_compensated(dX, dW, dC, workspace=wl.wsp, b_split_pass=True)
             hC.copy_(dC, non_blocking=True)
         e1.record(stream)
         torch.cuda.synchronize()
@@ -856,10 +872,13 @@ def main():
             "config": arm_config(ws),
             "pct_of_16bit_peak": 100.0 * mma_tflops / peak_sus,
             "prefill_presplit_weights": presplit,
+            "prefill_inkernel_split": inkernel,
             "attention_prefill": attn_prefill,
             "roofline": {"bound": "tensor", "achieved": mma_tflops, "peak": peak_sus, "unit": "TFLOP/s",
                          "frac": mma_tflops / peak_sus, "traffic": traffic,
-                         "kernel": "heal_gemm_pair_kernel (prefill, 256x256 CTA pair)", "peak_source": f"bf16_tflops_sustained, {peak_src}",
+                         "kernel": "heal_split_kernel (B split pass) + heal_gemm_pair_kernel (256x256 CTA pair) per "
+                                   "call; achieved counts the 3 MMAs over the time of both launches",
+                         "peak_source": f"bf16_tflops_sustained, {peak_src}",
                          "frac_of_burst_peak": mma_tflops / peak_burst},
             "attn_gbs": attn_gbs, "attn_frac_hbm": attn_gbs / hbm,
             "secondary": {"kv_writer_gbs": kvw_gbs, "kv_writer_frac_hbm": kvw_gbs / hbm, "decode_gemm": dec,

@@ -30,7 +30,7 @@ class GemmOpts(ctypes.Structure):
     _fields_ = [("tile_config", ctypes.c_int), ("chan_exp", ctypes.c_void_p), ("b_layout", ctypes.c_int),
                 ("b_presplit", ctypes.c_int), ("b_lo", ctypes.c_void_p), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_size_t), ("b_static", ctypes.c_int),
-                ("reserved", ctypes.c_int * 3)]
+                ("b_split_pass", ctypes.c_int), ("reserved", ctypes.c_int * 2)]
 
 
 _lib = None
@@ -116,7 +116,7 @@ def heal_split(x, hi, lo, fmt=SPLIT_FP16_S11, stream=None):
 
 
 def gemm_opts(tile_config=TILE_AUTO, chan_exp=None, b_layout=0, b_lo=None, workspace=None, b_static=False,
-              b_16bit=False):
+              b_16bit=False, b_split_pass=False):
     o = GemmOpts()
     o.tile_config = int(tile_config)
     o.chan_exp = None if chan_exp is None else chan_exp.data_ptr()
@@ -128,19 +128,22 @@ def gemm_opts(tile_config=TILE_AUTO, chan_exp=None, b_layout=0, b_lo=None, works
     o.workspace = None if workspace is None else workspace.data_ptr()
     o.workspace_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
     o.b_static = 1 if b_static else 0
+    o.b_split_pass = 1 if b_split_pass else 0
     return o
 
 
-def heal_gemm_workspace_bytes(M, N, K, tile_config=TILE_AUTO):
-    o = gemm_opts(tile_config)
+def heal_gemm_workspace_bytes(M, N, K, tile_config=TILE_AUTO, b_split_pass=False):
+    o = gemm_opts(tile_config, b_split_pass=b_split_pass)
     return int(lib().heal_gemm_workspace_bytes(int(M), int(N), int(K), ctypes.byref(o)))
 
 
 def heal_gemm_compensated(A, B, C, fmt=SPLIT_FP16_S11, tile_config=TILE_AUTO, chan_exp=None, b_layout=0,
-                          b_lo=None, workspace=None, b_static=False, b_16bit=False, stream=None):
+                          b_lo=None, workspace=None, b_static=False, b_16bit=False, b_split_pass=False,
+                          stream=None):
     """C[M,N] = A[M,K] . B with B [K,N] (b_layout 0) or [N,K] (b_layout 1); B may be the
     16-bit hi part with b_lo the lo part (pre-split weights), or a 16-bit matrix with
-    b_16bit=True (two products: only A is split)."""
+    b_16bit=True (two products: only A is split).  b_split_pass=True splits an FP32 B
+    into the workspace with one pass before the product (same bits)."""
     _cuda(A, B, C, chan_exp, b_lo, workspace)
     if A.dim() != 2 or B.dim() != 2 or C.dim() != 2 or A.stride(1) != 1 or B.stride(1) != 1 or C.stride(1) != 1:
         raise ValueError("heal_gemm_compensated takes 2-D row-major tensors")
@@ -148,7 +151,7 @@ def heal_gemm_compensated(A, B, C, fmt=SPLIT_FP16_S11, tile_config=TILE_AUTO, ch
     N = C.shape[1]
     if C.shape[0] != M or (B.shape != ((K, N) if b_layout == 0 else (N, K))):
         raise ValueError("shape mismatch")
-    o = gemm_opts(tile_config, chan_exp, b_layout, b_lo, workspace, b_static, b_16bit)
+    o = gemm_opts(tile_config, chan_exp, b_layout, b_lo, workspace, b_static, b_16bit, b_split_pass)
     st = lib().heal_gemm_compensated(M, N, K, _ptr(A), A.stride(0), _ptr(B), B.stride(0), _ptr(C), C.stride(0),
                                      int(fmt), ctypes.byref(o), _stream(stream))
     _check(st, "heal_gemm_compensated")

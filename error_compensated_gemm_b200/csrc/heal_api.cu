@@ -94,9 +94,18 @@ heal_status_t heal_split(const float* x, void* hi, void* lo, int64_t n, heal_spl
   return st;
 }
 
+// Split-K scratch of the tile configuration (0 when it uses none), rounded up to 256 bytes.
+static size_t splitk_bytes(int M, int N, int K, int cfg) {
+  const size_t b = cfg == HEAL_TILE_AUTO ? (M <= 64 ? gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK) : 0)
+                                         : gemm_workspace_bytes(M, N, K, cfg);
+  return (b + 255) & ~(size_t)255;
+}
+
 size_t heal_gemm_workspace_bytes(int M, int N, int K, const heal_gemm_opts_t* opts) {
   if (M <= 0 || N <= 0 || K <= 0) return 0;
   const int cfg = opts ? opts->tile_config : HEAL_TILE_AUTO;
+  const size_t b = splitk_bytes(M, N, K, cfg);
+  if (opts && opts->b_split_pass == 1) return b + (size_t)4 * K * N;   // hi and lo parts of B
   if (cfg == HEAL_TILE_AUTO) return M <= 64 ? gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK) : 0;
   return gemm_workspace_bytes(M, N, K, cfg);
 }
@@ -113,6 +122,7 @@ heal_status_t heal_gemm_compensated(int M, int N, int K, const float* A, int64_t
   if (o.b_layout != 0 && o.b_layout != 1) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.b_presplit < 0 || o.b_presplit > 2) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.b_static != 0 && o.b_static != 1) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.b_split_pass != 0 && o.b_split_pass != 1) return HEAL_ERR_INVALID_ARGUMENT;
   for (int r : o.reserved)
     if (r != 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.tile_config < HEAL_TILE_AUTO || o.tile_config > HEAL_TILE_SKINNY_FULLK) return HEAL_ERR_INVALID_ARGUMENT;
@@ -126,6 +136,30 @@ heal_status_t heal_gemm_compensated(int M, int N, int K, const float* A, int64_t
   if (o.b_presplit == 2 && o.b_lo) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.chan_exp && !aligned(o.chan_exp, 1)) return HEAL_ERR_INVALID_ARGUMENT;
   if (o.workspace && !aligned(o.workspace, 16)) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.b_split_pass) {
+    // split B into the workspace (after the split-K part), then the product on its parts
+    if (o.b_presplit != 0 || o.chan_exp != nullptr) return HEAL_ERR_INVALID_ARGUMENT;
+    if (ldb != b_min || ldb % 8 != 0) return HEAL_ERR_UNSUPPORTED;   // 16-byte rows of the 16-bit parts
+    const size_t head = splitk_bytes(M, N, K, o.tile_config);
+    if (!o.workspace || o.workspace_bytes < head + (size_t)4 * K * N) return HEAL_ERR_INVALID_ARGUMENT;
+    uint8_t* w = static_cast<uint8_t*>(o.workspace);
+    void* bhi = w + head;
+    void* blo = w + head + (size_t)2 * K * N;
+    heal_status_t st = split_launch(static_cast<const float*>(B), bhi, blo, (long long)K * N, (int)fmt,
+                                    (cudaStream_t)stream);
+    if (st == HEAL_OK) {
+      heal_gemm_opts_t o2 = o;
+      o2.b_split_pass = 0;
+      o2.b_presplit = 1;
+      o2.b_lo = blo;
+      o2.b_static = 0;                 // B's parts are written by the launch just before
+      o2.workspace_bytes = head;
+      if (head == 0) o2.workspace = nullptr;
+      st = gemm_launch(M, N, K, A, lda, bhi, ldb, C, ldc, (int)fmt, o2, (cudaStream_t)stream);
+    }
+    if (st == HEAL_ERR_CUDA) (void)cudaGetLastError();
+    return st;
+  }
   const heal_status_t st = gemm_launch(M, N, K, A, lda, B, ldb, C, ldc, (int)fmt, o, (cudaStream_t)stream);
   if (st == HEAL_ERR_CUDA) (void)cudaGetLastError();
   return st;

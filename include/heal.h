@@ -96,7 +96,15 @@ typedef struct {
                                touch A, chan_exp, C or the workspace; with b_static they may
                                request the first stages of B before that wait.  0: B is
                                waited for like A.                                           */
-  int reserved[3];          /* must be zero                                                  */
+  int b_split_pass;         /* 1 (b_presplit = 0, chan_exp null, B contiguous: ldb = N or K):
+                               B is split once per call by heal_split's kernel into the
+                               workspace (its hi and lo parts, 4*K*N bytes after the split-K
+                               part) and the product then reads the 16-bit parts, as with
+                               b_presplit = 1.  The same bits as 0; for large B the two
+                               launches are faster than splitting B inside every tile.
+                               heal_gemm_workspace_bytes counts these bytes when the flag
+                               is set.                                                       */
+  int reserved[2];          /* must be zero                                                  */
 } heal_gemm_opts_t;
 
 /* K1. Hi/lo split of n FP32 values (technical summary, section 2.B, "Mechanism").

@@ -32,6 +32,10 @@ def test_workspace_queries_are_host_only():
     # chunk values [64][1][4096] FP32
     assert heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK) == 64 * 4096 * 4
     assert heal.heal_gemm_workspace_bytes(4096, 4096, 4096, heal.TILE_128x128) == 0
+    # a split pass over B adds its hi and lo parts (2 + 2 bytes per element) after the split-K part
+    assert heal.heal_gemm_workspace_bytes(4096, 14336, 4096, b_split_pass=True) == 4 * 4096 * 14336
+    assert heal.heal_gemm_workspace_bytes(1, 4096, 4096, heal.TILE_SKINNY_SPLITK, b_split_pass=True) == \
+        64 * 4096 * 4 + 4 * 4096 * 4096
     assert heal.heal_attention_workspace_bytes(8, 32, 1, 8192) > 0
     assert heal.heal_attention_workspace_bytes(0, 32, 1, 8192) == 0
 
@@ -60,6 +64,15 @@ def test_invalid_arguments_rejected_before_launch():
     assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 8, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
     o.b_lo = None
     assert L.heal_gemm_compensated(4, 4, 4, fake, 4, fake, 4, fake, 4, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT  # ldb % 8
+    o.b_presplit = 0
+    o.b_split_pass = 2                               # only 0 / 1
+    assert L.heal_gemm_compensated(4, 8, 8, fake, 8, fake, 8, fake, 8, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.b_split_pass = 1                               # no workspace for B's parts
+    assert L.heal_gemm_compensated(4, 8, 8, fake, 8, fake, 8, fake, 8, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
+    o.workspace, o.workspace_bytes = 1 << 20, 4 * 8 * 8
+    assert L.heal_gemm_compensated(4, 8, 8, fake, 8, fake, 16, fake, 8, 0, ctypes.byref(o), None) == heal.HEAL_ERR_UNSUPPORTED  # B not contiguous
+    o.b_presplit, o.b_lo = 1, 1 << 20                # a split pass over a pre-split B makes no sense
+    assert L.heal_gemm_compensated(4, 8, 8, fake, 8, fake, 8, fake, 8, 0, ctypes.byref(o), None) == heal.HEAL_ERR_INVALID_ARGUMENT
     with pytest.raises(ValueError):
         heal.gemm_opts(b_lo=object(), b_16bit=True)
     assert L.heal_split(fake, fake, fake, -1, 0, None) == heal.HEAL_ERR_INVALID_ARGUMENT

@@ -304,3 +304,25 @@ def test_graph_replay_with_new_inputs(M):
         torch.cuda.synchronize()
         assert np.array_equal(got.view(np.uint32), to_np(ref).view(np.uint32)), seed
     status_ok()
+
+
+@pytest.mark.parametrize("M,b_layout,fmt", [(520, 0, heal.SPLIT_FP16_S11), (300, 1, heal.SPLIT_FP16_S11),
+                                            (8, 0, heal.SPLIT_FP16_S11), (256, 0, heal.SPLIT_BF16)])
+def test_split_pass_over_b_is_bitwise_identical(M, b_layout, fmt):
+    """b_split_pass: B split once into the workspace by the split kernel, then the product
+    on its 16-bit parts; the same bits as the in-kernel split of both operands."""
+    d = dev()
+    K, N = 328, 648
+    X = synthetic.normal((M, K), seed=31)
+    W = synthetic.with_outliers(synthetic.normal((K, N), seed=32), 0.01, 20.0, seed=33)
+    Bin = W if b_layout == 0 else W.T.contiguous()
+    A_d, B_d = X.to(d).contiguous(), Bin.to(d).contiguous()
+    c_ref = gemm(X.numpy(), Bin.numpy(), fmt=fmt, b_layout=b_layout)
+    ws = torch.empty(heal.heal_gemm_workspace_bytes(M, N, K, b_split_pass=True), dtype=torch.uint8, device=d)
+    C = torch.full((M, N), float("nan"), device=d)
+    heal.heal_gemm_compensated(A_d, B_d, C, fmt=fmt, b_layout=b_layout, workspace=ws, b_split_pass=True)
+    status_ok()
+    assert np.array_equal(C.cpu().numpy(), c_ref)
+    # and against the FP64 product (FP16 split: the 1e-6 bound)
+    if fmt == heal.SPLIT_FP16_S11:
+        assert G.normwise_rel_err(C.cpu().numpy().astype(np.float64), G.gemm_ref(X.numpy(), W.numpy())) <= TOL_FP16
