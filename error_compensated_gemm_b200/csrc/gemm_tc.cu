@@ -160,6 +160,33 @@ __device__ __forceinline__ void load_operand(uint8_t* dst, const CUtensorMap* ma
   }
 }
 
+// The same loads with an L2 evict-first hint: for an operand streamed once (the weights of
+// the split-K decode kernels), so that it does not push the chunk workspace out of L2.
+template <int R, bool MN, int PRE>
+__device__ __forceinline__ void load_operand_once(uint8_t* dst, const CUtensorMap* map, const CUtensorMap* map_lo,
+                                                  uint64_t* bar, int row0, int k0, uint64_t pol) {
+  if constexpr (PRE == 0) {
+    if constexpr (!MN) {
+      tma_load_2d_hint(dst, map, bar, k0, row0, pol);
+      tma_load_2d_hint(dst + R * 128, map, bar, k0 + 32, row0, pol);
+    } else {
+#pragma unroll
+      for (int b = 0; b < R / 32; ++b) tma_load_2d_hint(dst + b * 8192, map, bar, row0 + 32 * b, k0, pol);
+    }
+  } else {
+    if constexpr (!MN) {
+      tma_load_2d_hint(dst, map, bar, k0, row0, pol);
+      if constexpr (PRE == 1) tma_load_2d_hint(dst + R * 128, map_lo, bar, k0, row0, pol);
+    } else {
+#pragma unroll
+      for (int p = 0; p < R / 64; ++p) {
+        tma_load_2d_hint(dst + (2 * p) * 8192, map, bar, row0 + 64 * p, k0, pol);
+        if constexpr (PRE == 1) tma_load_2d_hint(dst + (2 * p + 1) * 8192, map_lo, bar, row0 + 64 * p, k0, pol);
+      }
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------
 // In-place split of one 2 KB region pair by one warp.
 // src0/src1 each hold one 128-byte-swizzled atom of 8 rows x 32 FP32 values; together
@@ -335,6 +362,12 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
       // still running.  An operand the caller declared static is requested for the first
       // stages right away; everything else waits for the preceding grid to finish.
       int pre = 0;
+      const uint64_t pol = l2_policy_evict_first();
+      // split-K: kernel-A (the weights) is read exactly once
+      auto load_a = [&](uint8_t* st, uint64_t* bar, int tm, int k0) {
+        if (args.splitk) load_operand_once<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, bar, tm * kBM, k0, pol);
+        else load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, bar, tm * kBM, k0);
+      };
       if (args.static_op != 0) {
         for (WorkIter w(args); w.valid() && pre < S; w.advance(), ++pre) {
           int tm, tn;
@@ -342,7 +375,7 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
           const int k0 = w.chunk * kBK;
           uint8_t* st = stages + pre * C::kStageBytes;
           mbar_arrive_expect_tx(&full[pre], kStageTx);
-          if (args.static_op == 1) load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, &full[pre], tm * kBM, k0);
+          if (args.static_op == 1) load_a(st, &full[pre], tm, k0);
           else load_operand<BN, B_MN, B_PRE>(st + C::kABytes, &tmB, &tmB_lo, &full[pre], tn * BN, k0);
         }
       }
@@ -357,7 +390,7 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
         const int k0 = w.chunk * kBK;
         uint8_t* st = stages + s * C::kStageBytes;
         if (it >= pre) mbar_arrive_expect_tx(&full[s], kStageTx);
-        if (it >= pre || args.static_op != 1) load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, &full[s], tm * kBM, k0);
+        if (it >= pre || args.static_op != 1) load_a(st, &full[s], tm, k0);
         if (it >= pre || args.static_op != 2)
           load_operand<BN, B_MN, B_PRE>(st + C::kABytes, &tmB, &tmB_lo, &full[s], tn * BN, k0);
       }
