@@ -21,7 +21,7 @@
 // Work decomposition: a persistent grid (two CTAs per SM); CTA c owns the contiguous
 // slice [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token
 // block) units.  Warp roles: a TMA producer streams 64-token K and V tiles (128-byte
-// swizzle) into a three-stage ring; four QK warps take 16 tokens each (exact S^T on the
+// swizzle) into a two-stage ring; four QK warps take 16 tokens each (exact S^T on the
 // integer tensor cores, logits, the block's softmax step with the row maximum shared by
 // the four warps, P' split into FP16 parts and written in the PV operand layout); four PV
 // warps each own a quarter of the dims of O and add V^T P'^T over the block's 64 tokens.
@@ -43,10 +43,10 @@ namespace {
 
 constexpr int kBlk = 64;          // tokens per pipeline stage
 // Warp roles per CTA: kQK warps for QK^T and the softmax step (16 tokens each), kPV warps
-// for PV (D/4 dims each), one TMA producer.  Three K/V stages per CTA, two CTAs per SM
-// (16 compute warps and six stages per SM).
+// for PV (D/4 dims each), one TMA producer.  Two K/V stages per CTA, two CTAs per SM
+// (16 compute warps and four stages per SM).
 constexpr int kQK = 4, kPV = 4;
-constexpr int kStages = 3;
+constexpr int kStages = 2;
 constexpr int kMinBlocks = 2;
 constexpr int kAttnThreads = (kQK + kPV + 1) * 32;
 constexpr int kRows = 8;          // query rows per CTA: (Hq/Hkv) * Tq <= 8
