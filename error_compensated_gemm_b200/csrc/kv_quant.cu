@@ -2,8 +2,10 @@
 // written straight into the [B, H, Tmax, D] cache (gist.science technical summary,
 // section 2.A: Q/K/V stored as INT16 at a 16-bit footprint).
 //
-// A warp takes one token (b, t) at a time and its H head rows in passes of 32/L rows,
-// one group of L = D/8 lanes per row; each lane owns 8 consecutive values: one 16-byte
+// A warp takes one unit at a time: a token (b, t) and a group of up to 4 * 32/L of its H
+// head rows (all of them when H is small; several units per token when H is large, so that
+// a step with few tokens, such as one decode query, still spreads over many warps), in
+// passes of 32/L rows, one group of L = D/8 lanes per row; each lane owns 8 consecutive values: one 16-byte
 // (bf16) or two 16-byte (fp32) streaming loads and one 16-byte int16 store.  The row
 // absmax is a shuffle reduction inside the group.  Every decision is taken in FP32:
 //   inv = 32767 / absmax (IEEE division), q = rint(x * inv) clamped to +-32767,
@@ -35,11 +37,16 @@ __global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restri
   const int warps_total = gridDim.x * (blockDim.x >> 5);
   const int warp_id = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
 
-  // one warp per token (b, t) at a time; its H head rows in passes of kRowsPerPass
-  for (int bt = warp_id; bt < tokens; bt += warps_total) {
+  // one warp per (token, head group) unit; the group's rows in kUnroll passes of kRowsPerPass
+  constexpr int kGroupRows = kRowsPerPass * kUnroll;
+  const int hgroups = (H + kGroupRows - 1) / kGroupRows;
+  const long long units = (long long)tokens * hgroups;
+  for (long long un = warp_id; un < units; un += warps_total) {
+    const int bt = (int)(un / hgroups), hg = (int)(un - (long long)bt * hgroups);
     const int b = bt / T, t = bt - b * T;
     const char* xrow = static_cast<const char*>(x) + (size_t)(b * sb + (long long)t * st) * (BF16 ? 2 : 4);
-    for (int h0 = 0; h0 < H; h0 += kRowsPerPass * kUnroll) {
+    {
+      const int h0 = hg * kGroupRows;
       // all loads of the pass group first, kept as raw words (4 registers per 16 bytes)
       uint4 raw[kUnroll][BF16 ? 1 : 2];
 #pragma unroll
@@ -128,7 +135,9 @@ heal_status_t kv_quant_launch(const void* x, int is_bf16, int B, int T, int H, i
   if (sms <= 0) return HEAL_ERR_CUDA;
   const int L = D / 8;
   const long long tokens = (long long)B * T;
-  long long grid = (tokens + 7) / 8;                     // 8 warps per block, one token each
+  const long long group_rows = 128 / L;                  // head rows per warp unit (4 passes of 32/L)
+  const long long units = tokens * ((H + group_rows - 1) / group_rows);
+  long long grid = (units + 7) / 8;                      // 8 warps per block, one unit each
   if (grid > (long long)sms * 8) grid = (long long)sms * 8;
   cudaError_t e;
   switch (L) {
