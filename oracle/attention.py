@@ -18,6 +18,8 @@ Attention definition (no chunking, no online softmax, no FP32):
   visible t : t < kv_len[b] and (not causal or t <= pos_i)
   logit_t   = S_int(q_i, k_t) * s_q * s_k[t] * softmax_scale      (float64)
   O_i       = sum_t softmax(logit)_t * s_v[t] * v_t               (float64)
+  a query with no visible token (causal, position < 0, i.e. kv_len < Tq) has O_i = 0
+  (the library's definition for that case; the pages do not reach it)
 
 Parity: pinned (exhaustive byte-split reconstruction, int64 dots against Python
 integers including extreme vectors, uniform-softmax and one-hot special cases,
@@ -63,11 +65,14 @@ def attention(q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len, softmax_sc
                 pos = L - Tq + np.arange(Tq)
                 mask = np.arange(L)[None, :] <= pos[:, None]
                 logits = np.where(mask, logits, -np.inf)
-            m = np.max(logits, axis=1, keepdims=True)
-            p = np.exp(logits - m)
-            p /= np.sum(p, axis=1, keepdims=True)
+            seen = np.isfinite(logits).any(axis=1) if L > 0 else np.zeros(Tq, bool)
             v = v_cache[b, hkv, :L].astype(np.float64) * v_scale[b, hkv, :L].astype(np.float64)[:, None]
-            out[b, hq] = p @ v
+            if seen.any():
+                lg = logits[seen]
+                m = np.max(lg, axis=1, keepdims=True)
+                p = np.exp(lg - m)
+                p /= np.sum(p, axis=1, keepdims=True)
+                out[b, hq][seen] = p @ v
         s_blocks.append(s_b)
     return (out, s_blocks) if return_s_int else out
 

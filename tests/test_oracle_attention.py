@@ -123,3 +123,16 @@ def test_causal_first_query_sees_only_first_token():
     deq = Q.dequantize(v, vs)
     for hq in range(4):
         np.testing.assert_allclose(out[0, hq, 0], deq[0, hq // 2, 0], rtol=1e-15)
+
+
+def test_queries_before_the_first_token_give_zero_rows():
+    # causal, kv_len 3 < Tq 6: queries 0..2 sit at positions -3..-1 and see nothing (O = 0);
+    # queries 3..5 are the queries at positions 0..2 of a 3-token context
+    q, qs, k, ks, v, vs = _tiny_case(7, Tq=6, Tmax=6)
+    out = A.attention(q, qs, k, ks, v, vs, np.array([3]), 0.2, causal=True)
+    assert np.all(out[:, :, :3] == 0.0)
+    ref = A.attention(q[:, :, 3:], qs[:, :, 3:], k, ks, v, vs, np.array([3]), 0.2, causal=True)
+    np.testing.assert_array_equal(out[:, :, 3:], ref)
+    deq = Q.dequantize(v, vs)
+    for hq in range(4):   # the first of them sees only token 0
+        np.testing.assert_allclose(out[0, hq, 3], deq[0, hq // 2, 0], rtol=1e-15)
