@@ -57,3 +57,13 @@ def test_noalloc_rejects_problems_beyond_the_fixed_scratch():
                                           i16(B, Hkv, Tmax, D), f32(B, Hkv, Tmax),
                                           torch.ones(B, dtype=torch.int32, device=d), 0.1, f32(B, Hq, 1, D))
     assert e.value.status == heal.HEAL_ERR_UNSUPPORTED
+
+
+def test_noalloc_prefill_shape_matches_workspace_entry_point():
+    # 4 query heads per KV head x 96 queries: the tcgen05 prefill kernel, whose byte planes
+    # fit the fixed scratch at this size; the two entry points give the same bits
+    d = dev()
+    inputs = make_inputs(B=1, Hq=8, Hkv=2, D=128, T=192, Tq=96, seed=11)
+    want = _run("workspace", inputs, [192], d)
+    got = _run("noalloc", inputs, [192], d)
+    assert np.array_equal(got, want)
