@@ -157,3 +157,15 @@ def test_prefill_head_dim_64_is_unsupported():
                                   i16(B, Hkv, Tmax, D), f32(B, Hkv, Tmax),
                                   torch.full((B,), Tmax, dtype=torch.int32, device=d), 64 ** -0.5,
                                   torch.empty(B, Hq, Tq, D, device=d), ws)
+
+
+def test_prefill_tiles_with_no_visible_token():
+    # causal, kv_len 100 < Tq 300: the first 128-row tile sees no token at all (its CTA
+    # loads nothing and writes zeros); rows 0..199 are zero, rows 200..299 are the queries
+    # at positions 0..99
+    q, qs, kq, kss, vq, vss = make_inputs(B=1, Hq=4, Hkv=2, D=128, T=300, Tq=300, Tmax=320, seed=9)
+    out, _ = run_gpu(q, qs, kq, kss, vq, vss, [100], SCALE, causal=True)
+    ref = OA.attention(q, qs, kq, kss, vq, vss, [100], SCALE, causal=True)
+    assert np.all(out[:, :, :200] == 0.0)
+    err = np.linalg.norm(out - ref) / np.linalg.norm(ref)
+    assert err <= tolerance(q[:, :, 200:], qs[:, :, 200:], kq, kss, [100], SCALE, 2), err
