@@ -38,6 +38,16 @@ def test_workspace_queries_are_host_only():
         64 * 4096 * 4 + 4 * 4096 * 4096
     assert heal.heal_attention_workspace_bytes(8, 32, 1, 8192) > 0
     assert heal.heal_attention_workspace_bytes(0, 32, 1, 8192) == 0
+    # decode shapes ((Hq/Hkv)*Tq <= 8) need the split-context partials only; prefill shapes
+    # the byte planes: 6 B per cache element + 2 B per query element + s_v*2^E + E
+    dec = heal.heal_attention_workspace_bytes_gqa(8, 32, 8, 2, 8192)
+    assert 0 < dec <= heal.heal_attention_workspace_bytes(8, 32, 2, 8192)
+    assert heal.heal_attention_workspace_bytes_gqa(1, 32, 8, 512, 640) == \
+        6 * 8 * 640 * 128 + 2 * 32 * 512 * 128 + 4 * 8 * 640 + 128
+    # the short form is an upper bound for every Hkv dividing Hq
+    for hkv in (1, 2, 4, 8, 16, 32):
+        assert heal.heal_attention_workspace_bytes_gqa(2, 32, hkv, 96, 192) <= heal.heal_attention_workspace_bytes(2, 32, 96, 192)
+    assert heal.heal_attention_workspace_bytes_gqa(1, 30, 8, 4, 64) == 0   # Hq % Hkv != 0
 
 
 def test_invalid_arguments_rejected_before_launch():
