@@ -26,12 +26,29 @@ def rope_tables(max_pos, head_dim, theta):
     return torch.cos(ang).float(), torch.sin(ang).float()
 
 
+_LINEARS = ("wqkv", "wo", "wgu", "wdown")
+
+
 class Decoder:
-    def __init__(self, cfg, weights, device, max_len=None):
+    def __init__(self, cfg, weights, device, max_len=None, presplit_weights=True):
+        """presplit_weights: split every linear weight once into its 16-bit hi and lo parts
+        (heal_split, the same encodings the GEMM kernels produce) and keep only those; the
+        GEMMs then split only the activations.  The results are the same bits either way."""
         self.cfg = c = cfg
         self.dev = device
         self.max_len = max_len or c.max_pos
         self.w = {k: v.to(device).contiguous() for k, v in weights.items()}
+        self.parts = {}
+        if presplit_weights:
+            names = [f"{n}{l}" for l in range(c.layers) for n in _LINEARS] + ["lm_head"]
+            for k in names:
+                w = self.w[k]
+                hi = torch.empty(w.shape, dtype=torch.int16, device=device)
+                lo = torch.empty(w.shape, dtype=torch.int16, device=device)
+                H.heal_split(w, hi, lo)
+                self.parts[k] = (hi, lo)
+                self.w[k] = None             # the FP32 copy is not needed any more
+            torch.cuda.synchronize(device)
         cos, sin = rope_tables(self.max_len, c.head_dim, c.rope_theta)
         self.cos, self.sin = cos.to(device), sin.to(device)
         f32, i16 = torch.float32, torch.int16
@@ -53,8 +70,12 @@ class Decoder:
         self.rms_w = None
 
     # ---- building blocks (each one library call) ----
-    def _linear(self, x, w, out):
-        H.heal_gemm_compensated(x, w, out, workspace=self.gemm_ws)
+    def _linear(self, x, key, out):
+        if key in self.parts:
+            hi, lo = self.parts[key]
+            H.heal_gemm_compensated(x, hi, out, b_lo=lo, workspace=self.gemm_ws, b_static=True)
+        else:
+            H.heal_gemm_compensated(x, self.w[key], out, workspace=self.gemm_ws)
 
     def _layer(self, l, h, n, p0):
         c = self.cfg
@@ -62,7 +83,7 @@ class Decoder:
         x = torch.empty_like(h)
         H.heal_rmsnorm(h, self.rms_w, x, c.eps)
         qkv = torch.empty(n, c.qkv_dim, device=d)
-        self._linear(x, self.w[f"wqkv{l}"], qkv)
+        self._linear(x, f"wqkv{l}", qkv)
         pos = self.positions[p0:p0 + n]
         qd = c.heads * c.head_dim
         H.heal_rope(qkv, c.heads, c.head_dim, pos, self.cos, self.sin)                 # q heads
@@ -106,15 +127,15 @@ class Decoder:
             attn = torch.empty(n, c.heads * D, device=d)
             H.heal_heads_to_rows(attn_h, attn.view(1, n, c.heads, D))
         o = torch.empty(n, c.hidden, device=d)
-        self._linear(attn, self.w[f"wo{l}"], o)
+        self._linear(attn, f"wo{l}", o)
         H.heal_add(h, o)
         H.heal_rmsnorm(h, self.rms_w, x, c.eps)
         gu = torch.empty(n, 2 * c.ffn, device=d)
-        self._linear(x, self.w[f"wgu{l}"], gu)
+        self._linear(x, f"wgu{l}", gu)
         act = torch.empty(n, c.ffn, device=d)
         H.heal_swiglu(gu, act)
         dn = torch.empty(n, c.hidden, device=d)
-        self._linear(act, self.w[f"wdown{l}"], dn)
+        self._linear(act, f"wdown{l}", dn)
         H.heal_add(h, dn)
 
     def forward(self, ids):
@@ -133,7 +154,7 @@ class Decoder:
         H.heal_rmsnorm(h[n - 1:n], self.rms_w, x, c.eps)
         self.last_hidden = x                     # final normed hidden state of the last position
         logits = torch.empty(1, c.vocab, device=self.dev)
-        self._linear(x, self.w["lm_head"], logits)
+        self._linear(x, "lm_head", logits)
         return logits
 
     def generate(self, prompt, steps):
