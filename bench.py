@@ -491,8 +491,9 @@ def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=1
             "prompt": prompt_len, "steps": steps, "bitwise_repeat": bool(torch.equal(tok, t_again)),
             "graph_tokens_equal_eager": same,
             "note": "decode_ms_per_token: each step launched from Python; decode_graph_ms_per_token: the "
-                    "same steps replayed as one CUDA graph; both stream ~3.85 GB of FP32 weights per token "
-                    "(2 layers + the 128256-row LM head)"}
+                    "same steps replayed as one CUDA graph; both stream ~3.85 GB of weights per token "
+                    "(2 layers + the 128256-row LM head), held as 16-bit hi + lo parts split once at load; "
+                    "the GEMMs split only the activations"}
 
 
 # causal INT16 self-attention over a long prompt (the prefill kernel: 128-row query tiles on
