@@ -76,24 +76,3 @@ def attention(q, q_scale, k_cache, k_scale, v_cache, v_scale, kv_len, softmax_sc
         s_blocks.append(s_b)
     return (out, s_blocks) if return_s_int else out
 
-
-def attention_float(q, k, v, kv_len, softmax_scale, Hkv, causal=False):
-    """Same definition on unquantized float inputs q [B,Hq,Tq,D], k/v [B,Hkv,Tmax,D]
-    (used to report the quantization effect, not for parity)."""
-    q = np.asarray(q, np.float64)
-    B, Hq, Tq, D = q.shape
-    G = Hq // Hkv
-    out = np.zeros((B, Hq, Tq, D), np.float64)
-    for b in range(B):
-        L = int(kv_len[b])
-        for hq in range(Hq):
-            hkv = hq // G
-            logits = q[b, hq] @ np.asarray(k[b, hkv, :L], np.float64).T * softmax_scale
-            if causal:
-                pos = L - Tq + np.arange(Tq)
-                logits = np.where(np.arange(L)[None, :] <= pos[:, None], logits, -np.inf)
-            m = np.max(logits, axis=1, keepdims=True)
-            p = np.exp(logits - m)
-            p /= np.sum(p, axis=1, keepdims=True)
-            out[b, hq] = p @ np.asarray(v[b, hkv, :L], np.float64)
-    return out

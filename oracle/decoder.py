@@ -14,8 +14,10 @@ Everything else is float64.  Teacher forcing: logits are evaluated on a given to
 sequence (the device's), at chosen positions.
 
 Parity: pinned (closed forms for RMSNorm, RoPE, SwiGLU, argmax; a stack with zeroed
-layers reduces to the final norm and LM head).  The full stack's agreement with the device
-is a tolerance check, not a pin.
+layers reduces to the final norm and LM head; the block body on hand-built scatter weights,
+written out element by element: one token at position 0, two layers in order, and two
+tokens whose RoPE turn, INT16 rounding after RoPE and causal mask are each visible in the
+logits).  The full stack's agreement with the device is a tolerance check, not a pin.
 """
 import math
 

@@ -167,3 +167,28 @@ def test_two_product_error_levels():
     assert 1e-7 < eb < 2e-5
     e_w = G.normwise_rel_err(G.gemm_two_product(X, W16, S.FP16_S11), G.gemm_ref(X, W))
     assert 1e-5 < e_w < 1e-3
+
+
+def test_bf16_downcast_exact_dyadic_cases():
+    """Hand-worked values of the boundary-truncation control (technical summary, section 1:
+    FP32 accumulators written to BF16 memory).  BF16 keeps 7 stored mantissa bits: the
+    spacing is 2^-7 in [1, 2) and 2^-6 in [2, 4)."""
+    d = 2.0 ** -10
+    # (a) the inputs are rounded first: 1 + 3*2^-10 lies below the half-way point 1 + 2^-8,
+    #     so each rounds to 1 and C = 3; the unrounded sum 3 + 9*2^-10 would have rounded up
+    #     to 3 + 2^-6 on the BF16 store
+    A = np.array([[1 + 3 * d, 1 + 3 * d, 1 + 3 * d]], np.float32)
+    B = np.ones((3, 1), np.float32)
+    assert G.gemm_bf16_downcast(A, B)[0, 0] == 3.0
+    # (b) the result is rounded on the store, ties to even: 1 + 1.5*2^-7 sits half-way
+    #     between 1 + 2^-7 (odd last bit) and 1 + 2^-6 (even), so it stores as 1 + 2^-6
+    A = np.ones((1, 3), np.float32)
+    B = np.array([[1.0], [2.0 ** -7], [2.0 ** -8]], np.float32)
+    assert G.gemm_bf16_downcast(A, B)[0, 0] == 1.0 + 2.0 ** -6
+    #     and 1 + 2^-8, half-way between 1 (even) and 1 + 2^-7, stores as 1
+    B = np.array([[1.0], [2.0 ** -9], [2.0 ** -9]], np.float32)
+    assert G.gemm_bf16_downcast(A, B)[0, 0] == 1.0
+    # (c) orientation: BF16-exact small integers with exact sums give C = A @ B, written out
+    A = np.array([[1, 2, 0], [-3, 1, 4]], np.float32)
+    B = np.array([[2, -1], [0, 5], [1, 3]], np.float32)
+    np.testing.assert_array_equal(G.gemm_bf16_downcast(A, B), [[2.0, 9.0], [-2.0, 20.0]])

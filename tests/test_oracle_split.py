@@ -99,3 +99,17 @@ def test_split_is_elementwise_and_deterministic():
     b = S.split(x[::-1].copy(), S.FP16_S11)
     np.testing.assert_array_equal(a[2], b[2][::-1])
     np.testing.assert_array_equal(a[3], b[3][::-1])
+
+
+def test_format_helpers_on_hand_worked_values():
+    """FP16 / BF16 roundings and encodings that the split builds on, written out by hand."""
+    # FP16 spacing in [1, 2) is 2^-10; half-way points go to the even neighbour
+    x = np.array([1 + 2.0 ** -11, 1 + 3 * 2.0 ** -11, 65504.0, 65520.0, 2.0 ** -24, 2.0 ** -25], np.float64)
+    h = S.to_fp16(x)
+    assert h.dtype == np.float16
+    np.testing.assert_array_equal(h.astype(np.float64), [1.0, 1 + 2.0 ** -9, 65504.0, np.inf, 2.0 ** -24, 0.0])
+    np.testing.assert_array_equal(h.view(np.uint16), [0x3C00, 0x3C02, 0x7BFF, 0x7C00, 0x0001, 0x0000])
+    # BF16: 1 + 2^-8 is half-way between 1 and 1 + 2^-7 (odd) -> 1; 1 + 3*2^-8 -> 1 + 2^-6
+    b = S.to_bf16_as_f32(np.array([1 + 2.0 ** -8, 1 + 3 * 2.0 ** -8, -2.5], np.float32))
+    np.testing.assert_array_equal(b, [1.0, 1 + 2.0 ** -6, -2.5])
+    np.testing.assert_array_equal(S.bf16_bits(b), [0x3F80, 0x3F82, 0xC020])
