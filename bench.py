@@ -306,135 +306,6 @@ class Workload:
     LAUNCHES_PER_STEP = 1 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
 
 
-class TorchDecoder:
-    """The same random-init decoder block in plain torch ops at one precision: a comparison
-    pipeline for the reproducibility study, not the library.  Every op reads and writes
-    `dtype` tensors (for bf16 this is the plain 16-bit stack whose results are stored in 16
-    bits at every kernel boundary); K and V are cached in `dtype`; attention is torch's
-    scaled_dot_product_attention."""
-
-    def __init__(self, torch, cfg, w, dtype, dev, max_len):
-        self.t, self.cfg, self.dtype, self.dev = torch, cfg, dtype, dev
-        self.w = {k: v.to(dev, dtype) for k, v in w.items()}
-        half = cfg.head_dim // 2
-        inv = torch.tensor([cfg.rope_theta ** (-2.0 * i / cfg.head_dim) for i in range(half)], dtype=torch.float64)
-        ang = torch.arange(max_len, dtype=torch.float64)[:, None] * inv[None, :]
-        self.cos, self.sin = torch.cos(ang).to(dev, dtype), torch.sin(ang).to(dev, dtype)
-        self.k = [torch.zeros(max_len, cfg.kv_heads, cfg.head_dim, dtype=dtype, device=dev) for _ in range(cfg.layers)]
-        self.v = [torch.zeros(max_len, cfg.kv_heads, cfg.head_dim, dtype=dtype, device=dev) for _ in range(cfg.layers)]
-        self.pos = 0
-
-    def _rms(self, x):
-        t = self.t
-        return x * t.rsqrt((x * x).mean(-1, keepdim=True) + self.cfg.eps)
-
-    def _rope(self, x, p0):
-        n, half = x.shape[0], self.cfg.head_dim // 2
-        c, s = self.cos[p0:p0 + n, None, :], self.sin[p0:p0 + n, None, :]
-        a, b = x[..., :half], x[..., half:]
-        return self.t.cat([a * c - b * s, b * c + a * s], dim=-1)
-
-    def forward(self, ids):
-        t, c = self.t, self.cfg
-        F = t.nn.functional
-        n, p0 = ids.numel(), self.pos
-        h = self.w["embed"][ids.long()]
-        qd, kd = c.heads * c.head_dim, c.kv_heads * c.head_dim
-        G = c.heads // c.kv_heads
-        for l in range(c.layers):
-            x = self._rms(h)
-            qkv = x @ self.w[f"wqkv{l}"]
-            q = self._rope(qkv[:, :qd].view(n, c.heads, c.head_dim), p0)
-            k = self._rope(qkv[:, qd:qd + kd].view(n, c.kv_heads, c.head_dim), p0)
-            self.k[l][p0:p0 + n] = k
-            self.v[l][p0:p0 + n] = qkv[:, qd + kd:].view(n, c.kv_heads, c.head_dim)
-            K = self.k[l][:p0 + n].repeat_interleave(G, dim=1).transpose(0, 1)   # [heads, T, D]
-            V = self.v[l][:p0 + n].repeat_interleave(G, dim=1).transpose(0, 1)
-            o = F.scaled_dot_product_attention(q.transpose(0, 1), K, V, is_causal=(n > 1 and p0 == 0),
-                                               scale=c.head_dim ** -0.5)
-            h = h + o.transpose(0, 1).reshape(n, qd) @ self.w[f"wo{l}"]
-            x = self._rms(h)
-            gu = x @ self.w[f"wgu{l}"]
-            h = h + (F.silu(gu[:, :c.ffn]) * gu[:, c.ffn:]) @ self.w[f"wdown{l}"]
-        self.pos = p0 + n
-        self.last_hidden = self._rms(h[n - 1:n])
-        return self.last_hidden @ self.w["lm_head"]
-
-
-def reproducibility_study(torch, heal, synthetic, dev, prompt_len=512, steps=128):
-    """Reproducibility analogue on the random-init 2-layer stack: the FP64 pipeline decodes
-    greedily; the FP32, plain-BF16 and HEAL pipelines are teacher-forced on its tokens, and
-    each step's logits and final hidden state are compared with FP64 (flips = steps whose
-    argmax differs).  Each pipeline's own greedy decode is timed per output token."""
-    from error_compensated_gemm_b200.decoder import Decoder
-    torch.backends.cuda.matmul.allow_tf32 = False
-    torch.backends.cudnn.allow_tf32 = False
-    cfg = synthetic.DecoderConfig(max_pos=prompt_len + steps + 64)
-    w = synthetic.decoder_weights(cfg)
-    prompt = synthetic.prompt_ids(prompt_len, cfg.vocab).to(dev)
-    max_len = prompt_len + steps + 64
-
-    def run(fw, reset, tokens=None):
-        """Prefill, then `steps` decode steps (teacher-forced on `tokens` if given, else greedy).
-        Returns (logits list, hidden list, token list)."""
-        reset()
-        lg = fw(prompt)
-        L, Hs, toks = [], [], []
-        for s in range(steps):
-            L.append(lg.double().flatten())
-            Hs.append(fw.__self__.last_hidden.double().flatten())
-            nxt = int(torch.argmax(lg.float()).item()) if tokens is None else tokens[s]
-            toks.append(nxt)
-            if s + 1 < steps:
-                lg = fw(torch.tensor([nxt], dtype=torch.int32, device=dev))
-        return L, Hs, toks
-
-    ref = TorchDecoder(torch, cfg, w, torch.float64, dev, max_len)
-    L64, H64, T64 = run(ref.forward, lambda: setattr(ref, "pos", 0))
-    del ref
-    torch.cuda.empty_cache()
-    out = {"study": "reproducibility analogue (random-init 2-layer stack, teacher-forced on the FP64 "
-                    "greedy tokens)", "prompt": prompt_len, "steps": steps, "pipelines": {}}
-    pipes = [("fp32", None), ("bf16_downcast", None), ("heal", None)]
-    for name, _ in pipes:
-        if name == "heal":
-            dec = Decoder(cfg, w, dev, max_len=max_len)
-            fw, reset = dec.forward, (lambda d=dec: setattr(d, "pos_len", 0))
-        else:
-            dec = TorchDecoder(torch, cfg, w, torch.float32 if name == "fp32" else torch.bfloat16, dev, max_len)
-            fw, reset = dec.forward, (lambda d=dec: setattr(d, "pos", 0))
-        L, Hs, _ = run(fw, reset, T64)
-        rel = [float(torch.linalg.norm(a - b) / torch.linalg.norm(b)) for a, b in zip(L, L64)]
-        mse = [float(((a - b) ** 2).mean()) for a, b in zip(Hs, H64)]
-        flips = sum(int(torch.argmax(a).item() != torch.argmax(b).item()) for a, b in zip(L, L64))
-        # own greedy decode, timed per output token (eager launches, CUDA events)
-        reset()
-        lg = fw(prompt)
-        torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        own = []
-        e0.record()
-        for s in range(steps):
-            nxt = torch.argmax(lg.float()).to(torch.int32).view(1)
-            own.append(nxt)
-            if s + 1 < steps:
-                lg = fw(nxt)
-        e1.record()
-        torch.cuda.synchronize()
-        own = [int(x.item()) for x in own]
-        first_div = next((i for i, (a, b) in enumerate(zip(own, T64)) if a != b), None)
-        out["pipelines"][name] = {
-            "logits_rel_err_mean": sum(rel) / len(rel), "logits_rel_err_max": max(rel),
-            "final_hidden_mse_mean": sum(mse) / len(mse), "argmax_flips": flips,
-            "first_divergence_free_running": first_div, "tpot_ms": e0.elapsed_time(e1) / steps}
-        del dec
-        torch.cuda.empty_cache()
-    b = out["pipelines"]["bf16_downcast"]["tpot_ms"]
-    for name in out["pipelines"]:
-        out["pipelines"][name]["tpot_vs_bf16"] = out["pipelines"][name]["tpot_ms"] / b
-    return out
-
-
 def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=128):
     """2-layer random-init decoder (hidden 4096, 32q/8kv heads, FFN 14336, vocab 128256):
     time of the 512-token prefill and per greedy decode step, and a bitwise repeat check."""
@@ -647,6 +518,7 @@ def main():
     ap.add_argument("--prompt-len", type=int, default=None,
                     help="prompt length of the prefill attention workload (profiling case)")
     ap.add_argument("--no-decoder", action="store_true", help="skip the 2-layer decoder measurement")
+    ap.add_argument("--no-study", action="store_true", help="skip the reproducibility analogue")
     ap.add_argument("--study", action="store_true",
                     help="reproducibility analogue: FP64 / FP32 / plain BF16 / HEAL pipelines on the decoder")
     args = ap.parse_args()
@@ -667,8 +539,9 @@ def main():
     dev = torch.device("cuda", local)
     heal.lib()
     if args.study:
+        from error_compensated_gemm_b200.study import reproducibility_study
         if rank == 0:
-            print(json.dumps(reproducibility_study(torch, heal, synthetic, dev)), flush=True)
+            print(json.dumps(reproducibility_study(dev)), flush=True)
         return 0
     peaks, peak_src = load_peaks()
     if args.only == "attention_prefill":
@@ -745,6 +618,13 @@ def main():
     mma_tflops = u["prefill_flop_mma"] / prefill_s / 1e12
     peak_sus = peaks.get("bf16_tflops_sustained", FALLBACK_PEAKS["bf16_tflops_sustained"])
     peak_burst = peaks.get("bf16_tflops", FALLBACK_PEAKS["bf16_tflops"])
+    # The tensor denominator follows the clock the timed region ran at: the burst peak (a
+    # short GEMM at full clock) unless the SM clock sampled under load fell well below its
+    # maximum (power capping, as in the sustained measurement), then the sustained one.
+    ck = clk.summary()
+    at_max = bool(ck.get("sm_mhz") and ck.get("sm_max_mhz") and ck["sm_mhz"] >= 0.9 * ck["sm_max_mhz"])
+    peak_tc, peak_tc_name = (peak_burst, "bf16_tflops (burst)") if at_max or not ck.get("sm_mhz") \
+        else (peak_sus, "bf16_tflops_sustained")
     hbm = peaks.get("hbm_gbs", FALLBACK_PEAKS["hbm_gbs"])
     attn_gbs = u["attn_bytes"] / (part_ms["attention"] / 1e3 / K) / 1e9
     kvw_gbs = u["kv_writer_bytes"] / (part_ms["kv_writer"] / 1e3 / K) / 1e9
@@ -789,7 +669,7 @@ def main():
             return t, reps
         t_pre, reps = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.Whi, wl.C, b_lo=wl.Wlo))
         presplit = {"tflops_effective": ws * u["prefill_flop_eff"] / t_pre / 1e12,
-                    "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_pre / 1e12 / peak_sus,
+                    "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_pre / 1e12 / peak_tc,
                     "ms": 1e3 * t_pre, "replays": reps,
                     "note": "the same product with W split once into hi/lo beforehand (static weights); "
                             "timed separately after the step"}
@@ -797,12 +677,12 @@ def main():
                                                                    b_split_pass=True))
         t_16, reps16 = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.W16, wl.C, b_16bit=True))
         w16 = {"tflops_effective": ws * u["prefill_flop_eff"] / t_16 / 1e12,
-               "pct_of_16bit_peak": 100.0 * (2.0 / 3.0) * u["prefill_flop_mma"] / t_16 / 1e12 / peak_sus,
+               "pct_of_16bit_peak": 100.0 * (2.0 / 3.0) * u["prefill_flop_mma"] / t_16 / 1e12 / peak_tc,
                "ms": 1e3 * t_16, "replays": reps16,
                "note": "the two-product form with FP16 weights (only X split; 2 MMAs); timed separately "
                        "after the step"}
         splitpass = {"tflops_effective": ws * u["prefill_flop_eff"] / t_sp / 1e12,
-                     "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_sp / 1e12 / peak_sus,
+                     "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_sp / 1e12 / peak_tc,
                      "ms": 1e3 * t_sp, "replays": reps,
                      "note": "the same product with B split by a streaming pass into a workspace first "
                              "(b_split_pass; B's parts go through HBM); timed separately after the step"}
@@ -865,6 +745,15 @@ def main():
             dec_res["prefill_ms"], dec_res["decode_ms_per_token"] = max_over_ranks(
                 [dec_res["prefill_ms"], dec_res["decode_ms_per_token"]], device=dev)
 
+    # the reproducibility analogue and the FP32-pipeline baseline (rank 0, after the timing)
+    study = None
+    if rank == 0 and not args.no_study:
+        try:
+            from error_compensated_gemm_b200.study import reproducibility_study
+            study = reproducibility_study(dev)
+        except Exception as exc:  # report, do not hide
+            study = {"error": repr(exc)}
+
     # DRAM bytes of one prefill launch from the committed ncu summary (a full-size capture)
     traffic = None
     prof = os.path.join(ROOT, "profiles", "heal_gemm_pair_kernel_prefill_traffic.md")
@@ -880,26 +769,29 @@ def main():
             "dtype": "f16x2-from-f32 (FP32 in/out, FP16 hi/lo tensor-core products, FP32 accumulate)",
             "data": "synthetic",
             "config": arm_config(ws),
-            "pct_of_16bit_peak": 100.0 * mma_tflops / peak_sus,
+            "pct_of_16bit_peak": 100.0 * mma_tflops / peak_tc,
             "prefill_presplit_weights": presplit,
             "prefill_split_pass_over_b": splitpass,
             "prefill_fp16_weights_two_products": w16,
             "attention_prefill": attn_prefill,
-            "roofline": {"bound": "tensor", "achieved": mma_tflops, "peak": peak_sus, "unit": "TFLOP/s",
-                         "frac": mma_tflops / peak_sus, "traffic": traffic,
+            "roofline": {"bound": "tensor", "achieved": mma_tflops, "peak": peak_tc, "unit": "TFLOP/s",
+                         "frac": mma_tflops / peak_tc, "traffic": traffic,
                          "kernel": "heal_gemm_pair_kernel<1, 0, 0> (256x256 CTA pair, both operands split by the "
                                    "producer-side split warps)",
-                         "peak_source": f"bf16_tflops_sustained, {peak_src}",
-                         "frac_of_burst_peak": mma_tflops / peak_burst},
+                         "peak_source": f"{peak_tc_name}, {peak_src}; chosen by the SM clock sampled under load "
+                                        f"({ck.get('sm_mhz')} of {ck.get('sm_max_mhz')} MHz)",
+                         "frac_of_burst_peak": mma_tflops / peak_burst,
+                         "frac_of_sustained_peak": mma_tflops / peak_sus},
             "attn_gbs": attn_gbs, "attn_frac_hbm": attn_gbs / hbm,
             "secondary": {"kv_writer_gbs": kvw_gbs, "kv_writer_frac_hbm": kvw_gbs / hbm, "decode_gemm": dec,
                           "ms_per_step_parts": {n: part_ms[n] / K for n in names},
                           "hbm_peak_gbs": hbm, "peak_source": peak_src},
             "decoder": dec_res,
+            "study": study,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": Workload.LAUNCHES_PER_STEP * K,
-            "clocks": clk.summary(),
+            "clocks": ck,
         }
         print(json.dumps(line), flush=True)
     if ws > 1:

@@ -1,9 +1,8 @@
 // attention_noalloc.cu -- heal_attention_int16_noalloc: the INT16 attention call for
-// callers that cannot allocate device memory at call time (stream capture into a CUDA
-// graph, serving loops with a fixed memory budget, plugin hosts that only hand over
-// input and output tensors).  The split-context partial results that heal_attention_int16
-// keeps in a caller-provided workspace live here in one fixed array of the library's own
-// device memory.
+// callers that cannot allocate device memory when they call it (serving loops that allow no
+// allocation after start-up, plugin hosts that hand over only input and output tensors).
+// The scratch that heal_attention_int16 takes from a caller-provided workspace lives here in
+// one fixed array of the library's own device memory.
 #include <mutex>
 
 #include "heal_internal.h"
@@ -20,7 +19,8 @@ std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
 
 // Device address of g_attn_scratch on the current device, looked up once per device (the
-// first call on a device does this; it must not run during stream capture).
+// first call on a device does this; it must not run during stream capture).  The address is
+// kept for the life of the process: it is not looked up again after cudaDeviceReset.
 heal_status_t scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {

@@ -30,16 +30,25 @@ _LINEARS = ("wqkv", "wo", "wgu", "wdown")
 
 
 class Decoder:
-    def __init__(self, cfg, weights, device, max_len=None, presplit_weights=True):
+    def __init__(self, cfg, weights, device, max_len=None, presplit_weights=True, weights16=False):
         """presplit_weights: split every linear weight once into its 16-bit hi and lo parts
         (heal_split, the same encodings the GEMM kernels produce) and keep only those; the
-        GEMMs then split only the activations.  The results are the same bits either way."""
+        GEMMs then split only the activations.  The results are the same bits either way.
+        weights16: hold every linear weight as FP16 values instead (the weights must be
+        FP16-representable, as a 16-bit model's are; converting others rounds them): every
+        GEMM is then the two-product form, Ah.W + 2^-11 Al.W with only the activations split
+        (technical summary, section 2.B), and streams half the weight bytes."""
         self.cfg = c = cfg
         self.dev = device
         self.max_len = max_len or c.max_pos
         self.w = {k: v.to(device).contiguous() for k, v in weights.items()}
         self.parts = {}
-        if presplit_weights:
+        self.w16 = {}
+        if weights16:
+            for k in [f"{n}{l}" for l in range(c.layers) for n in _LINEARS] + ["lm_head"]:
+                self.w16[k] = self.w[k].half()
+                self.w[k] = None
+        elif presplit_weights:
             names = [f"{n}{l}" for l in range(c.layers) for n in _LINEARS] + ["lm_head"]
             for k in names:
                 w = self.w[k]
@@ -71,7 +80,9 @@ class Decoder:
 
     # ---- building blocks (each one library call) ----
     def _linear(self, x, key, out):
-        if key in self.parts:
+        if key in self.w16:
+            H.heal_gemm_compensated(x, self.w16[key], out, b_16bit=True, workspace=self.gemm_ws, b_static=True)
+        elif key in self.parts:
             hi, lo = self.parts[key]
             H.heal_gemm_compensated(x, hi, out, b_lo=lo, workspace=self.gemm_ws, b_static=True)
         else:

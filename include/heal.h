@@ -200,27 +200,31 @@ size_t heal_attention_workspace_bytes_gqa(int B, int Hq, int Hkv, int Tq, int Tm
 size_t heal_attention_workspace_bytes(int B, int Hq, int Tq, int Tmax);
 
 /* Fixed-scratch variant of heal_attention_int16.  The paper has no counterpart to this
- * entry point; it exists for callers that cannot allocate device memory when they call
- * attention, and so cannot pass a `workspace`: code that runs while a stream is being
- * captured into a CUDA graph (allocation is not allowed during capture), serving loops
- * that forbid allocation after start-up to keep a fixed memory budget, and plugin hosts
- * that hand an operator only its input and output tensors.
+ * entry point.  It is for callers that cannot allocate device memory at the time they call
+ * attention, and so cannot pass a `workspace`: serving loops that forbid any allocation
+ * after start-up to keep a fixed memory budget, and plugin hosts that hand an operator only
+ * its input and output tensors and no allocator.
  * Arguments and results are those of heal_attention_int16 without workspace and
- * workspace_bytes.  The split-context partial results go instead to one array of
+ * workspace_bytes; the result is the same, bit for bit, as that call's.  The split-context
+ * partial results (and, for prefill shapes, the byte planes) go instead to one array of
  * HEAL_ATTN_STATIC_SCRATCH_BYTES bytes in libheal.so's own device memory, which every GPU
  * that loads the library holds until the process exits.  This call allocates and frees
  * nothing.
  *   - The first call on a device looks up that array's device address, with that device
- *     current.  Make this first call before any stream capture.
+ *     current, and keeps it for the life of the process.  Make this first call before any
+ *     stream capture.  The kept address does not survive cudaDeviceReset(): after a reset
+ *     of a device, do not call this entry point on that device again in the same process.
  *   - All calls share the one array and it keeps the last call's contents.  Nothing in it
  *     needs to start at zero: every partial result a call reads was written earlier in the
  *     same call.  Calls whose kernels overlap on the GPU (other streams, other host
  *     threads) race on the array and corrupt each other's results: serialise them.
  *   - Size limit: the scratch the workspace variant would need,
- *     heal_attention_workspace_bytes_gqa(B, Hq, Hkv, Tq, Tmax), must fit the array (for
- *     decode shapes: B * Hq * Tq <= 7939; the prefill kernel's byte planes need
- *     6 * B * Hkv * Tmax * 128 + 2 * B * Hq * Tq * 128 bytes).  Larger problems return
- *     HEAL_ERR_UNSUPPORTED and launch nothing.                                            */
+ *     heal_attention_workspace_bytes_gqa(B, Hq, Hkv, Tq, Tmax), must fit the array.  For
+ *     decode shapes ((Hq/Hkv) * Tq <= 8) that is B * Hq * Tq <= 7939; for prefill shapes
+ *     6 * B * Hkv * Tmax * 128 + 2 * B * Hq * Tq * 128 + 4 * B * Hkv * Tmax bytes, plus
+ *     4 * B * Hkv rounded up to a multiple of 128, must not exceed 8 MiB (one KV head of an
+ *     8192-token cache is already 6 MiB).  Larger problems return HEAL_ERR_UNSUPPORTED and
+ *     launch nothing.                                                                       */
 #define HEAL_ATTN_STATIC_SCRATCH_BYTES (8u << 20)
 heal_status_t heal_attention_int16_noalloc(const int16_t* q, const float* q_scale,
                                            const int16_t* k_cache, const float* k_scale,

@@ -10,6 +10,11 @@ workload, so no expected value comes from the CUDA path.
     accumulated in FP32.  The test bound is
         ||O - O_ref|| / ||O_ref||  <=  4 * (x_max + 8) * 2^-23 + 1e-6
     which is about 1e-5 at x_max ~ 12 and grows only with extreme logits.
+    The same bound holds row by row once it is taken relative to the softmax-weighted sum
+    of |v| (each weight's error multiplies |v_t|, never v_t's signed sum), so every query
+    row is also checked on its own:
+        ||O_row - O_ref_row|| <= tol * || sum_t p_t |v_t| ||_row
+    which localises one bad head or query that the whole-tensor ratio would average away.
 """
 import math
 
@@ -82,7 +87,18 @@ def check(q, qs, kq, kss, vq, vss, kv_len, scale, causal=False, hook=True):
     err = np.linalg.norm(out - ref) / np.linalg.norm(ref)
     assert np.all(np.isfinite(out))
     assert err <= tol, (err, tol)
+    abs_ref = OA.attention(q, qs, kq, kss, np.abs(np.asarray(vq, np.int64)), vss, kv_len, scale, causal=causal)
+    assert_rows_within(out, ref, abs_ref, tol)
     return err
+
+
+def assert_rows_within(out, ref, abs_ref, tol):
+    """Per query row: ||out - ref|| <= tol * ||sum_t p_t |v_t||| (rows that see no token
+    must be exactly zero on both sides)."""
+    d = np.linalg.norm((out - ref).reshape(-1, out.shape[-1]), axis=1)
+    a = np.linalg.norm(abs_ref.reshape(-1, out.shape[-1]), axis=1)
+    bad = np.nonzero(d > tol * a)[0]
+    assert bad.size == 0, [(int(r), float(d[r]), float(tol * a[r])) for r in bad[:8]]
 
 
 def test_decode_gqa_ragged_lengths():

@@ -21,6 +21,26 @@ TOL_BF16 = 2e-5
 TOL_ACCUM = 5e-7      # GPU vs the oracle's unrounded three-product emulation
 
 
+def assert_elementwise(C, A, B, fmt=S.FP16_S11, chan_exp=None, rows=None):
+    """Element-wise bound against the oracle's unrounded three-product emulation:
+        |C - C_emul|_ij <= (nc + 8) * 2^-24 * (|A| |B|)_ij,   nc = ceil(K / 64).
+    The ordered FP32 sum of the nc chunk values makes at most nc - 1 roundings of 2^-24 of a
+    partial sum bounded by (|A||B|)_ij; each chunk's value comes from four main tensor-core
+    steps that truncate to FP32 (2^-23 of the chunk's running magnitude each, 8 units of
+    2^-24 over all chunks) plus 2^-11-scaled corrections; the FP32 store adds one more.  A
+    wrong tile, a ragged edge read from the wrong place or a dropped term is O(|C|) and far
+    outside it.  `rows` selects the rows of A that C holds."""
+    A = np.asarray(A, np.float64 if A.dtype == np.float64 else np.float32)
+    if rows is not None:
+        A = A[rows]
+    emu = G.gemm_emulated(A, B, fmt, chan_exp)
+    absab = np.abs(np.asarray(A, np.float64)) @ np.abs(np.asarray(B, np.float64))
+    nc = -(-A.shape[1] // 64)
+    excess = np.abs(np.asarray(C, np.float64) - emu) - (nc + 8) * 2.0 ** -24 * absab
+    i, j = np.unravel_index(int(np.argmax(excess)), excess.shape)
+    assert excess[i, j] <= 0, (int(i), int(j), float(C[i, j]), float(emu[i, j]), float(absab[i, j]))
+
+
 def test_square_256_fp16_s11():
     A, B = synthetic.gemm_square(256, seed=0)
     A, B = A.numpy(), B.numpy()
@@ -28,6 +48,7 @@ def test_square_256_fp16_s11():
     ref = G.gemm_ref(A, B)
     assert G.normwise_rel_err(C, ref) <= TOL_FP16
     assert G.normwise_rel_err(C, G.gemm_emulated(A, B, S.FP16_S11)) <= TOL_ACCUM
+    assert_elementwise(C, A, B)
 
 
 def test_square_256_bf16():
@@ -37,6 +58,7 @@ def test_square_256_bf16():
     ref = G.gemm_ref(A, B)
     assert G.normwise_rel_err(C, ref) <= TOL_BF16
     assert G.normwise_rel_err(C, G.gemm_emulated(A, B, S.BF16)) <= TOL_ACCUM
+    assert_elementwise(C, A, B, S.BF16)
 
 
 @pytest.mark.parametrize("shape", [(200, 300, 333), (1, 129, 70), (257, 64, 1000), (130, 17, 64), (5, 1000, 37)])
@@ -51,6 +73,7 @@ def test_ragged_shapes_against_oracle(shape, b_layout):
     ref = G.gemm_ref(X, W)
     assert G.normwise_rel_err(C, ref) <= TOL_FP16
     assert np.all(np.isfinite(C))
+    assert_elementwise(C, X, W)
 
 
 @pytest.mark.parametrize("tile", [heal.TILE_128x128, heal.TILE_256x256_PAIR])
@@ -125,6 +148,7 @@ def test_outlier_channel_rescale():
     e = G.suggest_channel_exponents(A)
     good = gemm(A, B, tile=heal.TILE_128x128, chan_exp=e)
     assert G.normwise_rel_err(good, ref) <= TOL_FP16
+    assert_elementwise(good, A, B, chan_exp=e)
     good_skinny = gemm(A[:8], B, tile=heal.TILE_SKINNY_SPLITK, chan_exp=e)
     assert np.array_equal(good_skinny, good[:8])
 
@@ -142,6 +166,7 @@ def test_decode_shapes_full_oracle(M):
     X, W = X.numpy(), W.numpy()
     C = gemm(X, W)            # automatic config (skinny split-K)
     assert G.normwise_rel_err(C, G.gemm_ref(X, W)) <= TOL_FP16
+    assert_elementwise(C, X, W)
 
 
 def test_prefill_full_size_sampled_rows():
@@ -158,6 +183,7 @@ def test_prefill_full_size_sampled_rows():
     got = C[torch.as_tensor(rows, device=d)].cpu().numpy()
     assert G.normwise_rel_err(got, ref) <= TOL_FP16
     assert torch.isfinite(C).all()
+    assert_elementwise(got, X.numpy(), W.numpy(), rows=rows)
 
 
 @pytest.mark.parametrize("shape", [(512, 512, 512), (300, 520, 333), (256, 1000, 64), (777, 300, 1500)])
@@ -173,6 +199,7 @@ def test_cta_pair_config_bitwise_and_oracle(shape, b_layout):
     c_single = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_128x128)
     assert np.array_equal(c_pair, c_single)
     assert G.normwise_rel_err(c_pair, G.gemm_ref(X, W)) <= TOL_FP16
+    assert_elementwise(c_pair, X, W)
 
 
 @pytest.mark.parametrize("fmt", [heal.SPLIT_FP16_S11, heal.SPLIT_BF16])
@@ -326,3 +353,80 @@ def test_split_pass_over_b_is_bitwise_identical(M, b_layout, fmt):
     # and against the FP64 product (FP16 split: the 1e-6 bound)
     if fmt == heal.SPLIT_FP16_S11:
         assert G.normwise_rel_err(C.cpu().numpy().astype(np.float64), G.gemm_ref(X.numpy(), W.numpy())) <= TOL_FP16
+
+
+@pytest.mark.parametrize("M", [8, 64, 300])
+@pytest.mark.parametrize("b_layout", [0, 1])
+def test_two_product_with_outlier_channel_rescale(M, b_layout):
+    """The two-product form with the outlier-channel rescale (technical summary, section 2.B,
+    "Overflow Handling"): channels of X at 1e5 and 3e4 would overflow the FP16 hi part; the
+    caller scales W's rows by 2^e_k before the FP16 conversion and passes e, the kernel
+    scales X's columns by 2^-e_k before the split.  Same bits in every tile configuration,
+    within 1e-6 of the FP64 product with those 16-bit weights."""
+    K, N = 520, 648
+    X, W = synthetic.gemm_decode(M, K=K, N=N)
+    X = X.clone()
+    X[:, 5] *= 1e5
+    X[:, 301] *= 3e4
+    e = G.suggest_channel_exponents(X.numpy())
+    assert e[5] > 0 and e[301] > 0
+    Ws = torch.from_numpy(np.ldexp(W.numpy().astype(np.float64), e.astype(np.int64)[:, None]).astype(np.float32))
+    W16 = Ws.half()                                      # the rescaled 16-bit weights the caller keeps
+    assert torch.isfinite(W16.float()).all()
+    W16_eff = np.ldexp(W16.float().numpy().astype(np.float64), -e.astype(np.int64)[:, None])   # exact
+    ref = G.gemm_ref(X.numpy(), W16_eff)
+    Bin = W16 if b_layout == 0 else W16.t().contiguous()
+    d = dev()
+    ce = torch.as_tensor(e).to(d)
+    tiles = [heal.TILE_128x128, heal.TILE_256x256_PAIR] + (
+        [heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK] if M <= 64 else [])
+    outs = []
+    for t in tiles:
+        Xd, Wd = X.to(d).contiguous(), Bin.to(d).contiguous()
+        C = torch.full((M, N), float("nan"), device=d)
+        nbytes = heal.heal_gemm_workspace_bytes(M, N, K, t)
+        ws = torch.empty(nbytes // 4, dtype=torch.float32, device=d) if nbytes else None
+        heal.heal_gemm_compensated(Xd, Wd, C, tile_config=t, b_layout=b_layout, b_16bit=True, chan_exp=ce,
+                                   workspace=ws)
+        status_ok()
+        outs.append(to_np(C).astype(np.float64))
+    for t, o in zip(tiles[1:], outs[1:]):
+        assert np.array_equal(o, outs[0]), t
+    assert np.all(np.isfinite(outs[0]))
+    assert G.normwise_rel_err(outs[0], ref) <= TOL_FP16
+    # without the rescale the FP16 hi part of the outlier channels overflows
+    Xd = X.to(d).contiguous()
+    C = torch.empty(M, N, device=d)
+    heal.heal_gemm_compensated(Xd, Bin.to(d).contiguous(), C, tile_config=heal.TILE_128x128, b_layout=b_layout,
+                               b_16bit=True)
+    status_ok()
+    assert not torch.isfinite(C).all()
+
+
+def test_column_shards_reassemble_bitwise():
+    """The multi-GPU partition (output columns split into contiguous 128-aligned shards, one
+    per rank, no exchange) run as separate library calls on one device: each shard reads its
+    columns of B through the leading dimension and writes its columns of C at an offset, and
+    the shards put together are the single call's bits, in every world size tried."""
+    from error_compensated_gemm_b200.shard import shard_range
+    d = dev()
+    M, K, N = 300, 1000, 1800
+    X, W = synthetic.gemm_prefill(M=M, K=K, N=N)
+    Xd, Wd = X.to(d), W.to(d)
+    full = torch.empty(M, N, device=d)
+    heal.heal_gemm_compensated(Xd, Wd, full)
+    status_ok()
+    for world in (2, 3, 8):
+        C = torch.full((M, N), float("nan"), device=d)
+        for r in range(world):
+            n0, n1 = shard_range(N, world, r, align=128)
+            heal.heal_gemm_compensated(Xd, Wd[:, n0:n1], C[:, n0:n1])
+        status_ok()
+        assert torch.equal(C.view(torch.int32), full.view(torch.int32)), world
+    # row shards (the other partition) too
+    C = torch.full((M, N), float("nan"), device=d)
+    for r in range(3):
+        m0, m1 = shard_range(M, 3, r, align=64)
+        heal.heal_gemm_compensated(Xd[m0:m1], Wd, C[m0:m1])
+    status_ok()
+    assert torch.equal(C.view(torch.int32), full.view(torch.int32))
