@@ -18,7 +18,7 @@
 // sum 256*hi*P + lo*P = v*P.  These are the two FP16 tensors the INT16 value is unpacked
 // into for the floating-point contraction.
 //
-// Work decomposition: a persistent grid (two CTAs per SM); CTA c owns the contiguous
+// Work decomposition: a persistent grid (three CTAs per SM); CTA c owns the contiguous
 // slice [total*c/grid, total*(c+1)/grid) of the sequence of (batch*kv_head, 64-token
 // block) units.  Warp roles: a TMA producer streams 64-token K and V tiles (128-byte
 // swizzle) into a two-stage ring; four QK warps take 16 tokens each (exact S^T on the
@@ -43,11 +43,12 @@ namespace {
 
 constexpr int kBlk = 64;          // tokens per pipeline stage
 // Warp roles per CTA: kQK warps for QK^T and the softmax step (16 tokens each), kPV warps
-// for PV (D/4 dims each), one TMA producer.  Two K/V stages per CTA, two CTAs per SM
-// (16 compute warps and four stages per SM).
+// for PV (D/4 dims each), one TMA producer.  Two K/V stages per CTA, three CTAs per SM
+// (24 compute warps and six stages per SM: the consumers' instruction streams are latency
+// bound, so more warps per SM keep more K/V bytes moving).
 constexpr int kQK = 4, kPV = 4;
 constexpr int kStages = 2;
-constexpr int kMinBlocks = 2;
+constexpr int kMinBlocks = 3;
 constexpr int kAttnThreads = (kQK + kPV + 1) * 32;
 constexpr int kRows = 8;          // query rows per CTA: (Hq/Hkv) * Tq <= 8
 constexpr int kMaxGrid = 1024;
@@ -168,8 +169,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;                                                  // kStages x kStageBytes
-  uint4* pb = reinterpret_cast<uint4*>(smem + kStages * kStageBytes);      // [2][kQK steps][2 parts][32 lanes]
-  uint4* qf_sm = pb + 2 * kQK * 2 * 32;                                    // [kKSteps32][32 lanes]
+  uint4* pb = reinterpret_cast<uint4*>(smem + kStages * kStageBytes);      // [2][kQK steps][32 lanes]
+  uint4* qf_sm = pb + 2 * kQK * 32;                                        // [kKSteps32][32 lanes]
   float* sc_sm = reinterpret_cast<float*>(qf_sm + kKSteps32 * 32);         // [kStages][K, V][kBlk]
   float* meta = sc_sm + kStages * 2 * kBlk;                                // [2][16]: scale of O per row, E
   float* red = meta + 2 * 16;                                              // [2][kQK][kRows] block maxima
@@ -513,28 +514,23 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
           }
         }
       }
-      // FP16 P_hi and residual r = P' - P_hi, and both times 256: the B fragments of PV
-      uint32_t ph_[2], pr_[2], ph256[2], pr256[2];
+      // FP16 P_hi and residual r = P' - P_hi: the B fragments of PV (the PV warps form the
+      // 256x copies themselves)
+      uint32_t ph_[2], pr_[2];
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
         const __half2 h = __floats2half2_rn(pt[th][0], pt[th][1]);
         const float2 hf = __half22float2(h);
         const __half2 rr = __floats2half2_rn(__fsub_rn(pt[th][0], hf.x), __fsub_rn(pt[th][1], hf.y));
-        const __half2 k256 = __half2half2(__ushort_as_half(0x5C00));   // 256.0
-        const __half2 h256 = __hmul2(h, k256), r256 = __hmul2(rr, k256); // exact: powers of two
         ph_[th] = *reinterpret_cast<const uint32_t*>(&h);
         pr_[th] = *reinterpret_cast<const uint32_t*>(&rr);
-        ph256[th] = *reinterpret_cast<const uint32_t*>(&h256);
-        pr256[th] = *reinterpret_cast<const uint32_t*>(&r256);
       }
       // hand the block to the PV warps (the buffer is free once they finished block j - 2)
       if (!mbar_wait(&pfree[jb], jph ^ 1u, abort_flag, a.status, 213)) {
         ok = false;
         break;
       }
-      uint4* pbw = pb + ((jb * kQK + w) * 2) * 32;
-      pbw[lane] = make_uint4(ph256[0], ph256[1], ph_[0], ph_[1]);
-      pbw[32 + lane] = make_uint4(pr256[0], pr256[1], pr_[0], pr_[1]);
+      pb[(jb * kQK + w) * 32 + lane] = make_uint4(ph_[0], ph_[1], pr_[0], pr_[1]);
       if (w == 0) {
         if (g8 == 0) {
           meta[jb * 16 + qc] = __fmul_rn(alpha[0], escale);
@@ -611,8 +607,18 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
     // ---- O^T += V^T P'^T  (256*hi*P + lo*P with P = P_hi + r), 16 tokens per step ----
 #pragma unroll
     for (int ts = 0; ts < kQK; ++ts) {
-      const uint4 fh = pb[((jb * kQK + ts) * 2) * 32 + lane];        // P_hi * 256, P_hi
-      const uint4 fr = pb[((jb * kQK + ts) * 2 + 1) * 32 + lane];    // r * 256, r
+      const uint4 f = pb[(jb * kQK + ts) * 32 + lane];               // P_hi, r
+      // 256 * P_hi and 256 * r: exact (powers of two; |P'| < 64)
+      const __half2 k256 = __half2half2(__ushort_as_half(0x5C00));
+      uint4 fh, fr;                                                  // (256 x, x) of P_hi / r
+      {
+        const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&f.x), k256);
+        const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&f.y), k256);
+        const __half2 r0 = __hmul2(*reinterpret_cast<const __half2*>(&f.z), k256);
+        const __half2 r1 = __hmul2(*reinterpret_cast<const __half2*>(&f.w), k256);
+        fh = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1), f.x, f.y);
+        fr = make_uint4(*reinterpret_cast<const uint32_t*>(&r0), *reinterpret_cast<const uint32_t*>(&r1), f.z, f.w);
+      }
 #pragma unroll
       for (int dl = 0; dl < kDT; ++dl) {
         const int dt = v * kDT + dl;
@@ -689,7 +695,7 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
 template <int D>
 constexpr int attn_smem_bytes() {
   return kStages * (2 * kBlk * D * 2)          // K / V stages
-         + 2 * kQK * 2 * 32 * 16               // P' operand buffers
+         + 2 * kQK * 32 * 16                   // P' operand buffers
          + (D / 32) * 32 * 16                  // Q table
          + kStages * 2 * kBlk * 4              // K / V scales
          + (2 * 16 + 2 * kQK * kRows + kQK * kRows + kRows) * 4   // meta, maxima, sums
