@@ -367,6 +367,55 @@ def decoder_section(torch, heal, synthetic, dev, stream, prompt_len=512, steps=1
                     "the GEMMs split only the activations"}
 
 
+def glue_section(torch, heal, synthetic, dev, stream, reps):
+    """The split kernel on the prefill weights and each decoder glue kernel on the decoder's
+    prefill shapes (512 tokens, hidden 4096, 32/8 heads of 128, FFN 14336, vocab 128256),
+    each timed with CUDA events over `reps` launches: a profiling case for the small kernels."""
+    from error_compensated_gemm_b200.decoder import rope_tables
+    n, H, Hq, Hkv, D, F, V = 512, 4096, 32, 8, 128, 14336, 128256
+    W = synthetic.normal((4096, 14336), seed=1, std=0.02).to(dev)
+    hi = torch.empty(W.shape, dtype=torch.int16, device=dev)
+    lo = torch.empty_like(hi)
+    table = synthetic.normal((V, H), seed=10).to(dev)
+    ids = synthetic.prompt_ids(n, V).to(dev)
+    h = torch.empty(n, H, device=dev)
+    x = torch.empty(n, H, device=dev)
+    qkv = synthetic.normal((n, (Hq + 2 * Hkv) * D), seed=11).to(dev)
+    pos = torch.arange(n, dtype=torch.int32, device=dev)
+    cos, sin = (t.to(dev) for t in rope_tables(1024, D, 500000.0))
+    gu = synthetic.normal((n, 2 * F), seed=12).to(dev)
+    act = torch.empty(n, F, device=dev)
+    logits = synthetic.normal((8, V), seed=13).to(dev)
+    am = torch.empty(8, dtype=torch.int32, device=dev)
+    heads = synthetic.normal((1, Hq, n, D), seed=14).to(dev)
+    rows = torch.empty(1, n, Hq, D, device=dev)
+    calls = {
+        "split_4096x14336": lambda: heal.heal_split(W, hi, lo),
+        "embedding_gather": lambda: heal.heal_embedding_gather(table, ids, h),
+        "rmsnorm": lambda: heal.heal_rmsnorm(h, None, x, 1e-5),
+        "rope_q": lambda: heal.heal_rope(qkv, Hq, D, pos, cos, sin),
+        "swiglu": lambda: heal.heal_swiglu(gu, act),
+        "add": lambda: heal.heal_add(h, x),
+        "argmax_8x128256": lambda: heal.heal_argmax(logits, am),
+        "heads_to_rows": lambda: heal.heal_heads_to_rows(heads, rows),
+    }
+    out = {}
+    for name, fn in calls.items():
+        fn()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        out[name] = {"us_per_launch": 1e3 * e0.elapsed_time(e1) / reps}
+    st = heal.heal_get_device_status()
+    if st != heal.HEAL_OK:
+        raise SystemExit(f"device status: {heal.status_string(st)}")
+    return out
+
+
 # causal INT16 self-attention over a long prompt (the prefill kernel: 128-row query tiles on
 # the tcgen05 tensor cores), timed in its own loop after the step
 PREFILL_ATTN = {"B": 1, "T": 8192, "Hkv": 8, "Hq": 32, "D": 128}
@@ -511,8 +560,9 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--only", choices=["prefill", "decode", "kv_writer", "attention", "attention_prefill"],
-                    help="profiling case: run only this part of the step")
+    ap.add_argument("--only", choices=["prefill", "decode", "kv_writer", "attention", "attention_prefill", "glue"],
+                    help="profiling case: run only this part of the step (glue: the split kernel and the "
+                         "decoder glue kernels on the decoder's shapes)")
     ap.add_argument("--prefill-shape", default=None, help="M,N,K of the prefill GEMM (profiling case)")
     ap.add_argument("--kv-batch", type=int, default=None, help="batch of the KV workload (profiling case)")
     ap.add_argument("--prompt-len", type=int, default=None,
@@ -544,6 +594,11 @@ def main():
             print(json.dumps(reproducibility_study(dev)), flush=True)
         return 0
     peaks, peak_src = load_peaks()
+    if args.only == "glue":
+        res = glue_section(torch, heal, synthetic, dev, torch.cuda.current_stream(), max(1, args.steps))
+        if rank == 0:
+            print(json.dumps({"profiling_case": args.only, "result": res}), flush=True)
+        return 0
     if args.only == "attention_prefill":
         if args.prompt_len:
             PREFILL_ATTN["T"] = args.prompt_len

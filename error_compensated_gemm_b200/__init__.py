@@ -9,7 +9,7 @@ library; the first call does, and fails loudly if the CUDA extension is missing.
 """
 from ._binding import (  # noqa: F401
     EXPORTED, HEAL_ERR_CUDA, HEAL_ERR_INVALID_ARGUMENT, HEAL_ERR_TIMEOUT, HEAL_ERR_UNSUPPORTED, HEAL_OK,
-    SPLIT_BF16, SPLIT_FP16_S11, TILE_128x128, TILE_256x256_PAIR, TILE_AUTO, TILE_SKINNY_FULLK, TILE_SKINNY_SPLITK, GemmOpts, HealError,
+    SPLIT_BF16, SPLIT_FP16_S11, TILE_128x128, TILE_256x256_PAIR, TILE_AUTO, TILE_SKINNY_CHAIN, TILE_SKINNY_FULLK, TILE_SKINNY_SPLITK, GemmOpts, HealError,
     gemm_opts, heal_attention_int16, heal_attention_int16_noalloc, heal_attention_workspace_bytes,
     heal_attention_workspace_bytes_gqa, heal_gemm_compensated,
     heal_gemm_workspace_bytes, heal_get_device_status, heal_kv_quantize_int16, heal_split, heal_version, lib,

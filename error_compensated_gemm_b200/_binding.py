@@ -9,7 +9,7 @@ LIB_PATH = os.path.join(HERE, "libheal.so")
 
 HEAL_OK, HEAL_ERR_INVALID_ARGUMENT, HEAL_ERR_UNSUPPORTED, HEAL_ERR_CUDA, HEAL_ERR_TIMEOUT = range(5)
 SPLIT_FP16_S11, SPLIT_BF16 = 0, 1
-TILE_AUTO, TILE_128x128, TILE_256x256_PAIR, TILE_SKINNY_SPLITK, TILE_SKINNY_FULLK = -1, 0, 1, 2, 3
+TILE_AUTO, TILE_128x128, TILE_256x256_PAIR, TILE_SKINNY_SPLITK, TILE_SKINNY_FULLK, TILE_SKINNY_CHAIN = -1, 0, 1, 2, 3, 4
 
 # every symbol the public header declares
 EXPORTED = ("heal_split", "heal_gemm_compensated", "heal_gemm_workspace_bytes", "heal_kv_quantize_int16",

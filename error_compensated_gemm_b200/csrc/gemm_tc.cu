@@ -20,7 +20,11 @@
 //   warps 8-11  epilogue: drain each 64-wide K chunk from TMEM and add it to the running
 //               FP32 sum in registers (round-to-nearest, ascending chunk order), then
 //               store C.  In split-K mode every chunk value goes to a workspace instead,
-//               and heal_chunk_reduce adds them in the same order.
+//               and heal_chunk_reduce adds them in the same order.  In chain mode (a
+//               cluster of S CTAs per tile, each owning a contiguous run of chunks) every
+//               chunk keeps its own TMEM accumulator; at the end the running FP32 sum is
+//               handed from CTA to CTA through distributed shared memory in ascending chunk
+//               order, and the last CTA of the cluster stores C.
 // Because every chunk value comes from the same sequence of tensor-core instructions and
 // chunk values are added in a fixed order, C is identical bit for bit across runs, tile
 // shapes, operand swapping and split-K.
@@ -57,6 +61,8 @@ struct GemmArgs {
   int Mk, Nk, K;            // kernel-space rows of kernel-A, rows of kernel-B, reduction
   int tiles_m, tiles_n, num_chunks;
   int splitk;               // 1: write chunk partials to ws
+  int chain;                // S >= 2: chain mode, S CTAs (one cluster) per tile, 0 otherwise
+  int tmem_cols;            // TMEM columns this kernel allocates (power of two, 32 .. 512)
   float* out;
   long long out_si, out_sj; // element (i, j) -> out[i*si + j*sj]
   float* ws;                // [num_chunks][Nk][Mk] chunk values (split-K mode)
@@ -74,7 +80,9 @@ struct Cfg {
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (216 * 1024) / kStageBytes > 8 ? 8 : (216 * 1024) / kStageBytes;
   static constexpr int kTmemCols = (2 * BN) <= 32 ? 32 : (2 * BN) <= 64 ? 64 : (2 * BN) <= 128 ? 128 : (2 * BN) <= 256 ? 256 : 512;
-  static constexpr int kSmemBytes = kStages * kStageBytes + 1024 /*barriers*/ + 1024 /*align*/;
+  // chain mode (BN <= 32): the running sum a predecessor CTA hands over, 128 rows x BN FP32
+  static constexpr int kSumBytes = BN <= 32 ? kBM * BN * 4 : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kSumBytes + 1024 /*barriers*/ + 1024 /*align*/;
   static_assert(kStages >= 2, "at least two stages");
 };
 
@@ -88,8 +96,15 @@ struct WorkIter {
   __device__ WorkIter(const GemmArgs& a) {
     ntiles = a.tiles_m * a.tiles_n;
     nc = a.num_chunks;
-    splitk = a.splitk;
-    if (splitk) {
+    splitk = a.splitk || a.chain;
+    if (a.chain) {
+      // one tile per cluster of S CTAs; CTA rank r owns chunks [r*nc/S, (r+1)*nc/S)
+      const int S = a.chain, t = blockIdx.x / S, r = blockIdx.x % S;
+      u = t * nc + (r * nc) / S;
+      u_end = t * nc + ((r + 1) * nc) / S;
+      tile = t;
+      chunk = u - t * nc;
+    } else if (splitk) {
       const long long total = (long long)ntiles * nc;
       u = (int)((total * blockIdx.x) / gridDim.x);
       u_end = (int)((total * (blockIdx.x + 1)) / gridDim.x);
@@ -310,7 +325,8 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   // 1024-byte alignment of the shared-window address (128-byte swizzle atoms)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes);
+  float* sum_buf = reinterpret_cast<float*>(smem + S * C::kStageBytes);   // chain mode: [128 rows][BN]
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kSumBytes);
   uint64_t* full = bars;                 // TMA -> split       (tx bytes)
   uint64_t* split_done = bars + S;       // split -> MMA       (all split threads arrive)
   uint64_t* empty = bars + 2 * S;        // MMA -> TMA         (tcgen05.commit)
@@ -319,6 +335,7 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   uint64_t* mma_done = bars + 3 * S + 4; // MMA drain on exit
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
+  uint64_t* chain_bar = bars + 3 * S + 7; // chain mode: the predecessor's running sum has landed
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -335,11 +352,12 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
       mbar_init(&acc_empty[b], kNumEpiWarps * 32);
     }
     mbar_init(mma_done, 1);
+    mbar_init(chain_bar, kNumEpiWarps * 32);
     *abort_flag = 0;
     fence_mbar_init();
   }
   if (warp == 0) {
-    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_alloc(tmem_slot, (uint32_t)args.tmem_cols);
     tmem_relinquish();
   }
   if (warp == 1 && lane == 0) {
@@ -350,6 +368,7 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   }
   tc_fence_before();
   __syncthreads();
+  if (args.chain) cluster_sync_all();   // every CTA's chain barrier is initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
@@ -363,9 +382,9 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
       // stages right away; everything else waits for the preceding grid to finish.
       int pre = 0;
       const uint64_t pol = l2_policy_evict_first();
-      // split-K: kernel-A (the weights) is read exactly once
+      // split-K and chain modes: kernel-A (the weights) is read exactly once
       auto load_a = [&](uint8_t* st, uint64_t* bar, int tm, int k0) {
-        if (args.splitk) load_operand_once<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, bar, tm * kBM, k0, pol);
+        if (args.splitk || args.chain) load_operand_once<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, bar, tm * kBM, k0, pol);
         else load_operand<kBM, A_MN, A_PRE>(st, &tmA, &tmA_lo, bar, tm * kBM, k0);
       };
       if (args.static_op != 0) {
@@ -413,14 +432,15 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
         const int b = it & 1;
         const uint32_t aph = (uint32_t)(it >> 1) & 1u;
         if (!mbar_wait(&split_done[s], ph, abort_flag, args.status, 110)) break;
-        if (!mbar_wait(&acc_empty[b], aph ^ 1u, abort_flag, args.status, 111)) break;
+        if (!args.chain && !mbar_wait(&acc_empty[b], aph ^ 1u, abort_flag, args.status, 111)) break;
         tc_fence_after();
         const uint32_t sa = smem_u32(stages + s * C::kStageBytes);
         const uint32_t sb = sa + C::kABytes;
         const uint64_t a_hi = OperandDesc<kBM, A_MN>::hi(sa), a_lo = OperandDesc<kBM, A_MN>::lo(sa);
         const uint64_t b_hi = OperandDesc<BN, B_MN>::hi(sb), b_lo = OperandDesc<BN, B_MN>::lo(sb);
         constexpr uint64_t dA = OperandDesc<kBM, A_MN>::kStep, dB = OperandDesc<BN, B_MN>::kStep;
-        const uint32_t d = tmem_base + (uint32_t)(b * BN);
+        // chain mode: every chunk of this CTA has its own accumulator columns
+        const uint32_t d = tmem_base + (uint32_t)((args.chain ? it : b) * BN);
         // corrections first: Ah.Bl then Al.Bh in the caller's operand order (a 16-bit
         // operand has no residual, so its correction product is absent)
 #pragma unroll
@@ -439,8 +459,9 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
 #pragma unroll
         for (int j = 1; j < kBK / 16; ++j) mma_f16(d, a_hi + j * dA, b_hi + j * dB, kIdesc, 1u);
         tc_commit(&empty[s]);
-        tc_commit(&acc_full[b]);
+        if (!args.chain) tc_commit(&acc_full[b]);
       }
+      if (args.chain) tc_commit(&acc_full[0]);   // every chunk of this CTA is in TMEM
       // drain: every MMA issued by this thread has completed before TMEM is released
       tc_commit(mma_done);
       volatile int dummy = 0;
@@ -484,9 +505,71 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
     float acc[BN];
 #pragma unroll
     for (int t = 0; t < BN; ++t) acc[t] = 0.0f;
+    if constexpr (BN <= 32) {
+      if (args.chain) {
+        // ---- chain mode: add this CTA's chunk values onto the predecessor's running sum,
+        // in ascending chunk order, and hand the sum on (or store C at the end of K) ----
+        const WorkIter w0(args);
+        const int nloc = w0.u_end - w0.u;
+        const int r = (int)(blockIdx.x % (unsigned)args.chain);
+        bool ok = nloc > 0 && mbar_wait(&acc_full[0], 0u, abort_flag, args.status, 140);
+        if (ok) {
+          tc_fence_after();
+          if (r > 0) {
+            ok = mbar_wait_cluster(chain_bar, 0u, abort_flag, args.status, 141);
+            if (ok) {
+#pragma unroll
+              for (int t = 0; t < BN; t += 4) {
+                const float4 v4 = *reinterpret_cast<const float4*>(sum_buf + i_local * BN + t);
+                acc[t] = v4.x;
+                acc[t + 1] = v4.y;
+                acc[t + 2] = v4.z;
+                acc[t + 3] = v4.w;
+              }
+            }
+          }
+        }
+        if (ok) {
+          const uint32_t tq = tmem_base + ((uint32_t)(quarter * 32) << 16);
+          for (int k = 0; k < nloc; ++k) {
+            const bool first = (r == 0 && k == 0);
+#pragma unroll
+            for (int c = 0; c < BN / 16; ++c) {
+              uint32_t v[16];
+              tmem_ld16(tq + (uint32_t)(k * BN + c * 16), v);
+              tmem_ld_wait();
+#pragma unroll
+              for (int t = 0; t < 16; ++t) {
+                const float dv = __uint_as_float(v[t]);
+                acc[c * 16 + t] = first ? dv : __fadd_rn(acc[c * 16 + t], dv);
+              }
+            }
+          }
+          tc_fence_before();
+          int tm, tn;
+          tile_coords(w0.tile, args.tiles_m, args.tiles_n, tm, tn);
+          const int gi = tm * kBM + i_local;
+          if (r + 1 < args.chain) {
+            // into the successor's sum buffer (same offset in its shared memory), then
+            // release-arrive on its chain barrier
+            const uint32_t dst = mapa_shared(smem_u32(sum_buf + i_local * BN), (uint32_t)(r + 1));
+#pragma unroll
+            for (int t = 0; t < BN; t += 4) st_shared_cluster_v4(dst + (uint32_t)(t * 4), acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
+            mbar_arrive_cluster(mapa_shared(smem_u32(chain_bar), (uint32_t)(r + 1)));
+          } else if (gi < args.Mk) {
+#pragma unroll
+            for (int t = 0; t < BN; ++t) {
+              const int gj = tn * BN + t;
+              if (gj < args.Nk) args.out[(size_t)gi * args.out_si + (size_t)gj * args.out_sj] = acc[t];
+            }
+          }
+        }
+        (void)ok;
+      }
+    }
     int it = 0;
     bool ok = true;
-    for (WorkIter w(args); w.valid(); w.advance(), ++it) {
+    for (WorkIter w(args); !args.chain && w.valid(); w.advance(), ++it) {
       const int b = it & 1;
       const uint32_t aph = (uint32_t)(it >> 1) & 1u;
       if (!mbar_wait(&acc_full[b], aph, abort_flag, args.status, 130)) {
@@ -556,8 +639,10 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  // chain mode: no CTA leaves while a peer may still write into its shared memory
+  if (args.chain) cluster_sync_all();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem_base, C::kTmemCols);
+  if (warp == 0) tmem_dealloc(tmem_base, (uint32_t)args.tmem_cols);
 }
 
 // ---------------------------------------------------------------------------------
@@ -588,6 +673,31 @@ constexpr int kPairOtherRegs =
         : ((kPairLaunchRegs * kPairThreads - kPairEpiRegs * kPairEpiWarps * 32) / (kPairEpiWarp0 * 32)) / 8 * 8;
 static_assert(kPairEpiWarp0 * 32 * kPairOtherRegs + kPairEpiWarps * 32 * kPairEpiRegs <= kPairLaunchRegs * kPairThreads,
               "register shares exceed the launch allocation");
+// Region pairs of a stage handed to split warp sw: the contiguous run [first, first + count)
+// of the n pairs (n = 32: A and B split here; n = 16: only A).  The shares follow the SM
+// sub-partitions: split warps sw = 2, 3 (warps 4, 5) are the only split warps on theirs,
+// beside the producer (warp 0) and the MMA issuer or forwarder (warp 1), which mostly wait;
+// the other four share theirs two by two, so the two lone warps take the larger shares.
+// (first, count) of every warp is packed 10 bits per warp (6 + 4): register arithmetic
+// rather than a table in local memory.
+constexpr uint64_t pack_shares(int s0, int s1, int s2, int s3, int s4, int s5) {
+  const int c[6] = {s0, s1, s2, s3, s4, s5};
+  uint64_t v = 0;
+  int first = 0;
+  for (int i = 0; i < 6; ++i) {
+    v |= (uint64_t)(first | (c[i] << 6)) << (10 * i);
+    first += c[i];
+  }
+  return v;
+}
+__device__ __forceinline__ void split_share(int sw, int n, int& first, int& count) {
+  //                                      sw: 0  1  2  3  4  5
+  constexpr uint64_t k32 = pack_shares(5, 5, 6, 6, 5, 5), k16 = pack_shares(3, 3, 3, 3, 2, 2);
+  const uint32_t e = (uint32_t)((n == 32 ? k32 : k16) >> (10 * sw)) & 1023u;
+  first = (int)(e & 63u);
+  count = (int)(e >> 6);
+}
+static_assert(kPairSplitWarps == 6, "split_share's tables are written for six split warps");
 constexpr int kPairRows = 128;                      // rows of A and of B per CTA
 constexpr int kPairN = 256;                         // MMA N (= B columns per pair)
 constexpr int kPairStageBytes = 2 * kPairRows * kBK * 4;
@@ -614,6 +724,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   uint64_t* mma_done = bars + 3 * S + 4;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
+  uint64_t* split_local = bars + 3 * S + 8;  // peer CTA: its split warps -> its forwarder thread
+  uint64_t* acc_local = bars + 4 * S + 8;    // peer CTA: its epilogue warps -> its forwarder thread
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();
@@ -624,12 +736,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
       mbar_init(&full[s], 1);
-      mbar_init(&split_done[s], 2 * kPairSplitWarps);
+      mbar_init(&split_done[s], kPairSplitWarps + 1);   // the leader's split warps + the peer's forwarder
+      mbar_init(&split_local[s], kPairSplitWarps);
       mbar_init(&empty[s], 1);
     }
     for (int b = 0; b < 2; ++b) {
       mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 2 * kPairEpiWarps);
+      mbar_init(&acc_empty[b], kPairEpiWarps + 1);   // the leader's epilogue warps + the peer's forwarder
+      mbar_init(&acc_local[b], kPairEpiWarps);
     }
     mbar_init(mma_done, 1);
     *abort_flag = 0;
@@ -725,6 +839,37 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       tc_commit_pair(mapa_shared(smem_u32(mma_done), 0u));
       volatile int dummy = 0;
       mbar_wait(mma_done, 0, &dummy, args.status, 312);
+    } else if (rank == 1 && lane == 0) {
+      // ---- forwarder (peer CTA): each stage split here and each chunk drained here becomes
+      // one cluster-scope release-arrive on the leader's split_done / acc_empty.  The two
+      // streams interleave in an order that depends on timing, so both are polled.
+      const uint32_t sd_leader0 = mapa_shared(smem_u32(&split_done[0]), 0u);
+      const uint32_t ae_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0u);
+      const int total = ((ntiles - cid + ncl - 1) / ncl) * nc;   // (tile, chunk) iterations of this pair
+      int is = 0, ia = 0;
+      uint64_t t0 = globaltimer();
+      while ((is < total || ia < total) && !*abort_flag) {
+        bool moved = false;
+        if (is < total && mbar_test_wait(&split_local[is % S], (uint32_t)(is / S) & 1u)) {
+          mbar_arrive_cluster(sd_leader0 + (uint32_t)((is % S) * 8));
+          ++is;
+          moved = true;
+        }
+        if (ia < total && ia < is && mbar_test_wait(&acc_local[ia & 1], (uint32_t)(ia >> 1) & 1u)) {
+          mbar_arrive_cluster(ae_leader0 + (uint32_t)((ia & 1) * 8));
+          ++ia;
+          moved = true;
+        }
+        if (moved) {
+          t0 = globaltimer();
+        } else {
+          __nanosleep(32);   // leave the issue slots to the split and epilogue warps of this sub-partition
+          if (globaltimer() - t0 > kWaitLimitNs) {
+            *abort_flag = 1;
+            report_timeout(args.status, 313);
+          }
+        }
+      }
     }
   } else if (warp < kPairEpiWarp0) {
     // ------------------------------ split warps (both CTAs) ------------------------------
@@ -733,7 +878,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int sw = warp - 2;
     constexpr int kPairsA = kPairRows / 8, kPairsB = kPairRows / 8;
     static_assert(kPairEpiWarp0 == 2 + kPairSplitWarps, "split warps are warps 2 .. kPairEpiWarp0 - 1");
-    const uint32_t sd_leader0 = mapa_shared(smem_u32(&split_done[0]), 0u);
     int it = 0;
     bool ok = true;
     for (int tile = cid; tile < ntiles && ok; tile += ncl) {
@@ -747,7 +891,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         uint8_t* st = stages + s * kPairStageBytes;
         const int k0 = ch * kBK;
         constexpr int kLast = B_PRE ? kPairsA : kPairsA + kPairsB;
-        for (int t = sw; t < kLast; t += kPairSplitWarps) {
+        int t0, tn;
+        split_share(sw, kLast, t0, tn);
+        for (int t = t0; t < t0 + tn; ++t) {
           uint8_t *s0, *s1;
           int kboff;
           if (t < kPairsA) {
@@ -760,7 +906,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         fence_proxy_async_smem();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(sd_leader0 + (uint32_t)(s * 8));
+        // every split warp arrives on a barrier of its own CTA (a CTA-scope release): in the
+        // leader on split_done, which its MMA thread waits for; in the peer on split_local,
+        // which one thread forwards to the leader with a single cluster-scope release-arrive
+        // (that arrive costs several hundred cycles, off the split warps' path this way)
+        if (lane == 0) mbar_arrive(rank == 0 ? &split_done[s] : &split_local[s]);
       }
     }
   } else {
@@ -770,7 +920,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
     const int quarter = warp & 3;
     const int half = (warp - kPairEpiWarp0) >> 2;
     const int i_local = quarter * 32 + lane;
-    const uint32_t ae_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0u);
     float acc[128];
 #pragma unroll
     for (int t = 0; t < 128; ++t) acc[t] = 0.0f;
@@ -803,7 +952,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(ae_leader0 + (uint32_t)(b * 8));
+        if (lane == 0) mbar_arrive(rank == 0 ? &acc_empty[b] : &acc_local[b]);   // see the split warps
       }
       if (!ok) break;
       if (gi < args.Mk) {
@@ -907,6 +1056,9 @@ cudaError_t launch_variant(const CUtensorMap& a, const CUtensorMap& alo, const C
   }
   // programmatic dependent launch: the grid may start during the preceding kernel; every
   // role waits for it (griddepcontrol.wait) before touching data it may produce or read
+  if (args.chain)
+    return launch_pdl_cluster(kern, dim3(grid), dim3(Roles<BN>::kThreads), (size_t)smem, stream, args.chain, a, alo,
+                              b, blo, args);
   return launch_pdl(kern, dim3(grid), dim3(Roles<BN>::kThreads), (size_t)smem, stream, a, alo, b, blo, args);
 }
 
@@ -976,6 +1128,19 @@ cudaError_t launch_wide(bool b_mn, int fmt, const CUtensorMap& a, const CUtensor
 
 }  // namespace
 
+// CTAs per tile in chain mode: as many as the SMs allow for one wave of tiles (at most 8,
+// the portable cluster size, and at most one per chunk), provided each CTA's chunks fit in
+// TMEM as separate accumulators; 0 when no chain of at least two CTAs fits.
+int chain_size(int tiles, int nc, int BNk, int sms) {
+  if (BNk > 32 || tiles <= 0) return 0;
+  int S = sms / tiles;
+  if (S > 8) S = 8;
+  if (S > nc) S = nc;
+  if (S < 2) return 0;
+  if ((long long)((nc + S - 1) / S) * BNk > 512) return 0;
+  return S;
+}
+
 size_t gemm_workspace_bytes(int M, int N, int K, int tile_config) {
   if (tile_config != HEAL_TILE_SKINNY_SPLITK) return 0;
   const size_t nc = (size_t)((K + kBK - 1) / kBK);
@@ -987,16 +1152,19 @@ size_t gemm_workspace_bytes(int M, int N, int K, int tile_config) {
 heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, const void* B, long long ldb,
                           float* Cout, long long ldc, int fmt, const heal_gemm_opts_t& o, cudaStream_t stream) {
   int cfg = o.tile_config;
+  const int sms = device_sm_count();
+  if (sms <= 0) return HEAL_ERR_CUDA;
   if (cfg == HEAL_TILE_AUTO) {
+    const int bnk = M <= 16 ? 16 : 32;
     if (M <= 64 && o.workspace != nullptr && o.workspace_bytes >= gemm_workspace_bytes(M, N, K, HEAL_TILE_SKINNY_SPLITK))
       cfg = HEAL_TILE_SKINNY_SPLITK;
+    else if (M <= 32 && chain_size((N + kBM - 1) / kBM, (K + kBK - 1) / kBK, bnk, sms) >= 2)
+      cfg = HEAL_TILE_SKINNY_CHAIN;   // no workspace: K still spread over the SMs
     else if (M >= 256 && N >= 256)
       cfg = HEAL_TILE_256x256_PAIR;
     else
       cfg = HEAL_TILE_128x128;
   }
-  const int sms = device_sm_count();
-  if (sms <= 0) return HEAL_ERR_CUDA;
   const bool b_mn = (o.b_layout == 0);   // B stored K x N: N contiguous
   const int nc = (K + kBK - 1) / kBK;
   CUtensorMap ta{}, talo{}, tb{}, tblo{};
@@ -1046,6 +1214,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.expA_sign = -1;
     args.expB_sign = +1;
     args.static_op = o.b_static ? 2 : 0;   // kernel-B = B
+    args.tmem_cols = Cfg<BN>::kTmemCols;
     if (!operand_map(&ta, A, false, false, M, K, lda, kBM)) return HEAL_ERR_CUDA;
     if (!operand_map(&tb, B, b_mn, pre != 0, N, K, ldb, BN)) return HEAL_ERR_CUDA;
     if (pre == 1 && !operand_map(&tblo, o.b_lo, b_mn, true, N, K, ldb, BN)) return HEAL_ERR_CUDA;
@@ -1057,7 +1226,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     return err == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
   }
 
-  if (cfg == HEAL_TILE_SKINNY_SPLITK || cfg == HEAL_TILE_SKINNY_FULLK) {
+  if (cfg == HEAL_TILE_SKINNY_SPLITK || cfg == HEAL_TILE_SKINNY_FULLK || cfg == HEAL_TILE_SKINNY_CHAIN) {
     const bool split = (cfg == HEAL_TILE_SKINNY_SPLITK);
     if (M > 64) return HEAL_ERR_UNSUPPORTED;
     if (split && (o.workspace == nullptr || o.workspace_bytes < gemm_workspace_bytes(M, N, K, cfg)))
@@ -1076,11 +1245,21 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.expB_sign = -1;
     args.static_op = o.b_static ? 1 : 0;   // kernel-A = B^T
     const int BNk = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
+    args.tmem_cols = 2 * BNk < 32 ? 32 : 2 * BNk;
+    args.chain = 0;
+    const int S = cfg == HEAL_TILE_SKINNY_CHAIN ? chain_size(args.tiles_m, nc, BNk, sms) : 0;
+    if (S >= 2) {
+      args.chain = S;
+      const int per = (nc + S - 1) / S;
+      int cols = 32;
+      while (cols < per * BNk) cols *= 2;
+      args.tmem_cols = cols;
+    }
     if (!operand_map(&ta, B, b_mn, pre != 0, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (pre == 1 && !operand_map(&talo, o.b_lo, b_mn, true, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (!operand_map(&tb, A, false, false, M, K, lda, BNk)) return HEAL_ERR_CUDA;
     const long long units = split ? (long long)args.tiles_m * nc : (long long)args.tiles_m;
-    const int grid = (int)(units < sms ? units : sms);
+    const int grid = args.chain ? args.tiles_m * args.chain : (int)(units < sms ? units : sms);
     err = pre == 0 ? launch_skinny<0>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
         : pre == 1 ? launch_skinny<1>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
                    : launch_skinny<2>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);

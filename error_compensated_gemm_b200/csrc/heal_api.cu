@@ -125,7 +125,7 @@ heal_status_t heal_gemm_compensated(int M, int N, int K, const float* A, int64_t
   if (o.b_split_pass != 0 && o.b_split_pass != 1) return HEAL_ERR_INVALID_ARGUMENT;
   for (int r : o.reserved)
     if (r != 0) return HEAL_ERR_INVALID_ARGUMENT;
-  if (o.tile_config < HEAL_TILE_AUTO || o.tile_config > HEAL_TILE_SKINNY_FULLK) return HEAL_ERR_INVALID_ARGUMENT;
+  if (o.tile_config < HEAL_TILE_AUTO || o.tile_config > HEAL_TILE_SKINNY_CHAIN) return HEAL_ERR_INVALID_ARGUMENT;
   // TMA: 16-byte aligned bases, row strides multiples of 16 bytes
   if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 4)) return HEAL_ERR_INVALID_ARGUMENT;
   if (lda < K || lda % 4 != 0) return HEAL_ERR_INVALID_ARGUMENT;

@@ -37,6 +37,27 @@ cudaError_t launch_pdl(void (*kern)(Params...), dim3 grid, dim3 block, size_t sm
   return cudaLaunchKernelEx(&cfg, kern, static_cast<Params>(args)...);
 }
 
+// The same with a 1-D cluster of `cluster` CTAs (grid.x a multiple of it).
+template <typename... Params, typename... Args>
+cudaError_t launch_pdl_cluster(void (*kern)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+                               int cluster, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = (unsigned)cluster;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<Params>(args)...);
+}
+
 heal_status_t split_launch(const float* x, void* hi, void* lo, long long n, int fmt, cudaStream_t s);
 
 size_t gemm_workspace_bytes(int M, int N, int K, int tile_config);

@@ -61,7 +61,14 @@ enum {
                                  B; the default for M, N >= 256                           */
   HEAL_TILE_SKINNY_SPLITK = 2, /* operands swapped (weights on the MMA M side), K split
                                  over CTAs; needs a workspace (M <= 64)                 */
-  HEAL_TILE_SKINNY_FULLK = 3   /* operands swapped, full K per CTA, no workspace (M <= 64) */
+  HEAL_TILE_SKINNY_FULLK = 3,  /* operands swapped, full K per CTA, no workspace (M <= 64) */
+  HEAL_TILE_SKINNY_CHAIN = 4   /* operands swapped, K split over a cluster of 2-8 CTAs per
+                                 128-row tile of C^T; each CTA keeps its chunks in TMEM and
+                                 the running sum passes from CTA to CTA in ascending chunk
+                                 order through distributed shared memory; no workspace.
+                                 M <= 32; other shapes (or too few SMs for two CTAs per
+                                 tile) run HEAL_TILE_SKINNY_FULLK.  The automatic choice
+                                 for M <= 32 when no workspace is given                   */
 };
 
 typedef struct {

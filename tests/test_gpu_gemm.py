@@ -95,9 +95,11 @@ def test_tile_configs_bitwise_identical(M, b_layout):
     c_skinny = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_SKINNY_SPLITK)
     c_fullk = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_SKINNY_FULLK)
     c_pair = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_256x256_PAIR)
+    c_chain = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_SKINNY_CHAIN)
     assert np.array_equal(c_full, c_skinny)
     assert np.array_equal(c_full, c_fullk)
     assert np.array_equal(c_full, c_pair)
+    assert np.array_equal(c_full, c_chain)
     assert G.normwise_rel_err(c_full, G.gemm_ref(X, W)) <= TOL_FP16
 
 
@@ -131,7 +133,7 @@ def test_skinny_presplit_weights_bitwise(M, b_layout, fmt):
     lo = torch.empty(B_d.shape, dtype=torch.int16, device=d)
     heal.heal_split(B_d, hi, lo, fmt)
     c_ref = gemm(X.numpy(), Bin.numpy(), fmt=fmt, b_layout=b_layout, tile=heal.TILE_128x128)
-    for tile in (heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK, heal.TILE_AUTO):
+    for tile in (heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK, heal.TILE_SKINNY_CHAIN, heal.TILE_AUTO):
         c_pre = gemm(X.numpy(), hi, fmt=fmt, b_layout=b_layout, tile=tile, b_lo=lo)
         assert np.array_equal(c_pre, c_ref), tile
 
@@ -164,9 +166,23 @@ def test_non_contiguous_output_leading_dimension():
 def test_decode_shapes_full_oracle(M):
     X, W = synthetic.gemm_decode(M)
     X, W = X.numpy(), W.numpy()
-    C = gemm(X, W)            # automatic config (skinny split-K)
+    C = gemm(X, W)            # automatic config
     assert G.normwise_rel_err(C, G.gemm_ref(X, W)) <= TOL_FP16
     assert_elementwise(C, X, W)
+    for tile in (heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_CHAIN, heal.TILE_SKINNY_FULLK):
+        assert np.array_equal(gemm(X, W, tile=tile), C), tile
+
+
+@pytest.mark.parametrize("M,K,N", [(8, 1000, 5120), (1, 520, 8192), (3, 4096, 640), (32, 1500, 1000)])
+def test_chain_split_over_uneven_cta_runs(M, K, N):
+    """Chain mode with 2, 3 and 8 CTAs per tile and chunk runs of unequal length (K not a
+    multiple of the chain): the running sum handed from CTA to CTA gives the single-CTA bits."""
+    X, W = synthetic.gemm_decode(M, K=K, N=N)
+    X, W = X.numpy(), W.numpy()
+    c_chain = gemm(X, W, tile=heal.TILE_SKINNY_CHAIN)
+    c_ref = gemm(X, W, tile=heal.TILE_128x128)
+    assert np.array_equal(c_chain, c_ref)
+    assert G.normwise_rel_err(c_chain, G.gemm_ref(X, W)) <= TOL_FP16
 
 
 def test_prefill_full_size_sampled_rows():
@@ -218,7 +234,8 @@ def test_cta_pair_presplit_and_bf16(fmt):
 
 @pytest.mark.parametrize("M", [1, 8, 64, 300])
 @pytest.mark.parametrize("presplit", [False, True])
-def test_back_to_back_dependent_chain(M, presplit):
+@pytest.mark.parametrize("tile", [heal.TILE_AUTO, heal.TILE_SKINNY_CHAIN])
+def test_back_to_back_dependent_chain(M, presplit, tile):
     """Programmatic dependent launch: each call's A is the previous call's C and all calls
     share one workspace, issued back to back with weights declared static.  The chain must
     give the bits of the same calls separated by a device synchronisation."""
@@ -240,10 +257,12 @@ def test_back_to_back_dependent_chain(M, presplit):
         a = X
         for i, W in enumerate(Ws):
             c = torch.full((M, N), float("nan"), device=d)
+            t = tile if M <= 64 else heal.TILE_AUTO
             if presplit:
-                heal.heal_gemm_compensated(a, pre[i][0], c, b_lo=pre[i][1], workspace=use_ws, b_static=True)
+                heal.heal_gemm_compensated(a, pre[i][0], c, b_lo=pre[i][1], workspace=use_ws, b_static=True,
+                                           tile_config=t)
             else:
-                heal.heal_gemm_compensated(a, W, c, workspace=use_ws, b_static=True)
+                heal.heal_gemm_compensated(a, W, c, workspace=use_ws, b_static=True, tile_config=t)
             if sync:
                 torch.cuda.synchronize()
             outs.append(c)
@@ -290,7 +309,7 @@ def test_two_product_16bit_weights(fmt, b_layout, M):
     ref = G.gemm_ref(X.numpy(), W16.float().numpy())
     Bin = W16 if b_layout == 0 else W16.t().contiguous()
     tiles = [heal.TILE_128x128, heal.TILE_256x256_PAIR] + (
-        [heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK] if M <= 64 else [])
+        [heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK, heal.TILE_SKINNY_CHAIN] if M <= 64 else [])
     outs = [_gemm16(X, Bin, fmt, t, b_layout) for t in tiles]
     for o in outs[1:]:
         assert np.array_equal(o, outs[0])
@@ -302,8 +321,9 @@ def test_two_product_16bit_weights(fmt, b_layout, M):
     assert G.normwise_rel_err(outs[0], emu) <= (5e-7 if fmt == heal.SPLIT_FP16_S11 else 2e-5)
 
 
-@pytest.mark.parametrize("M", [1, 8, 64, 256])
-def test_graph_replay_with_new_inputs(M):
+@pytest.mark.parametrize("M,tile", [(1, heal.TILE_AUTO), (8, heal.TILE_AUTO), (64, heal.TILE_AUTO),
+                                    (256, heal.TILE_AUTO), (1, heal.TILE_SKINNY_CHAIN), (8, heal.TILE_SKINNY_CHAIN)])
+def test_graph_replay_with_new_inputs(M, tile):
     """A GEMM captured once in a CUDA graph and replayed after its input buffer was rewritten
     gives, at every replay, the bits of an eager call on the new input (nothing of an earlier
     launch may stand in for this one's data)."""
@@ -315,12 +335,12 @@ def test_graph_replay_with_new_inputs(M):
     ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(M, N, K, heal.TILE_SKINNY_SPLITK) // 4), device=d)
     use_ws = ws if M <= 64 else None
     X.copy_(synthetic.normal((M, K), seed=50).to(d))
-    heal.heal_gemm_compensated(X, W, C, workspace=use_ws, b_static=True)
+    heal.heal_gemm_compensated(X, W, C, workspace=use_ws, b_static=True, tile_config=tile)
     torch.cuda.synchronize()
     s = torch.cuda.Stream()
     g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g, stream=s):
-        heal.heal_gemm_compensated(X, W, C, workspace=use_ws, b_static=True)
+        heal.heal_gemm_compensated(X, W, C, workspace=use_ws, b_static=True, tile_config=tile)
     for seed in (51, 52, 53):
         X.copy_(synthetic.normal((M, K), seed=seed).to(d))
         g.replay()
@@ -379,7 +399,7 @@ def test_two_product_with_outlier_channel_rescale(M, b_layout):
     d = dev()
     ce = torch.as_tensor(e).to(d)
     tiles = [heal.TILE_128x128, heal.TILE_256x256_PAIR] + (
-        [heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK] if M <= 64 else [])
+        [heal.TILE_SKINNY_SPLITK, heal.TILE_SKINNY_FULLK, heal.TILE_SKINNY_CHAIN] if M <= 64 else [])
     outs = []
     for t in tiles:
         Xd, Wd = X.to(d).contiguous(), Bin.to(d).contiguous()
@@ -430,3 +450,17 @@ def test_column_shards_reassemble_bitwise():
         heal.heal_gemm_compensated(Xd[m0:m1], Wd, C[m0:m1])
     status_ok()
     assert torch.equal(C.view(torch.int32), full.view(torch.int32))
+
+
+@pytest.mark.parametrize("M", [1, 8, 32, 40])
+def test_auto_without_workspace_small_m(M):
+    """With no workspace the automatic choice for M <= 32 is the chain mode (K spread over a
+    cluster of CTAs per tile); it must give the single-CTA bits, as must M = 40 (128 x 128)."""
+    d = dev()
+    X, W = synthetic.gemm_decode(M, K=2048, N=3072)
+    Xd, Wd = X.to(d), W.to(d)
+    C = torch.full((M, 3072), float("nan"), device=d)
+    heal.heal_gemm_compensated(Xd, Wd, C)
+    status_ok()
+    ref = gemm(X.numpy(), W.numpy(), tile=heal.TILE_128x128)
+    assert np.array_equal(to_np(C).astype(np.float64), ref)
