@@ -841,8 +841,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       mbar_wait(mma_done, 0, &dummy, args.status, 312);
     } else if (rank == 1 && lane == 0) {
       // ---- forwarder (peer CTA): each stage split here and each chunk drained here becomes
-      // one cluster-scope release-arrive on the leader's split_done / acc_empty.  The two
-      // streams interleave in an order that depends on timing, so both are polled.
+      // one arrive on the leader's split_done / acc_empty.  The two streams interleave in an
+      // order that depends on timing, so both are polled.
       const uint32_t sd_leader0 = mapa_shared(smem_u32(&split_done[0]), 0u);
       const uint32_t ae_leader0 = mapa_shared(smem_u32(&acc_empty[0]), 0u);
       const int total = ((ntiles - cid + ncl - 1) / ncl) * nc;   // (tile, chunk) iterations of this pair
@@ -851,12 +851,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
       while ((is < total || ia < total) && !*abort_flag) {
         bool moved = false;
         if (is < total && mbar_test_wait(&split_local[is % S], (uint32_t)(is / S) & 1u)) {
-          mbar_arrive_cluster(sd_leader0 + (uint32_t)((is % S) * 8));
+          // release at CTA scope (mbarrier.arrive's default): this thread's acquire of the
+          // six local arrivals, each after its warp's split stores into this CTA's shared
+          // memory and fence.proxy.async, is ordered before the arrive the leader's MMA thread
+          // acquires.  A cluster-scope release costs ~1000 cycles here, CTA scope ~20.
+          mbar_arrive_remote(sd_leader0 + (uint32_t)((is % S) * 8));
           ++is;
           moved = true;
         }
         if (ia < total && ia < is && mbar_test_wait(&acc_local[ia & 1], (uint32_t)(ia >> 1) & 1u)) {
-          mbar_arrive_cluster(ae_leader0 + (uint32_t)((ia & 1) * 8));
+          // TMEM reuse only (the drains' tcgen05.ld completed before their tcgen05 fence and
+          // arrive; the MMA thread fences after its wait): no data to publish, no release
+          mbar_arrive_cluster_relaxed(ae_leader0 + (uint32_t)((ia & 1) * 8));
           ++ia;
           moved = true;
         }
@@ -908,8 +914,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         __syncwarp();
         // every split warp arrives on a barrier of its own CTA (a CTA-scope release): in the
         // leader on split_done, which its MMA thread waits for; in the peer on split_local,
-        // which one thread forwards to the leader with a single cluster-scope release-arrive
-        // (that arrive costs several hundred cycles, off the split warps' path this way)
+        // which one thread forwards to the leader (fewer arrivals crossing the cluster than
+        // six remote ones per stage, and measured ~2% faster)
         if (lane == 0) mbar_arrive(rank == 0 ? &split_done[s] : &split_local[s]);
       }
     }
