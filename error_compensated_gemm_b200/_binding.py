@@ -6,6 +6,10 @@ import os
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(HERE, "libheal.so")
+# The same kernels built with HEAL_DEBUG: every global store index they compute is checked
+# and a violation is reported by heal_get_device_status() instead of faulting.  A process
+# selects it with use_debug_library() before its first call.
+DEBUG_LIB_PATH = os.path.join(HERE, "libheal_debug.so")
 
 HEAL_OK, HEAL_ERR_INVALID_ARGUMENT, HEAL_ERR_UNSUPPORTED, HEAL_ERR_CUDA, HEAL_ERR_TIMEOUT = range(5)
 SPLIT_FP16_S11, SPLIT_BF16 = 0, 1
@@ -35,6 +39,14 @@ class GemmOpts(ctypes.Structure):
 
 _lib = None
 _vp, _i, _i64, _f, _sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+
+
+def use_debug_library():
+    """Make this process load libheal_debug.so instead of libheal.so (before the first call)."""
+    global LIB_PATH
+    if _lib is not None:
+        raise RuntimeError("the library is already loaded in this process")
+    LIB_PATH = DEBUG_LIB_PATH
 
 
 def lib():

@@ -32,8 +32,17 @@ def _needs(obj, src, deps):
     return any(os.path.getmtime(p) > t for p in [src] + deps)
 
 
-def build(verbose=False, jobs=None):
-    os.makedirs(BUILD, exist_ok=True)
+DEBUG_LIB = os.path.join(HERE, "libheal_debug.so")
+
+
+def build(verbose=False, jobs=None, debug=False):
+    """debug=True builds libheal_debug.so: the same sources with HEAL_DEBUG defined, whose
+    kernels check every global store index and TMA coordinate they compute and record a
+    violation in the device status word (HEAL_ERR_INVALID_ARGUMENT) instead of faulting."""
+    build_dir = os.path.join(BUILD, "debug") if debug else BUILD
+    lib = DEBUG_LIB if debug else LIB
+    flags = FLAGS + (["-DHEAL_DEBUG=1"] if debug else [])
+    os.makedirs(build_dir, exist_ok=True)
     srcs = sorted(f for f in os.listdir(CSRC) if f.endswith(".cu"))
     deps = [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))]
     deps.append(os.path.join(ROOT, "include", "heal.h"))
@@ -42,10 +51,10 @@ def build(verbose=False, jobs=None):
     cmds = []
     for f in srcs:
         src = os.path.join(CSRC, f)
-        obj = os.path.join(BUILD, f[:-3] + ".o")
+        obj = os.path.join(build_dir, f[:-3] + ".o")
         objs.append(obj)
         if _needs(obj, src, deps):
-            cmds.append([cc] + ARCH + FLAGS + ["-c", src, "-o", obj])
+            cmds.append([cc] + ARCH + flags + ["-c", src, "-o", obj])
 
     def run(cmd):
         r = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,10 +65,10 @@ def build(verbose=False, jobs=None):
 
     with concurrent.futures.ThreadPoolExecutor(max_workers=jobs or os.cpu_count() or 4) as ex:
         list(ex.map(run, cmds))
-    if cmds or not os.path.exists(LIB) or any(os.path.getmtime(o) > os.path.getmtime(LIB) for o in objs):
-        run([cc] + ARCH + ["-shared", "-cudart", "static", "-o", LIB] + objs)
-    return LIB
+    if cmds or not os.path.exists(lib) or any(os.path.getmtime(o) > os.path.getmtime(lib) for o in objs):
+        run([cc] + ARCH + ["-shared", "-cudart", "static", "-o", lib] + objs)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(verbose="-v" in sys.argv))
+    print(build(verbose="-v" in sys.argv, debug="--debug" in sys.argv))

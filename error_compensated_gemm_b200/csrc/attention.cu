@@ -68,6 +68,7 @@ struct AttnArgs {
   long long total;  // B*Hkv*nblk
   int grid;
   unsigned int* status;
+  long long ws_elems;   // FP32 elements of the workspace (debug-build checks)
 };
 
 // -------- INT16 byte split into FP16 pairs (bit construction, exact) --------
@@ -295,8 +296,10 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
         float L = 0.0f;
         for (int ww = 0; ww < kQK; ++ww) L = __fadd_rn(L, lsum[ww * kRows + lane]);
         float* sl = slot_ptr(a.ws, c, p, R, D) + R * D;
-        sl[2 * lane] = mq[lane];
-        sl[2 * lane + 1] = L;
+        if (HEAL_DCHECK((long long)(sl + 2 * lane + 1 - a.ws) < a.ws_elems, a.status, 250)) {
+          sl[2 * lane] = mq[lane];
+          sl[2 * lane + 1] = L;
+        }
       }
     };
 
@@ -424,7 +427,9 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
             xv = __fmul_rn(lg, kLog2e);
             if (a.qk_out) {
               const int tq = r / a.G, gq = r % a.G;
-              a.qk_out[((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq) * a.Tmax + t] = S;
+              const long long qi = ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq) * a.Tmax + t;
+              if (HEAL_DCHECK(qi < (long long)a.B * a.Hq * a.Tq * a.Tmax && t < a.Tmax, a.status, 251))
+                a.qk_out[qi] = S;
             }
           }
           x[th][e] = xv;
@@ -566,7 +571,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
       for (int e = 0; e < 4; ++e) {
         const int d = (v * kDT + dl) * 16 + g8 + ((e >> 1) << 3);
         const int r = qc + (e & 1);
-        if (r < R) sl[r * D + d] = mul_pow2(om[dl][e], -E_run);   // true units (x 2^-E_run)
+        if (r < R && HEAL_DCHECK((long long)(sl + r * D + d - a.ws) < a.ws_elems, a.status, 252))
+          sl[r * D + d] = mul_pow2(om[dl][e], -E_run);   // true units (x 2^-E_run)
         om[dl][e] = 0.0f;
       }
   };
@@ -689,7 +695,8 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
   const int b = p / a.Hkv, hkv = p % a.Hkv;
   const int tq = r / a.G, g = r % a.G;
   // a query with no visible token (causal, kv_len < Tq) gets zeros
-  a.out[(((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq) * D) + d] = L > 0.0f ? __fdiv_rn(O, L) : 0.0f;
+  const long long oi = (((long long)(b * a.Hq + hkv * a.G + g) * a.Tq + tq) * D) + d;
+  if (HEAL_DCHECK(oi < (long long)a.B * a.Hq * a.Tq * D, a.status, 253)) a.out[oi] = L > 0.0f ? __fdiv_rn(O, L) : 0.0f;
 }
 
 template <int D>
@@ -769,6 +776,7 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   if (grid > a.total) grid = a.total;
   a.grid = (int)grid;
   a.status = device_status_ptr();
+  a.ws_elems = (long long)(ws_bytes / sizeof(float));
   if ((size_t)(a.grid + (long long)B * Hkv) * (size_t)R * (size_t)(D + 2) * sizeof(float) > ws_bytes)
     return HEAL_ERR_INVALID_ARGUMENT;
 

@@ -122,7 +122,21 @@ struct PlanesArgs {
   long long nk8;          // K/V elements / 8
   long long nq8;          // Q elements / 8
   int B, Hkv, Tmax;
+  const uint8_t* ws;      // workspace base and size (debug-build checks of the plane writes)
+  long long ws_bytes;
+  unsigned int* status;
 };
+
+// debug builds: the byte range [p, p + n) lies inside the workspace
+__device__ __forceinline__ bool in_ws(const PlanesArgs& a, const void* p, long long n, int site) {
+#ifdef HEAL_DEBUG
+  const long long off = (long long)(reinterpret_cast<const uint8_t*>(p) - a.ws);
+  return debug_check(off >= 0 && off + n <= a.ws_bytes, a.status, site);
+#else
+  (void)a, (void)p, (void)n, (void)site;
+  return true;
+#endif
+}
 
 // x * 2^e exactly for |e| <= 252 (two steps, each a normal power of two).
 __device__ __forceinline__ float mul_pow2_p(float x, int e) {
@@ -161,8 +175,10 @@ __global__ void __launch_bounds__(256) heal_attn_planes_kernel(const PlanesArgs 
     for (long long i = tid; i < a.nk8; i += stride) {
       uint2 h, l;
       bytes8(__ldg(src + i), h, l);
-      dh[i] = h;
-      dl[i] = l;
+      if (in_ws(a, dh + i, 8, 270) && in_ws(a, dl + i, 8, 271)) {
+        dh[i] = h;
+        dl[i] = l;
+      }
     }
   } else if (blockIdx.y == 1) {
     const uint4* src = reinterpret_cast<const uint4*>(a.v);
@@ -175,8 +191,10 @@ __global__ void __launch_bounds__(256) heal_attn_planes_kernel(const PlanesArgs 
       vparts2(w.y, h.y, l.y);
       vparts2(w.z, h.z, l.z);
       vparts2(w.w, h.w, l.w);
-      dh[i] = h;
-      dl[i] = l;
+      if (in_ws(a, dh + i, 16, 272) && in_ws(a, dl + i, 16, 273)) {
+        dh[i] = h;
+        dl[i] = l;
+      }
     }
   } else if (blockIdx.y == 2) {
     const uint4* src = reinterpret_cast<const uint4*>(a.q);
@@ -185,8 +203,10 @@ __global__ void __launch_bounds__(256) heal_attn_planes_kernel(const PlanesArgs 
     for (long long i = tid; i < a.nq8; i += stride) {
       uint2 h, l;
       bytes8(__ldg(src + i), h, l);
-      dh[i] = h;
-      dl[i] = l;
+      if (in_ws(a, dh + i, 8, 274) && in_ws(a, dl + i, 8, 275)) {
+        dh[i] = h;
+        dl[i] = l;
+      }
     }
   } else {
     // E of (b, hkv) = blockIdx.x: the largest V scale of the visible tokens times 2^E in
@@ -209,12 +229,13 @@ __global__ void __launch_bounds__(256) heal_attn_planes_kernel(const PlanesArgs 
       for (int w = 0; w < (int)(blockDim.x >> 5); ++w) m = max(m, wmax[w]);
       const float smax = __uint_as_float(m);
       e_sh = (smax > 0.0f) ? 5 - ilogbf(smax) : 0;
-      a.E[p] = e_sh;
+      if (in_ws(a, a.E + p, 4, 276)) a.E[p] = e_sh;
     }
     __syncthreads();
     const int E = e_sh;
     float* cv = a.cv + (long long)p * a.Tmax;
-    for (int t = threadIdx.x; t < a.Tmax; t += blockDim.x) cv[t] = t < klen ? mul_pow2_p(__ldg(s + t), E) : 0.0f;
+    for (int t = threadIdx.x; t < a.Tmax; t += blockDim.x)
+      if (in_ws(a, cv + t, 4, 277)) cv[t] = t < klen ? mul_pow2_p(__ldg(s + t), E) : 0.0f;
   }
 }
 
@@ -523,7 +544,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
               if (!vis) xv = -INFINITY;
             }
             if constexpr (kHook) {
-              if (vis && qk_row) qk_row[t] = (long long)(int)rh[i] * 65536LL + (long long)low;
+              if (vis && qk_row && HEAL_DCHECK(t < a.Tmax && (long long)bh * a.Tq + tq < (long long)a.B * a.Hq * a.Tq,
+                                               a.status, 278))
+                qk_row[t] = (long long)(int)rh[i] * 65536LL + (long long)low;
             }
             x[q8 * 8 + i] = xv;
           }
@@ -630,6 +653,9 @@ __global__ void __launch_bounds__(kPThreads, 1)
 #pragma unroll
     for (int gi = 1; gi < kGroups; ++gi) L = __fadd_rn(L, lsm[gi * kPM + r]);
     float* dst = real ? a.out + ((long long)bh * a.Tq + tq) * kPD + hf * kOCols : nullptr;
+    if (dst && !HEAL_DCHECK(((long long)bh * a.Tq + tq) * kPD + (hf + 1) * kOCols <= (long long)a.B * a.Hq * a.Tq * kPD,
+                            a.status, 279))
+      dst = nullptr;
     if (ok && nb > 0) {
       if (dst) {
         float4* d4 = reinterpret_cast<float4*>(dst);
@@ -699,6 +725,9 @@ heal_status_t attention_prefill_launch(const int16_t* q, const float* qs, const 
   pa.B = B;
   pa.Hkv = Hkv;
   pa.Tmax = Tmax;
+  pa.ws = w;
+  pa.ws_bytes = (long long)ws_bytes;
+  pa.status = device_status_ptr();
 
   PrefillArgs a{};
   a.qs = qs;

@@ -71,6 +71,8 @@ struct GemmArgs {
   int static_op;            // 0: none; 1: kernel-A, 2: kernel-B is not written by the kernels
                             // before this one (its first stages may be requested early)
   unsigned int* status;     // device status word
+  long long out_extent;     // elements of `out` the call may write (debug-build checks)
+  long long ws_elems;       // FP32 elements of the workspace (debug-build checks)
 };
 
 template <int BN>
@@ -560,7 +562,8 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
 #pragma unroll
             for (int t = 0; t < BN; ++t) {
               const int gj = tn * BN + t;
-              if (gj < args.Nk) args.out[(size_t)gi * args.out_si + (size_t)gj * args.out_sj] = acc[t];
+              const long long o = (long long)gi * args.out_si + (long long)gj * args.out_sj;
+              if (gj < args.Nk && HEAL_DCHECK(o < args.out_extent, args.status, 150)) args.out[o] = acc[t];
             }
           }
         }
@@ -605,7 +608,9 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
               const int gj = tn * BN + c * 16 + t;
-              if (gj < args.Nk) wsc[(size_t)gj * args.Mk + gi] = __uint_as_float(r[t]);
+              if (gj < args.Nk &&
+                  HEAL_DCHECK(((long long)w.chunk * args.Nk + gj) * args.Mk + gi < args.ws_elems, args.status, 151))
+                wsc[(size_t)gj * args.Mk + gi] = __uint_as_float(r[t]);
             }
           }
         }
@@ -621,16 +626,22 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
           if (vec) {
 #pragma unroll
             for (int t = 0; t < BN; t += 4)
-              *reinterpret_cast<float4*>(orow + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
+              if (HEAL_DCHECK((long long)gi * args.out_si + gj0 + t + 3 < args.out_extent, args.status, 152))
+                *reinterpret_cast<float4*>(orow + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
           } else {
 #pragma unroll
             for (int t = 0; t < BN; ++t)
-              if (gj0 + t < args.Nk) orow[t] = acc[t];
+              if (gj0 + t < args.Nk &&
+                  HEAL_DCHECK((long long)gi * args.out_si + gj0 + t < args.out_extent, args.status, 153))
+                orow[t] = acc[t];
           }
         } else {
 #pragma unroll
           for (int t = 0; t < BN; ++t)
-            if (gj0 + t < args.Nk) args.out[(size_t)gi * args.out_si + (size_t)(gj0 + t) * args.out_sj] = acc[t];
+            if (gj0 + t < args.Nk) {
+              const long long o = (long long)gi * args.out_si + (long long)(gj0 + t) * args.out_sj;
+              if (HEAL_DCHECK(o < args.out_extent, args.status, 154)) args.out[o] = acc[t];
+            }
         }
       }
     }
@@ -967,11 +978,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
         if (((reinterpret_cast<uintptr_t>(orow) & 15) == 0) && (gj0 + 128 <= args.Nk)) {
 #pragma unroll
           for (int t = 0; t < 128; t += 4)
-            *reinterpret_cast<float4*>(orow + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
+            if (HEAL_DCHECK((long long)gi * args.out_si + gj0 + t + 3 < args.out_extent, args.status, 350))
+              *reinterpret_cast<float4*>(orow + t) = make_float4(acc[t], acc[t + 1], acc[t + 2], acc[t + 3]);
         } else {
 #pragma unroll
           for (int t = 0; t < 128; ++t)
-            if (gj0 + t < args.Nk) orow[t] = acc[t];
+            if (gj0 + t < args.Nk &&
+                HEAL_DCHECK((long long)gi * args.out_si + gj0 + t < args.out_extent, args.status, 351))
+              orow[t] = acc[t];
         }
       }
     }
@@ -993,7 +1007,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 // GEMM's CTAs can start next to them.
 constexpr int kRedBatch = 32;
 __global__ void __launch_bounds__(256) heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk,
-                                                                int Nk, float* out, long long si, long long sj) {
+                                                                int Nk, float* out, long long si, long long sj,
+                                                                long long out_extent, unsigned int* status) {
   pdl_launch_dependents();   // the next kernel may be scheduled; it waits for this grid
   pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed
   const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
@@ -1011,7 +1026,8 @@ __global__ void __launch_bounds__(256) heal_chunk_reduce_kernel(const float* __r
     for (int t = 0; t < kRedBatch; ++t)
       if (t < cn) acc = (c0 + t == 0) ? v[t] : __fadd_rn(acc, v[t]);
   }
-  out[(size_t)i * si + (size_t)j * sj] = acc;
+  const long long o = (long long)i * si + (long long)j * sj;
+  if (HEAL_DCHECK(o < out_extent, status, 160)) out[o] = acc;
 }
 
 // ---------------------------------------------------------------------------------
@@ -1181,6 +1197,8 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
   args.static_op = 0;
   const int pre = o.b_presplit;   // 0 FP32 B, 1 pre-split hi + lo, 2 16-bit B (two products)
   args.status = device_status_ptr();
+  args.out_extent = (long long)(M - 1) * ldc + N;   // C is M x N with row stride ldc in every config
+  args.ws_elems = o.workspace ? (long long)(o.workspace_bytes / sizeof(float)) : 0;
   cudaError_t err = cudaSuccess;
 
   if (cfg == HEAL_TILE_256x256_PAIR) {
@@ -1274,7 +1292,8 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     const long long rblocks = ((long long)N * M + 255) / 256;
     if (rblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
     const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(256), 0, stream,
-                                     (const float*)args.ws, nc, N, M, Cout, 1LL, (long long)ldc);
+                                     (const float*)args.ws, nc, N, M, Cout, 1LL, (long long)ldc, args.out_extent,
+                                     args.status);
     return e == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
   }
   return HEAL_ERR_UNSUPPORTED;

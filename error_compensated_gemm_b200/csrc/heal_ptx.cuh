@@ -23,6 +23,21 @@ __device__ __forceinline__ void report_timeout(unsigned int* status, int site) {
   if (status != nullptr && atomicOr(&status[0], kStatusTimeout) == 0u) status[1] = (unsigned int)site;
 }
 
+// Debug builds (HEAL_DEBUG, libheal_debug.so): every global store index and TMA
+// coordinate a kernel computes is checked against the extent it must stay in; a failed
+// check records kStatusBadInput and the site in the status word and the access is skipped,
+// so a wrong index shows up in heal_get_device_status() (HEAL_ERR_INVALID_ARGUMENT) instead
+// of as a fault.  In the normal build HEAL_DCHECK is the constant true and costs nothing.
+__device__ __forceinline__ bool debug_check(bool ok, unsigned int* status, int site) {
+  if (!ok && status != nullptr && atomicOr(&status[0], kStatusBadInput) == 0u) status[1] = (unsigned int)site;
+  return ok;
+}
+#ifdef HEAL_DEBUG
+#define HEAL_DCHECK(cond, status, site) ::heal::debug_check((cond), (status), (site))
+#else
+#define HEAL_DCHECK(cond, status, site) true
+#endif
+
 __device__ __forceinline__ uint64_t globaltimer() {
   uint64_t t;
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));

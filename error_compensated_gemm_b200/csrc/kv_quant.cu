@@ -22,7 +22,7 @@ template <int L, bool BF16>
 __global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restrict__ x, int B, int T, int H,
                                                             long long sb, long long st, long long sh,
                                                             int16_t* __restrict__ q, float* __restrict__ sc,
-                                                            int Tmax, int t_off) {
+                                                            int Tmax, int t_off, unsigned int* status) {
   // programmatic dependent launch: the next kernel may be scheduled now; the preceding one
   // (which may write x or read the cache) finishes before the first global access here
   pdl_launch_dependents();
@@ -109,8 +109,10 @@ __global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restri
         pk.y = (uint32_t)(qv[2] & 0xFFFF) | ((uint32_t)qv[3] << 16);
         pk.z = (uint32_t)(qv[4] & 0xFFFF) | ((uint32_t)qv[5] << 16);
         pk.w = (uint32_t)(qv[6] & 0xFFFF) | ((uint32_t)qv[7] << 16);
-        __stcs(reinterpret_cast<uint4*>(q + row_out * D + sub * 8), pk);
-        if (sub == 0) sc[row_out] = m > 0.0f ? __fdiv_rn(m, 32767.0f) : 0.0f;
+        if (HEAL_DCHECK(row_out < (long long)B * H * Tmax && t_off + t < Tmax && h < H, status, 400)) {
+          __stcs(reinterpret_cast<uint4*>(q + row_out * D + sub * 8), pk);
+          if (sub == 0) sc[row_out] = m > 0.0f ? __fdiv_rn(m, 32767.0f) : 0.0f;
+        }
       }
     }
   }
@@ -121,9 +123,9 @@ static cudaError_t launch_L(const void* x, int bf16, int B, int T, int H, long l
                             int16_t* q, float* sc, int Tmax, int t_off, int grid, cudaStream_t s) {
   if (bf16)
     return launch_pdl(heal_kv_quant_kernel<L, true>, dim3(grid), dim3(256), 0, s, x, B, T, H, sb, st, sh, q, sc, Tmax,
-                      t_off);
+                      t_off, device_status_ptr());
   return launch_pdl(heal_kv_quant_kernel<L, false>, dim3(grid), dim3(256), 0, s, x, B, T, H, sb, st, sh, q, sc, Tmax,
-                    t_off);
+                    t_off, device_status_ptr());
 }
 
 heal_status_t kv_quant_launch(const void* x, int is_bf16, int B, int T, int H, int D, long long sb, long long st,

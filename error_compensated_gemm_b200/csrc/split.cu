@@ -9,7 +9,8 @@ namespace heal {
 
 template <int FMT>
 __global__ void __launch_bounds__(256) heal_split_kernel(const float* __restrict__ x, uint16_t* __restrict__ hi,
-                                                         uint16_t* __restrict__ lo, long long n, int vec) {
+                                                         uint16_t* __restrict__ lo, long long n, int vec,
+                                                         unsigned int* status) {
   pdl_launch_dependents();   // programmatic dependent launch: see the launch below
   pdl_wait_prerequisites();  // x may come from the preceding kernel
   const long long stride = (long long)gridDim.x * blockDim.x;
@@ -26,16 +27,20 @@ __global__ void __launch_bounds__(256) heal_split_kernel(const float* __restrict
       h.y = split2<FMT>(a.z, a.w, l.y);
       h.z = split2<FMT>(b.x, b.y, l.z);
       h.w = split2<FMT>(b.z, b.w, l.w);
-      __stcs(reinterpret_cast<uint4*>(hi) + v, h);
-      __stcs(reinterpret_cast<uint4*>(lo) + v, l);
+      if (HEAL_DCHECK(8 * v + 8 <= n, status, 410)) {
+        __stcs(reinterpret_cast<uint4*>(hi) + v, h);
+        __stcs(reinterpret_cast<uint4*>(lo) + v, l);
+      }
     }
     tail = n8 << 3;
   }
   for (long long i = tail + gid; i < n; i += stride) {
     uint32_t l;
     const uint32_t h = split2<FMT>(x[i], 0.0f, l);
-    hi[i] = (uint16_t)(h & 0xFFFFu);
-    lo[i] = (uint16_t)(l & 0xFFFFu);
+    if (HEAL_DCHECK(i < n, status, 411)) {
+      hi[i] = (uint16_t)(h & 0xFFFFu);
+      lo[i] = (uint16_t)(l & 0xFFFFu);
+    }
   }
 }
 
@@ -55,9 +60,9 @@ heal_status_t split_launch(const float* x, void* hi, void* lo, long long n, int 
   const cudaError_t e =
       fmt == HEAL_SPLIT_FP16_S11
           ? launch_pdl(heal_split_kernel<0>, dim3((unsigned)blocks), dim3(256), 0, s, x, (uint16_t*)hi, (uint16_t*)lo, n,
-                       vec ? 1 : 0)
+                       vec ? 1 : 0, device_status_ptr())
           : launch_pdl(heal_split_kernel<1>, dim3((unsigned)blocks), dim3(256), 0, s, x, (uint16_t*)hi, (uint16_t*)lo, n,
-                       vec ? 1 : 0);
+                       vec ? 1 : 0, device_status_ptr());
   return e == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 
