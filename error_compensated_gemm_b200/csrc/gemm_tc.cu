@@ -49,11 +49,19 @@ constexpr int kSplitWarp0 = 2, kNumEpiWarps = 4;
 // epilogue warps (which must start at a multiple of 4 so that warp % 4 names the TMEM lane
 // quarter).  Six split warps for every tile width (ten measured no faster on the skinny
 // decode tiles, whose time goes elsewhere).
+// The skinny tiles with BN <= 32 have a second MMA issuer, one warp after the epilogue
+// warps: an N <= 32 MMA is short, so one thread's issue rate (tens of cycles per
+// tcgen05.mma plus the per-stage waits and commits) bounds these tiles; the two issuers take
+// alternate work units, each with its own TMEM accumulator buffer (chain mode keeps one
+// issuer).  BN = 64 keeps twelve warps: with a thirteenth, four warps share one SM
+// sub-partition and its 64-column epilogue would be held to 128 registers.
 template <int BN>
 struct Roles {
   static constexpr int kSplitWarps = 6;
   static constexpr int kEpiWarp0 = kSplitWarp0 + kSplitWarps;
-  static constexpr int kThreads = (kEpiWarp0 + kNumEpiWarps) * 32;
+  static constexpr int kMmaIssuers = BN <= 32 ? 2 : 1;
+  static constexpr int kMma2Warp = kEpiWarp0 + kNumEpiWarps;   // the second issuer's warp
+  static constexpr int kThreads = (kEpiWarp0 + kNumEpiWarps + kMmaIssuers - 1) * 32;
   static_assert(kEpiWarp0 % 4 == 0, "epilogue warps must start at a lane-quarter boundary");
 };
 
@@ -81,7 +89,11 @@ struct Cfg {
   static constexpr int kBBytes = BN * kBK * 4;
   static constexpr int kStageBytes = kABytes + kBBytes;
   static constexpr int kStages = (216 * 1024) / kStageBytes > 8 ? 8 : (216 * 1024) / kStageBytes;
-  static constexpr int kTmemCols = (2 * BN) <= 32 ? 32 : (2 * BN) <= 64 ? 64 : (2 * BN) <= 128 ? 128 : (2 * BN) <= 256 ? 256 : 512;
+  // TMEM accumulator buffers: four for the skinny tiles (the MMA issuers run up to three
+  // work units ahead of the epilogue), two for the 128-wide tile
+  static constexpr int kAccBufs = BN <= 64 ? 4 : 2;
+  static constexpr int kTmemCols = (kAccBufs * BN) <= 32 ? 32 : (kAccBufs * BN) <= 64 ? 64 : (kAccBufs * BN) <= 128 ? 128
+                                 : (kAccBufs * BN) <= 256 ? 256 : 512;
   // chain mode (BN <= 32): the running sum a predecessor CTA hands over, 128 rows x BN FP32
   static constexpr int kSumBytes = BN <= 32 ? kBM * BN * 4 : 0;
   static constexpr int kSmemBytes = kStages * kStageBytes + kSumBytes + 1024 /*barriers*/ + 1024 /*align*/;
@@ -122,9 +134,12 @@ struct WorkIter {
   __device__ bool valid() const { return splitk ? (u < u_end) : (tile < ntiles); }
   __device__ void advance() {
     if (splitk) {
+      // tile = u / nc, chunk = u % nc, kept incrementally (no division per unit)
       ++u;
-      tile = u / nc;
-      chunk = u % nc;
+      if (++chunk == nc) {
+        chunk = 0;
+        ++tile;
+      }
     } else if (++chunk == nc) {
       chunk = 0;
       tile += gridDim.x;
@@ -134,6 +149,11 @@ struct WorkIter {
 
 // Tile raster: groups of 8 kernel-A row tiles, column tiles inside a group.
 __device__ __forceinline__ void tile_coords(int tile, int tiles_m, int tiles_n, int& tm, int& tn) {
+  if (tiles_n == 1) {   // one column of tiles (the skinny kernels): the raster is the identity
+    tm = tile;
+    tn = 0;
+    return;
+  }
   constexpr int GM = 8;
   const int group = GM * tiles_n;
   const int g = tile / group;
@@ -332,12 +352,13 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   uint64_t* full = bars;                 // TMA -> split       (tx bytes)
   uint64_t* split_done = bars + S;       // split -> MMA       (all split threads arrive)
   uint64_t* empty = bars + 2 * S;        // MMA -> TMA         (tcgen05.commit)
-  uint64_t* acc_full = bars + 3 * S;     // MMA -> epilogue    (tcgen05.commit)
-  uint64_t* acc_empty = bars + 3 * S + 2;// epilogue -> MMA    (128 arrivals)
-  uint64_t* mma_done = bars + 3 * S + 4; // MMA drain on exit
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 5);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 6);
-  uint64_t* chain_bar = bars + 3 * S + 7; // chain mode: the predecessor's running sum has landed
+  constexpr int NB = C::kAccBufs;
+  uint64_t* acc_full = bars + 3 * S;          // MMA -> epilogue    (tcgen05.commit)
+  uint64_t* acc_empty = bars + 3 * S + NB;    // epilogue -> MMA    (128 arrivals)
+  uint64_t* mma_done = bars + 3 * S + 2 * NB; // MMA drain on exit
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + 3 * S + 2 * NB + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 3 * S + 2 * NB + 2);
+  uint64_t* chain_bar = bars + 3 * S + 2 * NB + 3; // chain mode: the predecessor's running sum has landed
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -349,11 +370,11 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
       mbar_init(&split_done[s], kNumSplitWarps * 32);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < NB; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kNumEpiWarps * 32);
     }
-    mbar_init(mma_done, 1);
+    mbar_init(mma_done, args.chain ? 1 : Roles<BN>::kMmaIssuers);
     mbar_init(chain_bar, kNumEpiWarps * 32);
     *abort_flag = 0;
     fence_mbar_init();
@@ -423,16 +444,22 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
         mbar_wait(&full[jt % S], (uint32_t)(jt / S) & 1u, &dummy, args.status, 101);
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------ MMA issuer ------------------------------
+  } else if (warp == 1 || (Roles<BN>::kMmaIssuers == 2 && warp == Roles<BN>::kMma2Warp)) {
+    // ------------------------------ MMA issuer(s) ------------------------------
+    // With two issuers, issuer q takes the work units it with it % 2 == q (TMEM buffers
+    // it % NB of that parity); every unit's MMAs come from one thread and its commits track
+    // exactly them.
     if constexpr (kRegSplit) setmaxnreg_dec<96>();
-    if (lane == 0) {
+    const int nis = args.chain ? 1 : Roles<BN>::kMmaIssuers;
+    const int q = warp == 1 ? 0 : 1;
+    if (lane == 0 && q < nis) {
       int it = 0;
       for (WorkIter w(args); w.valid(); w.advance(), ++it) {
+        if (nis == 2 && (it & 1) != q) continue;
         const int s = it % S;
         const uint32_t ph = (uint32_t)(it / S) & 1u;
-        const int b = it & 1;
-        const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+        const int b = it % NB;
+        const uint32_t aph = (uint32_t)(it / NB) & 1u;
         if (!mbar_wait(&split_done[s], ph, abort_flag, args.status, 110)) break;
         if (!args.chain && !mbar_wait(&acc_empty[b], aph ^ 1u, abort_flag, args.status, 111)) break;
         tc_fence_after();
@@ -573,8 +600,8 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
     int it = 0;
     bool ok = true;
     for (WorkIter w(args); !args.chain && w.valid(); w.advance(), ++it) {
-      const int b = it & 1;
-      const uint32_t aph = (uint32_t)(it >> 1) & 1u;
+      const int b = it % NB;
+      const uint32_t aph = (uint32_t)(it / NB) & 1u;
       if (!mbar_wait(&acc_full[b], aph, abort_flag, args.status, 130)) {
         ok = false;
         break;
@@ -598,22 +625,27 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
           }
         }
       } else {
+        // all of the chunk's columns are loaded before one wait, and the TMEM buffer is
+        // handed back before the stores
         float* wsc = args.ws + (size_t)w.chunk * args.Nk * args.Mk;
+        uint32_t r[BN / 16][16];
 #pragma unroll
-        for (int c = 0; c < BN / 16; ++c) {
-          uint32_t r[16];
-          tmem_ld16(taddr + c * 16, r);
-          tmem_ld_wait();
-          if (gi < args.Mk) {
+        for (int c = 0; c < BN / 16; ++c) tmem_ld16(taddr + c * 16, r[c]);
+        tmem_ld_wait();
+        tc_fence_before();
+        mbar_arrive(&acc_empty[b]);
+        if (gi < args.Mk) {
+#pragma unroll
+          for (int c = 0; c < BN / 16; ++c)
 #pragma unroll
             for (int t = 0; t < 16; ++t) {
               const int gj = tn * BN + c * 16 + t;
               if (gj < args.Nk &&
                   HEAL_DCHECK(((long long)w.chunk * args.Nk + gj) * args.Mk + gi < args.ws_elems, args.status, 151))
-                wsc[(size_t)gj * args.Mk + gi] = __uint_as_float(r[t]);
+                wsc[(size_t)gj * args.Mk + gi] = __uint_as_float(r[c][t]);
             }
-          }
         }
+        continue;
       }
       tc_fence_before();
       mbar_arrive(&acc_empty[b]);
@@ -999,35 +1031,53 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 }
 
 // Ordered sum of chunk values: out(i, j) = ((ws[0] + ws[1]) + ws[2]) + ...
-// One thread per output; a warp covers 32 consecutive i of one j, so every chunk row it
-// reads is one coalesced 128-byte line.  Each thread requests kRedBatch chunk values at once
-// (registers, no shared memory), then adds them in ascending chunk order.  Without shared
-// memory the blocks fit beside a resident GEMM CTA: launched with programmatic dependent
-// launch they are already on the SMs, waiting, when the GEMM grid finishes, and the next
-// GEMM's CTAs can start next to them.
-constexpr int kRedBatch = 32;
-__global__ void __launch_bounds__(256) heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk,
-                                                                int Nk, float* out, long long si, long long sj,
-                                                                long long out_extent, unsigned int* status) {
+// A block covers 32 consecutive outputs (lane = output, so every chunk row a warp reads is
+// one coalesced 128-byte line) and walks the chunks in rounds of kRedWarps x kRedPer: in a
+// round, warp w holds chunks [base + w*kRedPer, base + (w+1)*kRedPer).  Every warp requests
+// its values at once (registers), then the running sums pass from warp to warp (and from
+// round to round) through shared memory, each warp adding its values in ascending chunk
+// order: the same left-to-right sum as one thread walking all chunks, with a single
+// dependent memory round trip per round instead of one per chunk.
+constexpr int kRedWarps = 8, kRedPer = 8;
+__global__ void __launch_bounds__(kRedWarps * 32) heal_chunk_reduce_kernel(const float* __restrict__ ws,
+                                                                           int num_chunks, int Mk, int Nk, float* out,
+                                                                           long long si, long long sj,
+                                                                           long long out_extent, unsigned int* status) {
+  __shared__ float run[kRedWarps][32];
   pdl_launch_dependents();   // the next kernel may be scheduled; it waits for this grid
   pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= (long long)Mk * Nk) return;
-  const int i = (int)(idx % Mk), j = (int)(idx / Mk);
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const long long o = (long long)blockIdx.x * 32 + lane;
+  const bool valid = o < (long long)Mk * Nk;
+  const int i = valid ? (int)(o % Mk) : 0, j = valid ? (int)(o / Mk) : 0;
   const size_t plane = (size_t)Mk * Nk;
   const float* p = ws + (size_t)j * Mk + i;
   float acc = 0.0f;
-  for (int c0 = 0; c0 < num_chunks; c0 += kRedBatch) {
-    const int cn = min(kRedBatch, num_chunks - c0);
-    float v[kRedBatch];
+  for (int base = 0; base < num_chunks; base += kRedWarps * kRedPer) {
+    const int c0 = base + w * kRedPer;
+    float v[kRedPer];
 #pragma unroll
-    for (int t = 0; t < kRedBatch; ++t) v[t] = t < cn ? __ldcs(p + (size_t)(c0 + t) * plane) : 0.0f;
+    for (int t = 0; t < kRedPer; ++t) v[t] = (valid && c0 + t < num_chunks) ? __ldcs(p + (size_t)(c0 + t) * plane) : 0.0f;
+    // the values must be in registers here, not loaded inside this warp's turn below (which
+    // would serialise the warps' memory round trips)
 #pragma unroll
-    for (int t = 0; t < kRedBatch; ++t)
-      if (t < cn) acc = (c0 + t == 0) ? v[t] : __fadd_rn(acc, v[t]);
+    for (int t = 0; t < kRedPer; ++t) asm volatile("" ::"f"(v[t]));
+    for (int s = 0; s < kRedWarps; ++s) {
+      if (s == w) {
+        if (w > 0) acc = run[w - 1][lane];
+        else if (base > 0) acc = run[kRedWarps - 1][lane];
+#pragma unroll
+        for (int t = 0; t < kRedPer; ++t)
+          if (c0 + t < num_chunks) acc = (c0 + t == 0) ? v[t] : __fadd_rn(acc, v[t]);
+        run[w][lane] = acc;
+      }
+      __syncthreads();
+    }
   }
-  const long long o = (long long)i * si + (long long)j * sj;
-  if (HEAL_DCHECK(o < out_extent, status, 160)) out[o] = acc;
+  if (w == kRedWarps - 1 && valid) {
+    const long long oi = (long long)i * si + (long long)j * sj;
+    if (HEAL_DCHECK(oi < out_extent, status, 160)) out[oi] = acc;
+  }
 }
 
 // ---------------------------------------------------------------------------------
@@ -1269,7 +1319,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     args.expB_sign = -1;
     args.static_op = o.b_static ? 1 : 0;   // kernel-A = B^T
     const int BNk = M <= 16 ? 16 : (M <= 32 ? 32 : 64);
-    args.tmem_cols = 2 * BNk < 32 ? 32 : 2 * BNk;
+    args.tmem_cols = 4 * BNk < 32 ? 32 : 4 * BNk;   // four accumulator buffers (Cfg::kAccBufs)
     args.chain = 0;
     const int S = cfg == HEAL_TILE_SKINNY_CHAIN ? chain_size(args.tiles_m, nc, BNk, sms) : 0;
     if (S >= 2) {
@@ -1289,9 +1339,9 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
                    : launch_skinny<2>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
     if (err != cudaSuccess) return HEAL_ERR_CUDA;
     if (!split) return HEAL_OK;
-    const long long rblocks = ((long long)N * M + 255) / 256;
+    const long long rblocks = ((long long)N * M + 31) / 32;
     if (rblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
-    const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(256), 0, stream,
+    const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(kRedWarps * 32), 0, stream,
                                      (const float*)args.ws, nc, N, M, Cout, 1LL, (long long)ldc, args.out_extent,
                                      args.status);
     return e == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
