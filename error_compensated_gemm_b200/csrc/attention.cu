@@ -652,30 +652,32 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
 }
 
 // out[b, hq, tq, :] = sum_c o_c 2^(m_c - M) / sum_c l_c 2^(m_c - M), c ascending.
-// The partials of kCombBatch CTAs are requested together (independent loads) and then
-// applied one by one in ascending CTA order, so the sums are the same as a one-at-a-time
-// loop while the number of dependent memory round trips drops by kCombBatch.
+// When a pair's partials come from at most kCombBatch CTAs (the usual case) m, l and o are
+// requested together, so the whole merge costs one memory round trip; otherwise the
+// partials of kCombBatch CTAs are requested together per step, the maximum first.  Either
+// way they are applied one by one in ascending CTA order, so the sums are the same as a
+// one-at-a-time loop.
 constexpr int kCombBatch = 8;
 template <int D>
 __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) {
+  pdl_launch_dependents();              // the next kernel may be scheduled; it waits for this grid
   pdl_wait_prerequisites();             // the decode kernel that wrote the partials has completed
   const int pr = blockIdx.x;            // (pair, row)
   const int p = pr / a.R, r = pr % a.R;
   const int d = threadIdx.x;
   const long long ufirst = (long long)p * a.nblk, ulast = ufirst + a.nblk - 1;
   const int c0 = cta_of(ufirst, a.total, a.grid), c1 = cta_of(ulast, a.total, a.grid);
-  float M = -INFINITY;
-  for (int cb = c0; cb <= c1; cb += kCombBatch) {
-    float m[kCombBatch];
+  float M = -INFINITY, L = 0.0f, O = 0.0f;
+  auto apply = [&](const float (&m)[kCombBatch], const float (&l)[kCombBatch], const float (&o)[kCombBatch]) {
 #pragma unroll
-    for (int t = 0; t < kCombBatch; ++t)
-      m[t] = (cb + t <= c1) ? slot_ptr(a.ws, cb + t, p, a.R, D)[a.R * D + 2 * r] : -INFINITY;
-#pragma unroll
-    for (int t = 0; t < kCombBatch; ++t) M = fmaxf(M, m[t]);
-  }
-  float L = 0.0f, O = 0.0f;
-  for (int cb = c0; cb <= c1; cb += kCombBatch) {
-    float m[kCombBatch], l[kCombBatch], o[kCombBatch];
+    for (int t = 0; t < kCombBatch; ++t) {
+      if (m[t] == -INFINITY) continue;
+      const float f = exp2f(m[t] - M);
+      L = __fadd_rn(L, __fmul_rn(l[t], f));
+      O = __fadd_rn(O, __fmul_rn(o[t], f));
+    }
+  };
+  auto load = [&](int cb, float (&m)[kCombBatch], float (&l)[kCombBatch], float (&o)[kCombBatch]) {
 #pragma unroll
     for (int t = 0; t < kCombBatch; ++t) {
       const bool in = cb + t <= c1;
@@ -684,12 +686,29 @@ __global__ void __launch_bounds__(D) heal_attn_combine_kernel(const AttnArgs a) 
       l[t] = in ? sl[a.R * D + 2 * r + 1] : 0.0f;
       o[t] = in ? sl[r * D + d] : 0.0f;
     }
+    // all of them in flight before any is used (not sunk into the adds that need them)
 #pragma unroll
-    for (int t = 0; t < kCombBatch; ++t) {
-      if (m[t] == -INFINITY) continue;
-      const float f = exp2f(m[t] - M);
-      L = __fadd_rn(L, __fmul_rn(l[t], f));
-      O = __fadd_rn(O, __fmul_rn(o[t], f));
+    for (int t = 0; t < kCombBatch; ++t) asm volatile("" ::"f"(m[t]), "f"(l[t]), "f"(o[t]));
+  };
+  if (c1 - c0 < kCombBatch) {
+    float m[kCombBatch], l[kCombBatch], o[kCombBatch];
+    load(c0, m, l, o);
+#pragma unroll
+    for (int t = 0; t < kCombBatch; ++t) M = fmaxf(M, m[t]);
+    apply(m, l, o);
+  } else {
+    for (int cb = c0; cb <= c1; cb += kCombBatch) {
+      float m[kCombBatch];
+#pragma unroll
+      for (int t = 0; t < kCombBatch; ++t)
+        m[t] = (cb + t <= c1) ? slot_ptr(a.ws, cb + t, p, a.R, D)[a.R * D + 2 * r] : -INFINITY;
+#pragma unroll
+      for (int t = 0; t < kCombBatch; ++t) M = fmaxf(M, m[t]);
+    }
+    for (int cb = c0; cb <= c1; cb += kCombBatch) {
+      float m[kCombBatch], l[kCombBatch], o[kCombBatch];
+      load(cb, m, l, o);
+      apply(m, l, o);
     }
   }
   const int b = p / a.Hkv, hkv = p % a.Hkv;

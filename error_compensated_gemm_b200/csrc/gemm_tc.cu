@@ -1031,53 +1031,39 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPairThreads, 1)
 }
 
 // Ordered sum of chunk values: out(i, j) = ((ws[0] + ws[1]) + ws[2]) + ...
-// A block covers 32 consecutive outputs (lane = output, so every chunk row a warp reads is
-// one coalesced 128-byte line) and walks the chunks in rounds of kRedWarps x kRedPer: in a
-// round, warp w holds chunks [base + w*kRedPer, base + (w+1)*kRedPer).  Every warp requests
-// its values at once (registers), then the running sums pass from warp to warp (and from
-// round to round) through shared memory, each warp adding its values in ascending chunk
-// order: the same left-to-right sum as one thread walking all chunks, with a single
-// dependent memory round trip per round instead of one per chunk.
-constexpr int kRedWarps = 8, kRedPer = 8;
-__global__ void __launch_bounds__(kRedWarps * 32) heal_chunk_reduce_kernel(const float* __restrict__ ws,
-                                                                           int num_chunks, int Mk, int Nk, float* out,
-                                                                           long long si, long long sj,
-                                                                           long long out_extent, unsigned int* status) {
-  __shared__ float run[kRedWarps][32];
+// One warp per block and 32 consecutive outputs per warp (lane = output, so every chunk
+// row the warp reads is one coalesced 128-byte line).  Each lane requests kRedBatch chunk
+// values at once (registers), then adds them in ascending chunk order: K = 4096 takes one
+// memory round trip.  Blocks of one warp spread the loads over every SM, and without shared
+// memory they fit beside a resident GEMM CTA: launched with programmatic dependent launch
+// they are already on the SMs, waiting, when the GEMM grid finishes.
+constexpr int kRedBatch = 64;
+__global__ void __launch_bounds__(32) heal_chunk_reduce_kernel(const float* __restrict__ ws, int num_chunks, int Mk,
+                                                               int Nk, float* out, long long si, long long sj,
+                                                               long long out_extent, unsigned int* status) {
   pdl_launch_dependents();   // the next kernel may be scheduled; it waits for this grid
   pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed
-  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
-  const long long o = (long long)blockIdx.x * 32 + lane;
-  const bool valid = o < (long long)Mk * Nk;
-  const int i = valid ? (int)(o % Mk) : 0, j = valid ? (int)(o / Mk) : 0;
+  const long long o = (long long)blockIdx.x * 32 + threadIdx.x;
+  if (o >= (long long)Mk * Nk) return;
+  const int i = (int)(o % Mk), j = (int)(o / Mk);
   const size_t plane = (size_t)Mk * Nk;
   const float* p = ws + (size_t)j * Mk + i;
   float acc = 0.0f;
-  for (int base = 0; base < num_chunks; base += kRedWarps * kRedPer) {
-    const int c0 = base + w * kRedPer;
-    float v[kRedPer];
+  for (int c0 = 0; c0 < num_chunks; c0 += kRedBatch) {
+    const int cn = min(kRedBatch, num_chunks - c0);
+    float v[kRedBatch];
 #pragma unroll
-    for (int t = 0; t < kRedPer; ++t) v[t] = (valid && c0 + t < num_chunks) ? __ldcs(p + (size_t)(c0 + t) * plane) : 0.0f;
-    // the values must be in registers here, not loaded inside this warp's turn below (which
-    // would serialise the warps' memory round trips)
+    for (int t = 0; t < kRedBatch; ++t) v[t] = t < cn ? __ldcs(p + (size_t)(c0 + t) * plane) : 0.0f;
+    // every value is requested before the first add (the loads must not be interleaved with
+    // the dependent adds, which would make one memory round trip per chunk)
 #pragma unroll
-    for (int t = 0; t < kRedPer; ++t) asm volatile("" ::"f"(v[t]));
-    for (int s = 0; s < kRedWarps; ++s) {
-      if (s == w) {
-        if (w > 0) acc = run[w - 1][lane];
-        else if (base > 0) acc = run[kRedWarps - 1][lane];
+    for (int t = 0; t < kRedBatch; ++t) asm volatile("" ::"f"(v[t]));
 #pragma unroll
-        for (int t = 0; t < kRedPer; ++t)
-          if (c0 + t < num_chunks) acc = (c0 + t == 0) ? v[t] : __fadd_rn(acc, v[t]);
-        run[w][lane] = acc;
-      }
-      __syncthreads();
-    }
+    for (int t = 0; t < kRedBatch; ++t)
+      if (t < cn) acc = (c0 + t == 0) ? v[t] : __fadd_rn(acc, v[t]);
   }
-  if (w == kRedWarps - 1 && valid) {
-    const long long oi = (long long)i * si + (long long)j * sj;
-    if (HEAL_DCHECK(oi < out_extent, status, 160)) out[oi] = acc;
-  }
+  const long long oi = (long long)i * si + (long long)j * sj;
+  if (HEAL_DCHECK(oi < out_extent, status, 160)) out[oi] = acc;
 }
 
 // ---------------------------------------------------------------------------------
@@ -1341,7 +1327,7 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     if (!split) return HEAL_OK;
     const long long rblocks = ((long long)N * M + 31) / 32;
     if (rblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
-    const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(kRedWarps * 32), 0, stream,
+    const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(32), 0, stream,
                                      (const float*)args.ws, nc, N, M, Cout, 1LL, (long long)ldc, args.out_extent,
                                      args.status);
     return e == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;

@@ -173,6 +173,21 @@ def test_decode_shapes_full_oracle(M):
         assert np.array_equal(gemm(X, W, tile=tile), C), tile
 
 
+@pytest.mark.parametrize("M,K,N", [(1, 14336, 384), (8, 4160, 640), (40, 200, 256), (64, 8256, 384)])
+def test_splitk_reduce_rounds_and_ragged_chunk_counts(M, K, N):
+    """The chunk reduce walks the chunks in rounds of 8 warps x 8 chunks: K = 14336 (224
+    chunks, four rounds), 4160 (65: a second round of one chunk), 200 (4: warps with no
+    chunk pass the running sum on) and 8256 (129).  Split-K must give the bits of the
+    single-CTA chunk sum and stay within the oracle's bound."""
+    X, W = synthetic.gemm_decode(M, K=K, N=N)
+    X, W = X.numpy(), W.numpy()
+    c_split = gemm(X, W, tile=heal.TILE_SKINNY_SPLITK)
+    c_ref = gemm(X, W, tile=heal.TILE_128x128)
+    assert np.array_equal(c_split, c_ref)
+    assert G.normwise_rel_err(c_split, G.gemm_ref(X, W)) <= TOL_FP16
+    assert_elementwise(c_split, X, W)
+
+
 @pytest.mark.parametrize("M,K,N", [(8, 1000, 5120), (1, 520, 8192), (3, 4096, 640), (32, 1500, 1000)])
 def test_chain_split_over_uneven_cta_runs(M, K, N):
     """Chain mode with 2, 3 and 8 CTAs per tile and chunk runs of unequal length (K not a
