@@ -175,10 +175,10 @@ def test_decode_shapes_full_oracle(M):
 
 @pytest.mark.parametrize("M,K,N", [(1, 14336, 384), (8, 4160, 640), (40, 200, 256), (64, 8256, 384)])
 def test_splitk_reduce_rounds_and_ragged_chunk_counts(M, K, N):
-    """The chunk reduce walks the chunks in rounds of 8 warps x 8 chunks: K = 14336 (224
-    chunks, four rounds), 4160 (65: a second round of one chunk), 200 (4: warps with no
-    chunk pass the running sum on) and 8256 (129).  Split-K must give the bits of the
-    single-CTA chunk sum and stay within the oracle's bound."""
+    """The chunk reduce adds the chunk values in batches of 64 loads: K = 14336 (224 chunks,
+    four batches, the last one partial), 4160 (65: a second batch of one chunk), 200 (4: one
+    partial batch) and 8256 (129).  Split-K must give the bits of the single-CTA chunk sum
+    and stay within the oracle's bound."""
     X, W = synthetic.gemm_decode(M, K=K, N=N)
     X, W = X.numpy(), W.numpy()
     c_split = gemm(X, W, tile=heal.TILE_SKINNY_SPLITK)
