@@ -104,38 +104,80 @@ __global__ void add_kernel(float* __restrict__ x, const float* __restrict__ y, l
     x[e] += y[e];
 }
 
-// index of the largest value of each row (lowest index among equal maxima; NaN never wins)
-__global__ void argmax_kernel(const float* __restrict__ x, int rows, int n, int32_t* __restrict__ out) {
+// index of the largest value of each row (lowest index among equal maxima; NaN never wins).
+// One block of 1024 threads per row: 16-byte loads, four of them in flight per thread
+// (a 128256-wide vocabulary row is 31 float4 per thread), then warp shuffles and one pass
+// over the 32 warps' candidates.  The order of the comparisons does not matter: the rule
+// picks the same index whatever the order.
+constexpr int kArgThreads = 1024;
+__device__ __forceinline__ void arg_take(float v, int j, float& best, int& idx) {
+  if (v > best || (v == best && j < idx)) {
+    best = v;
+    idx = j;
+  }
+}
+__global__ void __launch_bounds__(kArgThreads) argmax_kernel(const float* __restrict__ x, int rows, int n,
+                                                            int32_t* __restrict__ out) {
   pdl_launch_dependents();
   pdl_wait_prerequisites();
-  __shared__ float bv[kThreads];
-  __shared__ int bi[kThreads];
+  __shared__ float wv[kArgThreads / 32];
+  __shared__ int wi[kArgThreads / 32];
   const int r = blockIdx.x;
   const float* xr = x + (size_t)r * n;
   float best = -FLT_MAX;
   int idx = 0x7fffffff;
-  for (int j = threadIdx.x; j < n; j += blockDim.x) {
-    const float v = xr[j];
-    if (v > best || (v == best && j < idx)) {
-      best = v;
-      idx = j;
-    }
-  }
-  bv[threadIdx.x] = best;
-  bi[threadIdx.x] = idx;
-  __syncthreads();
-  for (int s = blockDim.x / 2; s > 0; s >>= 1) {
-    if ((int)threadIdx.x < s) {
-      const float v = bv[threadIdx.x + s];
-      const int j = bi[threadIdx.x + s];
-      if (v > bv[threadIdx.x] || (v == bv[threadIdx.x] && j < bi[threadIdx.x])) {
-        bv[threadIdx.x] = v;
-        bi[threadIdx.x] = j;
+  const bool vec = (n % 4 == 0) && ((reinterpret_cast<uintptr_t>(xr) & 15) == 0);
+  if (vec) {
+    const float4* x4 = reinterpret_cast<const float4*>(xr);
+    const int n4 = n / 4;
+    for (int q0 = threadIdx.x; q0 < n4; q0 += 4 * kArgThreads) {
+      float4 a[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int q = q0 + u * kArgThreads;
+        a[u] = q < n4 ? x4[q] : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int j = 4 * (q0 + u * kArgThreads);
+        arg_take(a[u].x, j, best, idx);
+        arg_take(a[u].y, j + 1, best, idx);
+        arg_take(a[u].z, j + 2, best, idx);
+        arg_take(a[u].w, j + 3, best, idx);
       }
     }
-    __syncthreads();
+  } else {
+    for (int j0 = threadIdx.x; j0 < n; j0 += 4 * kArgThreads) {
+      float a[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) a[u] = j0 + u * kArgThreads < n ? xr[j0 + u * kArgThreads] : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) arg_take(a[u], j0 + u * kArgThreads, best, idx);
+    }
   }
-  if (threadIdx.x == 0) out[r] = bi[0] == 0x7fffffff ? 0 : bi[0];
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_down_sync(0xffffffffu, best, o);
+    const int oi = __shfl_down_sync(0xffffffffu, idx, o);
+    arg_take(ov, oi, best, idx);
+  }
+  const int w = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (lane == 0) {
+    wv[w] = best;
+    wi[w] = idx;
+  }
+  __syncthreads();
+  if (w == 0) {
+    best = wv[lane];
+    idx = wi[lane];
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_down_sync(0xffffffffu, best, o);
+      const int oi = __shfl_down_sync(0xffffffffu, idx, o);
+      arg_take(ov, oi, best, idx);
+    }
+    if (lane == 0) out[r] = idx == 0x7fffffff ? 0 : idx;
+  }
 }
 
 int grid_for(long long n) {
@@ -228,7 +270,7 @@ heal_status_t heal_argmax(const float* x, int rows, int n, int32_t* out, heal_st
   if (rows < 0 || n <= 0) return HEAL_ERR_INVALID_ARGUMENT;
   if (rows == 0) return HEAL_OK;
   if (!x || !out) return HEAL_ERR_INVALID_ARGUMENT;
-  return launch_pdl(argmax_kernel, dim3(rows), dim3(kThreads), 0, (cudaStream_t)stream, x, rows, n, out) ==
+  return launch_pdl(argmax_kernel, dim3(rows), dim3(kArgThreads), 0, (cudaStream_t)stream, x, rows, n, out) ==
                  cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
 }
 

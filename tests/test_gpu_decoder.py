@@ -133,3 +133,21 @@ def test_heads_to_rows_is_an_exact_transpose():
 
 def to_np_t(t):
     return t.detach().cpu()
+
+
+def test_argmax_vector_and_scalar_paths():
+    """The argmax kernel reads 16-byte vectors when a row is 16-byte aligned (n % 4 == 0) and
+    single values otherwise; both give numpy's first maximum, on ties, a lone finite value
+    among -inf, and maxima at the first and the last index (the ragged tail)."""
+    d = torch.device("cuda:0")
+    rng = np.random.default_rng(7)
+    for n in (128256, 10001, 4, 3):
+        x = rng.standard_normal((5, n)).astype(np.float32)
+        x[1, n // 3] = x[1, n - 1] = 60.0
+        x[2, :] = -np.inf
+        x[2, n - 1] = -1e38
+        x[3, 0] = 70.0
+        x[4, n - 1] = 80.0
+        idx = torch.empty(5, dtype=torch.int32, device=d)
+        heal.heal_argmax(torch.from_numpy(x).to(d), idx)
+        assert list(idx.cpu().numpy()) == [OD.argmax_lowest(r) for r in x], n
