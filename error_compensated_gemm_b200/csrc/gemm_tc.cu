@@ -79,7 +79,8 @@ struct GemmArgs {
   int static_op;            // 0: none; 1: kernel-A, 2: kernel-B is not written by the kernels
                             // before this one (its first stages may be requested early)
   unsigned int* status;     // device status word
-  long long out_extent;     // elements of `out` the call may write (debug-build checks)
+  long long out_extent;
+  int ws_tma;               // split K, BN = 64: chunk tiles go to ws by TMA store (map in the B-lo slot)     // elements of `out` the call may write (debug-build checks)
   long long ws_elems;       // FP32 elements of the workspace (debug-build checks)
 };
 
@@ -96,7 +97,10 @@ struct Cfg {
                                  : (kAccBufs * BN) <= 256 ? 256 : 512;
   // chain mode (BN <= 32): the running sum a predecessor CTA hands over, 128 rows x BN FP32
   static constexpr int kSumBytes = BN <= 32 ? kBM * BN * 4 : 0;
-  static constexpr int kSmemBytes = kStages * kStageBytes + kSumBytes + 1024 /*barriers*/ + 1024 /*align*/;
+  // split K at BN = 64: one chunk tile (BN rows x 128 FP32) staged for a TMA store to the
+  // workspace (the 64-column stores per thread otherwise bound the epilogue)
+  static constexpr int kStoreBytes = BN == 64 ? kBM * BN * 4 : 0;
+  static constexpr int kSmemBytes = kStages * kStageBytes + kSumBytes + kStoreBytes + 1024 /*barriers*/ + 1024 /*align*/;
   static_assert(kStages >= 2, "at least two stages");
 };
 
@@ -348,7 +352,8 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
   uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint8_t* stages = smem;
   float* sum_buf = reinterpret_cast<float*>(smem + S * C::kStageBytes);   // chain mode: [128 rows][BN]
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kSumBytes);
+  float* out_stage = reinterpret_cast<float*>(smem + S * C::kStageBytes + C::kSumBytes);   // [BN][128] (BN = 64)
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S * C::kStageBytes + C::kSumBytes + C::kStoreBytes);
   uint64_t* full = bars;                 // TMA -> split       (tx bytes)
   uint64_t* split_done = bars + S;       // split -> MMA       (all split threads arrive)
   uint64_t* empty = bars + 2 * S;        // MMA -> TMA         (tcgen05.commit)
@@ -634,6 +639,27 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
         tmem_ld_wait();
         tc_fence_before();
         mbar_arrive(&acc_empty[b]);
+        if constexpr (C::kStoreBytes > 0 && B_PRE == 0) {
+          if (args.ws_tma) {
+            // the chunk tile through shared memory and one TMA store (the workspace's map
+            // rides in the kernel-B lo slot: kernel-B, the activations, is never pre-split
+            // here).  The previous tile's store must have read the staging buffer first.
+            const bool issuer = (warp == kEpiWarp0 && lane == 0);
+            if (issuer) bulk_wait_group_read0();
+            named_bar_sync(1, kNumEpiWarps * 32);
+#pragma unroll
+            for (int c = 0; c < BN / 16; ++c)
+#pragma unroll
+              for (int t = 0; t < 16; ++t) out_stage[(c * 16 + t) * kBM + i_local] = __uint_as_float(r[c][t]);
+            fence_proxy_async_smem();
+            named_bar_sync(1, kNumEpiWarps * 32);
+            if (issuer && HEAL_DCHECK(w.chunk < args.num_chunks, args.status, 156)) {
+              tma_store_3d(&tmB_lo, out_stage, tm * kBM, tn * BN, w.chunk);
+              bulk_commit_group();
+            }
+            continue;
+          }
+        }
         if (gi < args.Mk) {
 #pragma unroll
           for (int c = 0; c < BN / 16; ++c)
@@ -676,6 +702,9 @@ __global__ void __launch_bounds__(Roles<BN>::kThreads, 1)
             }
         }
       }
+    }
+    if constexpr (C::kStoreBytes > 0 && B_PRE == 0) {
+      if (args.ws_tma && warp == kEpiWarp0 && lane == 0) bulk_wait_group0();   // every tile stored
     }
     (void)ok;
   }
@@ -1318,6 +1347,18 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
     if (!operand_map(&ta, B, b_mn, pre != 0, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (pre == 1 && !operand_map(&talo, o.b_lo, b_mn, true, N, K, ldb, kBM)) return HEAL_ERR_CUDA;
     if (!operand_map(&tb, A, false, false, M, K, lda, BNk)) return HEAL_ERR_CUDA;
+    args.ws_tma = 0;
+    if (split && BNk == 64 && N % 4 == 0 && (reinterpret_cast<uintptr_t>(o.workspace) & 15) == 0) {
+      // the workspace as [nc][M][N] FP32 for the TMA stores of chunk tiles (BN x 128)
+      const cuuint64_t dims[3] = {(cuuint64_t)N, (cuuint64_t)M, (cuuint64_t)nc};
+      const cuuint64_t strides[2] = {(cuuint64_t)N * 4, (cuuint64_t)N * M * 4};
+      const cuuint32_t box[3] = {(cuuint32_t)kBM, 64u, 1u};
+      const cuuint32_t es[3] = {1, 1, 1};
+      if (!encode_tensor_map(&tblo, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, o.workspace, dims, strides, box, es,
+                             CU_TENSOR_MAP_SWIZZLE_NONE))
+        return HEAL_ERR_CUDA;
+      args.ws_tma = 1;
+    }
     const long long units = split ? (long long)args.tiles_m * nc : (long long)args.tiles_m;
     const int grid = args.chain ? args.tiles_m * args.chain : (int)(units < sms ? units : sms);
     err = pre == 0 ? launch_skinny<0>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream)
