@@ -1095,6 +1095,56 @@ __global__ void __launch_bounds__(32) heal_chunk_reduce_kernel(const float* __re
   if (HEAL_DCHECK(oi < out_extent, status, 160)) out[oi] = acc;
 }
 
+// The same ordered sum for large outputs (M >= 32: 8-67 MB of chunk values): each lane
+// takes four consecutive outputs of one column j and reads them as one 16-byte vector per
+// chunk, so a warp moves 512 contiguous bytes of each chunk plane per request (4x longer
+// runs in DRAM than the one-value-per-lane kernel), kRedWideBatch chunks per round trip.
+constexpr int kRedWideBatch = 16;
+__global__ void __launch_bounds__(128) heal_chunk_reduce_wide_kernel(const float* __restrict__ ws, int num_chunks,
+                                                                     int Mk, int Nk, float* out, long long sj,
+                                                                     long long out_extent, unsigned int* status) {
+  pdl_launch_dependents();   // the next kernel may be scheduled; it waits for this grid
+  pdl_wait_prerequisites();   // the GEMM kernel that wrote ws has completed
+  const int q4 = Mk / 4;     // float4 per column (Mk % 4 == 0)
+  const long long v = (long long)blockIdx.x * blockDim.x + threadIdx.x;   // float4 index
+  if (v >= (long long)q4 * Nk) return;
+  const int j = (int)(v / q4), i0 = (int)(v % q4) * 4;
+  const size_t plane4 = (size_t)Mk * Nk / 4;
+  const float4* p = reinterpret_cast<const float4*>(ws) + (size_t)j * q4 + i0 / 4;
+  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+  for (int c0 = 0; c0 < num_chunks; c0 += kRedWideBatch) {
+    const int cn = min(kRedWideBatch, num_chunks - c0);
+    float4 x[kRedWideBatch];
+#pragma unroll
+    for (int t = 0; t < kRedWideBatch; ++t)
+      x[t] = t < cn ? __ldcs(p + (size_t)(c0 + t) * plane4) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    // all requested before the first add (not sunk into the dependent adds)
+#pragma unroll
+    for (int t = 0; t < kRedWideBatch; ++t) asm volatile("" ::"f"(x[t].x), "f"(x[t].y), "f"(x[t].z), "f"(x[t].w));
+#pragma unroll
+    for (int t = 0; t < kRedWideBatch; ++t) {
+      if (t >= cn) break;
+      const bool first = (c0 + t == 0);
+      acc[0] = first ? x[t].x : __fadd_rn(acc[0], x[t].x);
+      acc[1] = first ? x[t].y : __fadd_rn(acc[1], x[t].y);
+      acc[2] = first ? x[t].z : __fadd_rn(acc[2], x[t].z);
+      acc[3] = first ? x[t].w : __fadd_rn(acc[3], x[t].w);
+    }
+  }
+  // out(i, j) at out[i + j * sj]
+  float* o = out + (long long)j * sj + i0;
+  if (HEAL_DCHECK((long long)j * sj + i0 + 3 < out_extent, status, 161)) {
+    if ((reinterpret_cast<uintptr_t>(o) & 15) == 0)
+      *reinterpret_cast<float4*>(o) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+    else {
+      o[0] = acc[0];
+      o[1] = acc[1];
+      o[2] = acc[2];
+      o[3] = acc[3];
+    }
+  }
+}
+
 // ---------------------------------------------------------------------------------
 // Host side
 // ---------------------------------------------------------------------------------
@@ -1366,6 +1416,15 @@ heal_status_t gemm_launch(int M, int N, int K, const float* A, long long lda, co
                    : launch_skinny<2>(BNk, b_mn, fmt, ta, talo, tb, tblo, args, grid, stream);
     if (err != cudaSuccess) return HEAL_ERR_CUDA;
     if (!split) return HEAL_OK;
+    if (M >= 32 && N % 4 == 0 && (reinterpret_cast<uintptr_t>(o.workspace) & 15) == 0) {
+      const long long vec = (long long)N / 4 * M;
+      const long long wblocks = (vec + 127) / 128;
+      if (wblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
+      const cudaError_t e = launch_pdl(heal_chunk_reduce_wide_kernel, dim3((unsigned)wblocks), dim3(128), 0, stream,
+                                       (const float*)args.ws, nc, N, M, Cout, (long long)ldc, args.out_extent,
+                                       args.status);
+      return e == cudaSuccess ? HEAL_OK : HEAL_ERR_CUDA;
+    }
     const long long rblocks = ((long long)N * M + 31) / 32;
     if (rblocks >= (1LL << 31)) return HEAL_ERR_UNSUPPORTED;
     const cudaError_t e = launch_pdl(heal_chunk_reduce_kernel, dim3((unsigned)rblocks), dim3(32), 0, stream,
