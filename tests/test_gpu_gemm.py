@@ -188,6 +188,20 @@ def test_splitk_reduce_rounds_and_ragged_chunk_counts(M, K, N):
     assert_elementwise(c_split, X, W)
 
 
+@pytest.mark.parametrize("M,N,K,b_layout", [(48, 1002, 320, 1), (64, 1000, 512, 0), (33, 998, 256, 1)])
+def test_splitk_wide_tiles_store_and_reduce_forms(M, N, K, b_layout):
+    """Split K with the 64-column tile: N % 4 == 0 takes the TMA-store epilogue and the
+    16-byte-vector reduce (N = 1000, ragged last 128-row tile), N % 4 != 0 takes the
+    scalar stores and the one-value-per-lane reduce.  Both give the single-CTA bits."""
+    X, W = synthetic.gemm_decode(M, K=K, N=N)
+    X, W = X.numpy(), W.numpy()
+    Bin = W if b_layout == 0 else np.ascontiguousarray(W.T)
+    c_split = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_SKINNY_SPLITK)
+    c_ref = gemm(X, Bin, b_layout=b_layout, tile=heal.TILE_128x128)
+    assert np.array_equal(c_split, c_ref)
+    assert G.normwise_rel_err(c_split, G.gemm_ref(X, W)) <= TOL_FP16
+
+
 @pytest.mark.parametrize("M,K,N", [(8, 1000, 5120), (1, 520, 8192), (3, 4096, 640), (32, 1500, 1000)])
 def test_chain_split_over_uneven_cta_runs(M, K, N):
     """Chain mode with 2, 3 and 8 CTAs per tile and chunk runs of unequal length (K not a
