@@ -6,21 +6,24 @@
 // and C = A.B is synthesised from three 16-bit products with FP32 accumulation,
 //     C ~= Ah.Bh + 2^-L (Ah.Bl + Al.Bh).
 //
-// Kernel structure (one persistent CTA per SM, 12 warps):
+// Kernel structure (one persistent CTA per SM, 12 warps; 13 for the tiles with BN <= 32):
 //   warp 0      TMA producer: FP32 tiles of both operands, 128-byte swizzled, into a
 //               ring of shared-memory stages (one stage = 64 values of K).
 //   warp 1      MMA issuer (one thread): per stage, the two correction products into a
 //               fresh TMEM accumulator, then Ah.Bh with scale-input-d = L, which scales
 //               the corrections by 2^-L as it adds the main product, then the rest of
-//               Ah.Bh.  The accumulator is double-buffered in TMEM.
+//               Ah.Bh.  Two TMEM accumulator buffers for the 128-wide tile, four for the
+//               skinny tiles; with BN <= 32 a second issuer (warp 12) takes every other
+//               work unit.
 //   warps 2-7   split warps: read the FP32 stage, write hi and lo back into the same
 //               shared memory in the UMMA 128-byte-swizzle canonical layout, fence the
 //               async proxy and release the stage to the MMA issuer.  (No split pass
 //               goes through HBM.)
 //   warps 8-11  epilogue: drain each 64-wide K chunk from TMEM and add it to the running
 //               FP32 sum in registers (round-to-nearest, ascending chunk order), then
-//               store C.  In split-K mode every chunk value goes to a workspace instead,
-//               and heal_chunk_reduce adds them in the same order.  In chain mode (a
+//               store C.  In split-K mode every chunk value goes to a workspace instead
+//               (at BN = 64 through shared memory and a TMA store), and a reduce kernel
+//               adds them in the same order.  In chain mode (a
 //               cluster of S CTAs per tile, each owning a contiguous run of chunks) every
 //               chunk keeps its own TMEM accumulator; at the end the running FP32 sum is
 //               handed from CTA to CTA through distributed shared memory in ascending chunk
