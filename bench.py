@@ -35,6 +35,8 @@ PREFILL = (4096, 4096, 14336)
 DECODE_M = (1, 8, 64)
 CHAIN = 8             # decode GEMMs issued back to back in the chain part
 KV = dict(B=8, T=8192, Hkv=8, Hq=32, D=128)
+L2_CLEAN_BYTES = 256 * 1024 * 1024
+REF_COPY_BYTES = 4 * 4096 * 4096          # bytes a decode GEMM reads (FP32 4096 x 4096 weights)
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 
 
@@ -116,6 +118,13 @@ class Workload:
         self.only = only
         M, K, N = PREFILL
         so = seed_offset
+        # L2 cleaning before every part of a step (outside the part's events): a buffer
+        # larger than L2 (126 MB) is written, then a second one is read, so that each part
+        # starts with none of its inputs in L2 and without another part's dirty lines, whose
+        # write-back it would otherwise pay for.
+        self.l2_w = torch.zeros(L2_CLEAN_BYTES // 4, device=dev)
+        self.l2_r = torch.zeros(L2_CLEAN_BYTES // 4, device=dev)
+        self.l2_acc = torch.zeros(1, device=dev)
         need = lambda part: only is None or only == part or (part == "kv_writer" and only == "attention")
         if need("prefill"):
             X, W = synthetic.gemm_prefill(M=M, K=K, N=N, seed_x=0 + so, seed_w=1 + so)
@@ -132,6 +141,11 @@ class Workload:
             self.W16 = self.W.half()
         self.dec = []
         if need("decode"):
+            # a plain device copy moving as many bytes as one decode GEMM reads (32 MB read,
+            # 32 MB written): the single-launch streaming time at this size, timed like the
+            # decode parts (torch's copy kernel, not this library's; context only)
+            self.ref_src = torch.zeros(REF_COPY_BYTES // 8, device=dev)
+            self.ref_dst = torch.zeros(REF_COPY_BYTES // 8, device=dev)
             for i, m in enumerate(DECODE_M):
                 Xd, Wd = synthetic.gemm_decode(m, seed_x=0 + so, seed_w=1 + so + 10 * (i + 1))
                 ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(m, 4096, 4096, heal.TILE_SKINNY_SPLITK) // 4),
@@ -195,8 +209,18 @@ class Workload:
         h = self.heal
         out = []
         only = self.only
+        # Independent parts, each timed after an L2 clean (run_graphs): the KV writer (which
+        # fills the caches attention reads), the prefill product, attention, the decode GEMMs.
+        if only in (None, "kv_writer", "attention"):
+            out.append(("kv_writer", lambda: (h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs),
+                                              h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks),
+                                              h.heal_kv_quantize_int16(self.Vb, self.vc, self.vs))))
         if only in (None, "prefill"):
             out.append(("prefill", lambda: self.prefill()))
+        if only in (None, "attention"):
+            out.append(("attention", lambda: h.heal_attention_int16(
+                self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len, KV["D"] ** -0.5, self.out,
+                self.aws)))
         if only in (None, "decode"):
             for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
                 out.append((f"decode{m}", lambda Xd=Xd, Wd=Wd, Cd=Cd, ws=ws: h.heal_gemm_compensated(
@@ -210,14 +234,7 @@ class Workload:
             out.append(("decode1_chain", lambda: self.run_chain(False)))
             out.append(("decode1_chain_presplit", lambda: self.run_chain(True)))
             out.append(("decode1_chain_w16", lambda: self.run_chain16()))
-        if only in (None, "kv_writer", "attention"):
-            out.append(("kv_writer", lambda: (h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs),
-                                              h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks),
-                                              h.heal_kv_quantize_int16(self.Vb, self.vc, self.vs))))
-        if only in (None, "attention"):
-            out.append(("attention", lambda: h.heal_attention_int16(
-                self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len, KV["D"] ** -0.5, self.out,
-                self.aws)))
+            out.append(("ref_copy_67MB", lambda: self.ref_dst.copy_(self.ref_src)))
         return out
 
     def prefill(self):
@@ -250,8 +267,13 @@ class Workload:
                 fn()
             self.graphs.append((name, g))
 
+    def l2_clean(self):
+        self.l2_w.zero_()
+        self.torch.sum(self.l2_r, dim=0, out=self.l2_acc[0])
+
     def run_graphs(self, ev=None):
         for name, g in self.graphs:
+            self.l2_clean()
             if ev is not None:
                 ev[name][0].record()
             g.replay()
@@ -259,49 +281,14 @@ class Workload:
                 ev[name][1].record()
 
     def run(self, ev=None):
-        """One step.  ev: dict name -> (start, end) CUDA events, recorded around each part."""
-        h = self.heal
-
-        def rec(name, i):
+        """One step, eagerly (the warm-up before capture).  ev: dict name -> (start, end) CUDA
+        events, recorded around each part."""
+        for name, fn in self.parts():
             if ev is not None:
-                ev[name][i].record()
-
-        only = self.only
-        if only in (None, "prefill"):
-            rec("prefill", 0)
-            self.prefill()
-            rec("prefill", 1)
-        if only in (None, "decode"):
-            for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
-                rec(f"decode{m}", 0)
-                h.heal_gemm_compensated(Xd, Wd, Cd, workspace=ws)
-                rec(f"decode{m}", 1)
-            for (m, Xd, Wd, Cd, ws, whi, wlo) in self.dec:
-                rec(f"decode{m}_presplit", 0)
-                h.heal_gemm_compensated(Xd, whi, Cd, b_lo=wlo, workspace=ws)
-                rec(f"decode{m}_presplit", 1)
-            for (m, Xd, W16, Cd, ws) in self.dec16:
-                rec(f"decode{m}_w16", 0)
-                h.heal_gemm_compensated(Xd, W16, Cd, workspace=ws, b_16bit=True)
-                rec(f"decode{m}_w16", 1)
-            for name, pre in (("decode1_chain", False), ("decode1_chain_presplit", True)):
-                rec(name, 0)
-                self.run_chain(pre)
-                rec(name, 1)
-            rec("decode1_chain_w16", 0)
-            self.run_chain16()
-            rec("decode1_chain_w16", 1)
-        if only in (None, "kv_writer", "attention"):
-            rec("kv_writer", 0)
-            h.heal_kv_quantize_int16(self.Qb, self.qc, self.qs)
-            h.heal_kv_quantize_int16(self.Kb, self.kc, self.ks)
-            h.heal_kv_quantize_int16(self.Vb, self.vc, self.vs)
-            rec("kv_writer", 1)
-        if only in (None, "attention"):
-            rec("attention", 0)
-            h.heal_attention_int16(self.qc, self.qs, self.kc, self.ks, self.vc, self.vs, self.kv_len,
-                                   KV["D"] ** -0.5, self.out, self.aws)
-            rec("attention", 1)
+                ev[name][0].record()
+            fn()
+            if ev is not None:
+                ev[name][1].record()
 
     LAUNCHES_PER_STEP = 1 + 3 * 2 * len(DECODE_M) + 3 * 2 * CHAIN + 3 + 2
 
@@ -517,8 +504,9 @@ def arm_config(n):
                         "(K=N=4096), the INT16 KV writer and INT16 decode attention "
                         "(B=8, 32q/8kv heads, D=128, context 8192)",
             "parallelism": f"independent shards x{n}" if n > 1 else "single GPU",
-            "l2": "cold: inputs larger than L2 or separate buffers with >1 GB of other traffic "
-                  "between reuses"}
+            "l2": "cold: before every part of a step, outside its events, a 256 MB buffer is written "
+                  "and another 256 MB read (the part starts with none of its inputs in L2 and no dirty "
+                  "line of another part); part order: KV writer, prefill, attention, decode GEMMs"}
 
 
 def reference_arm(args):
@@ -623,7 +611,7 @@ def main():
 
     dec_names = ([f"decode{m}" for m in DECODE_M] + [f"decode{m}_presplit" for m in DECODE_M] +
                  [f"decode{m}_w16" for m in DECODE_M] +
-                 ["decode1_chain", "decode1_chain_presplit", "decode1_chain_w16"])
+                 ["decode1_chain", "decode1_chain_presplit", "decode1_chain_w16", "ref_copy_67MB"])
     names = ["prefill"] + dec_names + ["kv_writer", "attention"]
     if args.only:
         keep = {"prefill": ["prefill"], "decode": dec_names,
@@ -693,6 +681,11 @@ def main():
         t = part_ms[f"decode{m}_w16"] / 1e3 / K
         dec[f"M{m}_fp16_weights_two_products"] = {"gbs": u["decode16_bytes"][m] / t / 1e9, "us": 1e6 * t,
                                                   "frac_hbm": u["decode16_bytes"][m] / t / 1e9 / hbm}
+    t = part_ms["ref_copy_67MB"] / 1e3 / K
+    dec["streaming_copy_reference"] = {
+        "us": 1e6 * t, "gbs": REF_COPY_BYTES / t / 1e9, "frac_hbm": REF_COPY_BYTES / t / 1e9 / hbm,
+        "note": "torch device copy, 32 MB read + 32 MB written (a decode GEMM's weight bytes), timed in the step "
+                "like the decode parts: what one launch of this size streams at"}
     for suffix, key, nb in (("", "M1_chain", "chain_bytes"), ("_presplit", "M1_chain_presplit_weights", "chain_bytes"),
                             ("_w16", "M1_chain_fp16_weights_two_products", "chain16_bytes")):
         t = part_ms[f"decode1_chain{suffix}"] / 1e3 / K

@@ -82,8 +82,8 @@ struct GemmArgs {
   int static_op;            // 0: none; 1: kernel-A, 2: kernel-B is not written by the kernels
                             // before this one (its first stages may be requested early)
   unsigned int* status;     // device status word
-  long long out_extent;
-  int ws_tma;               // split K, BN = 64: chunk tiles go to ws by TMA store (map in the B-lo slot)     // elements of `out` the call may write (debug-build checks)
+  long long out_extent;      // elements of `out` the call may write (debug-build checks)
+  int ws_tma;               // split K, BN = 64: chunk tiles go to ws by TMA store (map in the B-lo slot)
   long long ws_elems;       // FP32 elements of the workspace (debug-build checks)
 };
 

@@ -10,6 +10,9 @@
 // absmax is a shuffle reduction inside the group.  Every decision is taken in FP32:
 //   inv = 32767 / absmax (IEEE division), q = rint(x * inv) clamped to +-32767,
 //   s = absmax / 32767; an all-zero row gives q = 0 and s = 0.
+// A unit's divisions (two per row) are spread over the warp's lanes, one division
+// sequence per 16 rows, and rint is an FP32 add of 1.5 * 2^23 whose low 16 bits are
+// the code: the per-value work is a multiply, an add and half a byte permute.
 // HBM-bound: 2 (bf16) or 4 (fp32) bytes read and 2 bytes written per value.
 #include <cuda_bf16.h>
 
@@ -19,7 +22,7 @@
 namespace heal {
 
 template <int L, bool BF16>
-__global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restrict__ x, int B, int T, int H,
+__global__ void __launch_bounds__(256, 4) heal_kv_quant_kernel(const void* __restrict__ x, int B, int T, int H,
                                                             long long sb, long long st, long long sh,
                                                             int16_t* __restrict__ q, float* __restrict__ sc,
                                                             int Tmax, int t_off, unsigned int* status) {
@@ -67,52 +70,84 @@ __global__ void __launch_bounds__(256) heal_kv_quant_kernel(const void* __restri
           if constexpr (!BF16) raw[u][1] = make_uint4(0, 0, 0, 0);
         }
       }
+      // widen to FP32 and take each row's absmax (a shuffle reduction inside the group)
+      float vv[kUnroll][8];
+      float mrow[kUnroll];
 #pragma unroll
       for (int u = 0; u < kUnroll; ++u) {
-        float vv[8];
         if constexpr (BF16) {
           // bf16 -> fp32 is exact: the bf16 bits are the top half of the fp32 pattern
           const uint32_t w[4] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w};
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            vv[2 * j] = __uint_as_float(w[j] << 16);
-            vv[2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
+            vv[u][2 * j] = __uint_as_float(w[j] << 16);
+            vv[u][2 * j + 1] = __uint_as_float(w[j] & 0xFFFF0000u);
           }
         } else {
           const uint32_t w[8] = {raw[u][0].x, raw[u][0].y, raw[u][0].z, raw[u][0].w,
                                  raw[u][1].x, raw[u][1].y, raw[u][1].z, raw[u][1].w};
 #pragma unroll
-          for (int j = 0; j < 8; ++j) vv[j] = __uint_as_float(w[j]);
+          for (int j = 0; j < 8; ++j) vv[u][j] = __uint_as_float(w[j]);
         }
         float m = 0.0f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(vv[j]));
+        for (int j = 0; j < 8; ++j) m = fmaxf(m, fabsf(vv[u][j]));
 #pragma unroll
         for (int o = L / 2; o >= 1; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        mrow[u] = m;
+      }
+      // The unit's IEEE divisions, spread over the lanes instead of repeated in every lane
+      // of a row group: task j = 2 * row + kind, kind 0 -> inv = 32767 / absmax, kind 1 ->
+      // s = absmax / 32767 (row = u * kRowsPerPass + group; 0 for an all-zero row).
+      constexpr int kTasks = 2 * kGroupRows;
+      constexpr int kSeq = (kTasks + 31) / 32;
+      float res[kSeq];
+#pragma unroll
+      for (int sq = 0; sq < kSeq; ++sq) {
+        const int j = sq * 32 + lane;
+        const int row = (j >> 1) < kGroupRows ? (j >> 1) : kGroupRows - 1;
+        const int ur = row / kRowsPerPass, gr = row % kRowsPerPass;
+        float mm = 0.0f;
+#pragma unroll
+        for (int u = 0; u < kUnroll; ++u) {
+          const float tv = __shfl_sync(0xffffffffu, mrow[u], gr * L);
+          if (u == ur) mm = tv;
+        }
+        const bool kind_s = (j & 1) != 0;
+        res[sq] = mm > 0.0f ? __fdiv_rn(kind_s ? mm : 32767.0f, kind_s ? 32767.0f : mm) : 0.0f;
+        const int h = h0 + row;
+        if (kind_s && j < kTasks && h < H) {
+          const long long row_out = ((long long)b * H + h) * Tmax + t_off + t;
+          if (HEAL_DCHECK(row_out < (long long)B * H * Tmax && t_off + t < Tmax, status, 401)) sc[row_out] = res[sq];
+        }
+      }
+      // Codes.  |x * inv| <= 32767 (1 + 2^-24) rounded, so rint never leaves [-32767, 32767]
+      // and the clamp of the definition is never active.  rint (ties to even) is taken by
+      // adding 1.5 * 2^23: the sum lies in [2^23, 2^24), where the FP32 spacing is 1, so its
+      // round-to-nearest-even is 1.5 * 2^23 + rint(y) and the low 16 bits of its pattern are
+      // rint(y) in two's complement.  (A row with absmax 0 has inv = 0 and codes 0.)
+#pragma unroll
+      for (int u = 0; u < kUnroll; ++u) {
+        const int jt = 2 * (u * kRowsPerPass + grp);   // the task holding this row's inv
+        float inv = 0.0f;
+#pragma unroll
+        for (int sq = (2 * u * kRowsPerPass) / 32; sq <= (2 * (u + 1) * kRowsPerPass - 1) / 32 && sq < kSeq; ++sq) {
+          const float tv = __shfl_sync(0xffffffffu, res[sq], jt & 31);
+          if ((jt >> 5) == sq) inv = tv;
+        }
         const int h = h0 + u * kRowsPerPass + grp;
         if (h >= H) continue;
         const long long row_out = ((long long)b * H + h) * Tmax + t_off + t;
-        int qv[8];
-        if (m > 0.0f) {
-          const float inv = __fdiv_rn(32767.0f, m);
+        uint32_t c[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const int qi = __float2int_rn(__fmul_rn(vv[j], inv));
-            qv[j] = qi > 32767 ? 32767 : (qi < -32767 ? -32767 : qi);
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 8; ++j) qv[j] = 0;
-        }
+        for (int j = 0; j < 8; ++j) c[j] = __float_as_uint(__fadd_rn(__fmul_rn(vv[u][j], inv), 12582912.0f));
         uint4 pk;
-        pk.x = (uint32_t)(qv[0] & 0xFFFF) | ((uint32_t)qv[1] << 16);
-        pk.y = (uint32_t)(qv[2] & 0xFFFF) | ((uint32_t)qv[3] << 16);
-        pk.z = (uint32_t)(qv[4] & 0xFFFF) | ((uint32_t)qv[5] << 16);
-        pk.w = (uint32_t)(qv[6] & 0xFFFF) | ((uint32_t)qv[7] << 16);
-        if (HEAL_DCHECK(row_out < (long long)B * H * Tmax && t_off + t < Tmax && h < H, status, 400)) {
+        pk.x = __byte_perm(c[0], c[1], 0x5410);
+        pk.y = __byte_perm(c[2], c[3], 0x5410);
+        pk.z = __byte_perm(c[4], c[5], 0x5410);
+        pk.w = __byte_perm(c[6], c[7], 0x5410);
+        if (HEAL_DCHECK(row_out < (long long)B * H * Tmax && t_off + t < Tmax, status, 400))
           __stcs(reinterpret_cast<uint4*>(q + row_out * D + sub * 8), pk);
-          if (sub == 0) sc[row_out] = m > 0.0f ? __fdiv_rn(m, 32767.0f) : 0.0f;
-        }
       }
     }
   }

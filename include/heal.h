@@ -157,7 +157,8 @@ size_t heal_gemm_workspace_bytes(int M, int N, int K, const heal_gemm_opts_t* op
  * Per (token, head) row: absmax = max|x|, inv = fp32(32767/absmax),
  * q = clamp(rint(fp32(x*inv)), +-32767), s = fp32(absmax/32767); an all-zero row gives
  * q = 0, s = 0.  D must be a power of two in [8, 256]; x, q_cache 16-byte aligned;
- * strides multiples of 8 elements.  t_offset + T <= Tmax.                              */
+ * strides multiples of 8 elements.  t_offset + T <= Tmax.  Rows holding a NaN or an
+ * infinity get unspecified codes (the definition above does not cover them).          */
 heal_status_t heal_kv_quantize_int16(const void* x, int x_is_bf16,
                                      int B, int T, int H, int D,
                                      int64_t x_stride_batch, int64_t x_stride_tok,

@@ -60,6 +60,39 @@ def test_kv_quantize_bit_exact(in_dtype, D):
     assert np.all(sn[:, :, :t_off] == -1.0) and np.all(sn[:, :, t_off + T:] == -1.0)
 
 
+@pytest.mark.parametrize("in_dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("D,H", [(8, 3), (16, 5), (32, 12), (128, 12), (128, 40), (256, 5)])
+def test_kv_quantize_head_dims_and_ragged_head_groups(in_dtype, D, H):
+    """Every row-group width (8 lanes' worth of values per lane group: D = 8 .. 256) and
+    head counts that leave the last group of a token partly empty; one row of half-integer
+    products (absmax 65534 -> inv = 0.5 exactly, odd inputs) checks that ties round to
+    even."""
+    d = dev()
+    B, T, Tmax, t_off = 2, 67, 80, 5
+    g = torch.Generator().manual_seed(1000 + D + H)
+    x = (torch.randn(B, T, H, D, generator=g) * torch.exp(torch.randn(B, T, H, 1, generator=g))).to(in_dtype)
+    x[1, 2, H - 1] = 0
+    if in_dtype == torch.float32:
+        row = torch.arange(D, dtype=torch.float32) * 2 - (D - 1)     # odd values
+        row[0] = 65534.0
+        x[0, 1, 0] = row
+    qc = torch.full((B, H, Tmax, D), 7, dtype=torch.int16, device=d)
+    sc = torch.full((B, H, Tmax), -1.0, dtype=torch.float32, device=d)
+    heal.heal_kv_quantize_int16(x.to(d), qc, sc, t_offset=t_off)
+    status_ok()
+    q_ref, s_ref = Q.quantize_kv(x.float().numpy())
+    qn, sn = to_np(qc), to_np(sc)
+    np.testing.assert_array_equal(qn[:, :, t_off:t_off + T], q_ref)
+    np.testing.assert_array_equal(sn[:, :, t_off:t_off + T].view(np.uint32), s_ref.view(np.uint32))
+    assert np.all(qn[:, :, :t_off] == 7) and np.all(qn[:, :, t_off + T:] == 7)
+    assert np.all(sn[:, :, :t_off] == -1.0) and np.all(sn[:, :, t_off + T:] == -1.0)
+    if in_dtype == torch.float32:
+        # 0.5 * odd k is a tie; the even neighbour wins
+        k = np.arange(D) * 2 - (D - 1)
+        want = np.rint(k[1:] * 0.5).astype(np.int16)
+        assert np.array_equal(qn[0, 0, t_off + 1, 1:], want) and qn[0, 0, t_off + 1, 0] == 32767
+
+
 def test_kv_quantize_strided_input_and_full_size():
     """Config-sized K cache (B=8, T=8192, Hkv=8, D=128) from a strided view: bit-exact on
     every row."""
