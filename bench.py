@@ -705,32 +705,44 @@ def main():
             reps = max(10, min(K, 50))
             p0, p1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             torch.cuda.synchronize()
-            p0.record(stream)
-            for _ in range(reps):
-                g.replay()
-            p1.record(stream)
-            torch.cuda.synchronize()
+            with ClockSampler(smi_index) as cs:
+                p0.record(stream)
+                for _ in range(reps):
+                    g.replay()
+                p1.record(stream)
+                torch.cuda.synchronize()
             t = p0.elapsed_time(p1) / 1e3 / reps
             if ws > 1:
                 t = max_over_ranks([t], device=dev)[0]
             del g
-            return t, reps
-        t_pre, reps = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.Whi, wl.C, b_lo=wl.Wlo))
+            return t, reps, cs.summary()
+
+        def pct_at_clock(flop_mma, t, ckx):
+            """% of the 16-bit peak that applies at the clock sampled during this loop (a
+            back-to-back GEMM loop can run into the power cap, unlike the mixed step)."""
+            full = bool(ckx.get("sm_mhz") and ckx.get("sm_max_mhz") and ckx["sm_mhz"] >= 0.9 * ckx["sm_max_mhz"])
+            pk = peak_burst if full or not ckx.get("sm_mhz") else peak_sus
+            return 100.0 * flop_mma / t / 1e12 / pk, ("bf16_tflops (burst)" if pk == peak_burst else
+                                                    "bf16_tflops_sustained")
+        t_pre, reps, ck_pre = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.Whi, wl.C, b_lo=wl.Wlo))
+        pc, pn = pct_at_clock(u["prefill_flop_mma"], t_pre, ck_pre)
         presplit = {"tflops_effective": ws * u["prefill_flop_eff"] / t_pre / 1e12,
-                    "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_pre / 1e12 / peak_tc,
+                    "pct_of_16bit_peak": pc, "peak": pn, "clocks": ck_pre,
                     "ms": 1e3 * t_pre, "replays": reps,
                     "note": "the same product with W split once into hi/lo beforehand (static weights); "
                             "timed separately after the step"}
-        t_sp, reps = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.W, wl.C, workspace=wl.wsp,
-                                                                   b_split_pass=True))
-        t_16, reps16 = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.W16, wl.C, b_16bit=True))
+        t_sp, reps, ck_sp = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.W, wl.C, workspace=wl.wsp,
+                                                                          b_split_pass=True))
+        t_16, reps16, ck_16 = time_call(lambda: heal.heal_gemm_compensated(wl.X, wl.W16, wl.C, b_16bit=True))
+        pc16, pn16 = pct_at_clock((2.0 / 3.0) * u["prefill_flop_mma"], t_16, ck_16)
         w16 = {"tflops_effective": ws * u["prefill_flop_eff"] / t_16 / 1e12,
-               "pct_of_16bit_peak": 100.0 * (2.0 / 3.0) * u["prefill_flop_mma"] / t_16 / 1e12 / peak_tc,
+               "pct_of_16bit_peak": pc16, "peak": pn16, "clocks": ck_16,
                "ms": 1e3 * t_16, "replays": reps16,
                "note": "the two-product form with FP16 weights (only X split; 2 MMAs); timed separately "
                        "after the step"}
+        pcs, pns = pct_at_clock(u["prefill_flop_mma"], t_sp, ck_sp)
         splitpass = {"tflops_effective": ws * u["prefill_flop_eff"] / t_sp / 1e12,
-                     "pct_of_16bit_peak": 100.0 * u["prefill_flop_mma"] / t_sp / 1e12 / peak_tc,
+                     "pct_of_16bit_peak": pcs, "peak": pns, "clocks": ck_sp,
                      "ms": 1e3 * t_sp, "replays": reps,
                      "note": "the same product with B split by a streaming pass into a workspace first "
                              "(b_split_pass; B's parts go through HBM); timed separately after the step"}
