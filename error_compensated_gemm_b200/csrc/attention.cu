@@ -8,11 +8,13 @@
 // with S_hh = sum qh*kh, S_x = sum (qh*kl + ql*kh), S_ll = sum ql*kl.  QK^T runs these four
 // byte products on the integer tensor cores (mma.sync m16n8k32, signed hi bytes and
 // unsigned lo bytes, exact int32 accumulation: for head_dim <= 128 no partial sum exceeds
-// 2^24); the three sums are combined in int64.
-//   logit = fp32( (double(S_int) * (double(s_q) * double(s_k))) * double(softmax_scale) )
-// FP32 online softmax in base 2.  P is folded with the per-token V scale and a per-block
-// power of two 2^E (chosen so the block's largest V scale times 2^E lies in [32, 64)),
-// then split into FP16 P_hi and the FP16 residual r = P - P_hi; the byte-split V
+// 2^24); the test hook receives their exact int64 combination.  The logit, in log2 units:
+//   x = fp32( fp32(fp32(S_int) * s_k) * fp32(fp32(s_q * softmax_scale) * log2(e)) )
+// with fp32(S_int) = fp32(65536*S_hh + fp32(256*S_x + S_ll)) (S_hh exact in FP32; two
+// roundings), as in the prefill kernel.  FP32 online softmax in base 2.  P is folded with
+// the per-token V scale and a per-block power of two 2^E (chosen so the block's largest V
+// scale times 2^E lies in [32, 64)), then split into FP16 P_hi and the FP16 residual
+// r = P - P_hi; the byte-split V
 // (hi = v >> 8, lo = v & 255, each an exact FP16 value) meets (256*P_hi, P_hi, 256*r, r) in
 // four FP16 tensor-core products that accumulate into one FP32 accumulator:
 // sum 256*hi*P + lo*P = v*P.  These are the two FP16 tensors the INT16 value is unpacked
@@ -73,6 +75,11 @@ struct AttnArgs {
 
 // -------- INT16 byte split into FP16 pairs (bit construction, exact) --------
 // Two int16 values packed in x -> (lo0, lo1) and (hi0, hi1) as half2.
+// n (|n| < 2^22) as FP32, exactly: the integer lands in the mantissa of 1.5 * 2^23.
+__device__ __forceinline__ float small_int_to_float(int n) {
+  return __fsub_rn(__int_as_float(0x4B400000 + n), 12582912.0f);
+}
+
 __device__ __forceinline__ uint32_t lo_pair(uint32_t x) {
   // 0x6400 | b is the FP16 value 1024 + b for b in [0, 1023]
   const uint32_t u = (x & 0x00FF00FFu) | 0x64006400u;
@@ -267,7 +274,7 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
     // depend on the order of its terms).
     const int w = warp;
     const int tw = w * 16;                    // this warp's first token inside the tile
-    float sq[2] = {0.0f, 0.0f};
+    float sqc[2] = {0.0f, 0.0f};             // fp32(fp32(s_q * softmax_scale) * log2(e)) per row
     int pos[2] = {0, 0};
     float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
     int E_run = 0;                            // power of two folded into P (decreases only)
@@ -320,7 +327,9 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
           const int r = qc + e;
           const bool real = r < R;
           const int tq = real ? r / a.G : 0, gq = real ? r % a.G : 0;
-          sq[e] = real ? __ldg(a.qs + ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq)) : 0.0f;
+          sqc[e] = real ? __fmul_rn(__fmul_rn(__ldg(a.qs + ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq)),
+                                              a.scale), kLog2e)
+                        : 0.0f;
           pos[e] = klen - a.Tq + tq;
         }
         // B fragments of Q^T (query row g8), byte-split, one table per CTA:
@@ -412,8 +421,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
           const int i = 2 * th + e;
           const int t = t0 + tw + th * 8 + g8;
           const int r = qc + e;
-          const long long S = ((long long)shh[i] << 16) + (((long long)sxa[i] + (long long)sxb[i]) << 8) +
-                              (long long)sll[i];
+          // S = 65536*S_hh + low, low = 256*S_x + S_ll (|low| < 2^31 for head_dim <= 128)
+          const int low = (sxa[i] + sxb[i]) * 256 + sll[i];
           const bool real = r < R;
           const bool vis = real && t < klen && (!a.causal || t <= pos[e]);
           float xv;
@@ -422,10 +431,10 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
           } else if (!vis) {
             xv = -INFINITY;
           } else {
-            const double coef = (double)sq[e] * (double)skr[th];
-            const float lg = (float)(((double)S * coef) * (double)a.scale);
-            xv = __fmul_rn(lg, kLog2e);
+            const float sf = __fmaf_rn(small_int_to_float(shh[i]), 65536.0f, __int2float_rn(low));
+            xv = __fmul_rn(__fmul_rn(sf, skr[th]), sqc[e]);
             if (a.qk_out) {
+              const long long S = (long long)shh[i] * 65536LL + (long long)low;
               const int tq = r / a.G, gq = r % a.G;
               const long long qi = ((long long)(b * a.Hq + hkv * a.G + gq) * a.Tq + tq) * a.Tmax + t;
               if (HEAL_DCHECK(qi < (long long)a.B * a.Hq * a.Tq * a.Tmax && t < a.Tmax, a.status, 251))

@@ -178,9 +178,9 @@ heal_status_t heal_kv_quantize_int16(const void* x, int x_is_bf16,
  * four 8-bit integer tensor-core products, combined in int64); FP32 online softmax; PV
  * with P split into two FP16 parts and V byte-split into two exact FP16 values.
  * Two kernels, chosen by the number of query rows per KV head, R = (Hq/Hkv) * Tq:
- *   R <= 8 (decode): logit = fp32(S_int * (s_q * s_k) * softmax_scale) evaluated in
- *     double; the context is cut into chunks whose partial results are merged in
- *     ascending chunk order.
+ *   R <= 8 (decode): logit * log2(e) = fp32(fp32(fp32(S_int) * s_k) *
+ *     fp32(s_q * softmax_scale * log2(e))) in FP32, as in the prefill kernel; the context
+ *     is cut into chunks whose partial results are merged in ascending chunk order.
  *   R > 8 (prefill, D = 128 only): 128 query rows per tile on the tcgen05 tensor cores;
  *     logit * log2(e) = fp32(fp32(S_int) * s_k) * fp32(s_q * softmax_scale * log2(e))
  *     in FP32; a conversion pass first writes the byte planes of Q, K and V into the
