@@ -165,7 +165,10 @@ __device__ __forceinline__ float* slot_ptr(float* ws, int c, int p, int R, int D
   return ws + (size_t)(c + p) * (size_t)R * (size_t)(D + 2);
 }
 
-template <int D>
+// PK (R <= 4): the PV B fragment packs P_hi of the (at most four) query rows into columns
+// 0-3 and the residual r into columns 4-7, so each V fragment meets two FP16 MMAs instead
+// of four; the two column halves of the accumulator are added when the partial is written.
+template <int D, bool PK>
 __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                        const __grid_constant__ CUtensorMap tmV,
                                                                        const AttnArgs a) {
@@ -503,8 +506,9 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
       }
 
       // ---- P' = P * s_v * 2^E (S^T layout), moved to the B layout of PV: lane (g8, c)
-      // needs tokens 2c, 2c + 1, 2c + 8, 2c + 9 of query row g8.  Token 2c + jj lives in lane
-      // 4 * (2c + jj) + g8 / 2 (halves th = 0 / 1 for +0 / +8), query row g8 in slot g8 & 1.
+      // needs tokens 2c, 2c + 1, 2c + 8, 2c + 9 of query row g8 (PK: of row g8 & 3).  Token
+      // 2c + jj lives in lane 4 * (2c + jj) + row / 2 (halves th = 0 / 1 for +0 / +8), the row
+      // in slot row & 1.
       float pp[2][2];
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
@@ -519,7 +523,7 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
         const bool odd = (g8 & 1) != 0;
 #pragma unroll
         for (int jj = 0; jj < 2; ++jj) {
-          const int src = 4 * (2 * cq + jj) + (g8 >> 1);
+          const int src = 4 * (2 * cq + jj) + ((PK ? (g8 & 3) : g8) >> 1);
 #pragma unroll
           for (int th = 0; th < 2; ++th) {
             const float v0 = __shfl_sync(0xffffffffu, pp[th][0], src);
@@ -529,7 +533,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
         }
       }
       // FP16 P_hi and residual r = P' - P_hi: the B fragments of PV (the PV warps form the
-      // 256x copies themselves)
+      // 256x copies themselves).  PK: columns 4-7 (g8 >= 4) carry r, so both slots hold
+      // the column's own part.
       uint32_t ph_[2], pr_[2];
 #pragma unroll
       for (int th = 0; th < 2; ++th) {
@@ -538,6 +543,7 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
         const __half2 rr = __floats2half2_rn(__fsub_rn(pt[th][0], hf.x), __fsub_rn(pt[th][1], hf.y));
         ph_[th] = *reinterpret_cast<const uint32_t*>(&h);
         pr_[th] = *reinterpret_cast<const uint32_t*>(&rr);
+        if (PK && g8 >= 4) ph_[th] = pr_[th];
       }
       // hand the block to the PV warps (the buffer is free once they finished block j - 2)
       if (!mbar_wait(&pfree[jb], jph ^ 1u, abort_flag, a.status, 213)) {
@@ -574,13 +580,20 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
 
   auto finalize_o = [&](int p) {
     float* sl = slot_ptr(a.ws, c, p, R, D);
+    if constexpr (PK) {
+      // columns 4-7 (lanes with c >= 2) hold the residual part of rows 0-3
+#pragma unroll
+      for (int dl = 0; dl < kDT; ++dl)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) om[dl][e] = __fadd_rn(om[dl][e], __shfl_xor_sync(0xffffffffu, om[dl][e], 2));
+    }
 #pragma unroll
     for (int dl = 0; dl < kDT; ++dl)
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
         const int d = (v * kDT + dl) * 16 + g8 + ((e >> 1) << 3);
         const int r = qc + (e & 1);
-        if (r < R && HEAL_DCHECK((long long)(sl + r * D + d - a.ws) < a.ws_elems, a.status, 252))
+        if (r < R && (!PK || qc < 4) && HEAL_DCHECK((long long)(sl + r * D + d - a.ws) < a.ws_elems, a.status, 252))
           sl[r * D + d] = mul_pow2(om[dl][e], -E_run);   // true units (x 2^-E_run)
         om[dl][e] = 0.0f;
       }
@@ -608,7 +621,8 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
     }
     const uint32_t vst = smem_u32(stages + s * kStageBytes) + kTileBytes;
     // rescale O^T columns qc, qc + 1 by the block's softmax step and change of 2^E
-    const float a0 = meta[jb * 16 + qc], a1 = meta[jb * 16 + qc + 1];
+    const int qr = PK ? (qc & 3) : qc;                 // the query rows of this lane's columns
+    const float a0 = meta[jb * 16 + qr], a1 = meta[jb * 16 + qr + 1];
     E_run = __float_as_int(meta[jb * 16 + 8]);
     if (!__all_sync(0xffffffffu, a0 == 1.0f && a1 == 1.0f)) {
 #pragma unroll
@@ -626,7 +640,12 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
       // 256 * P_hi and 256 * r: exact (powers of two; |P'| < 64)
       const __half2 k256 = __half2half2(__ushort_as_half(0x5C00));
       uint4 fh, fr;                                                  // (256 x, x) of P_hi / r
-      {
+      if constexpr (PK) {
+        const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&f.x), k256);
+        const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&f.y), k256);
+        fh = make_uint4(*reinterpret_cast<const uint32_t*>(&h0), *reinterpret_cast<const uint32_t*>(&h1), f.x, f.y);
+        fr = fh;
+      } else {
         const __half2 h0 = __hmul2(*reinterpret_cast<const __half2*>(&f.x), k256);
         const __half2 h1 = __hmul2(*reinterpret_cast<const __half2*>(&f.y), k256);
         const __half2 r0 = __hmul2(*reinterpret_cast<const __half2*>(&f.z), k256);
@@ -647,8 +666,10 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
         const uint32_t l0 = lo_pair(r0), l1 = lo_pair(r1), l2 = lo_pair(r2), l3 = lo_pair(r3);
         mma16816(om[dl], h0, h1, h2, h3, fh.x, fh.y);
         mma16816(om[dl], l0, l1, l2, l3, fh.z, fh.w);
-        mma16816(om[dl], h0, h1, h2, h3, fr.x, fr.y);
-        mma16816(om[dl], l0, l1, l2, l3, fr.z, fr.w);
+        if constexpr (!PK) {
+          mma16816(om[dl], h0, h1, h2, h3, fr.x, fr.y);
+          mma16816(om[dl], l0, l1, l2, l3, fr.z, fr.w);
+        }
       }
     }
     __syncwarp();
@@ -785,17 +806,29 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
   const int di = (D == 128) ? 0 : 1;
   int per_sm = per_sm_cache[dev][di];
   if (per_sm == 0) {
-    if (cudaFuncSetAttribute(heal_attn_decode_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    if (cudaFuncSetAttribute(heal_attn_decode_kernel<128, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              attn_smem_bytes<128>()) != cudaSuccess ||
-        cudaFuncSetAttribute(heal_attn_decode_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        cudaFuncSetAttribute(heal_attn_decode_kernel<128, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn_smem_bytes<128>()) != cudaSuccess ||
+        cudaFuncSetAttribute(heal_attn_decode_kernel<64, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             attn_smem_bytes<64>()) != cudaSuccess ||
+        cudaFuncSetAttribute(heal_attn_decode_kernel<64, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              attn_smem_bytes<64>()) != cudaSuccess)
       return HEAL_ERR_CUDA;
-    if (D == 128)
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<128>, kAttnThreads,
+    // both forms of a head size are built for the same residency (launch bounds)
+    int p0 = 0, p1 = 0;
+    if (D == 128) {
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p0, heal_attn_decode_kernel<128, false>, kAttnThreads,
                                                     attn_smem_bytes<128>());
-    else
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, heal_attn_decode_kernel<64>, kAttnThreads,
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p1, heal_attn_decode_kernel<128, true>, kAttnThreads,
+                                                    attn_smem_bytes<128>());
+    } else {
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p0, heal_attn_decode_kernel<64, false>, kAttnThreads,
                                                     attn_smem_bytes<64>());
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&p1, heal_attn_decode_kernel<64, true>, kAttnThreads,
+                                                    attn_smem_bytes<64>());
+    }
+    per_sm = p0 < p1 ? p0 : p1;
     if (per_sm < 1) per_sm = 1;
     per_sm_cache[dev][di] = per_sm;
   }
@@ -820,13 +853,15 @@ heal_status_t attention_launch(const int16_t* q, const float* qs, const int16_t*
                          CU_TENSOR_MAP_SWIZZLE_128B))
     return HEAL_ERR_CUDA;
   cudaError_t e;
+  const bool pk = R <= 4;
+  const dim3 g(a.grid), t(kAttnThreads);
   if (D == 128) {
-    e = launch_pdl(heal_attn_decode_kernel<128>, dim3(a.grid), dim3(kAttnThreads), (size_t)attn_smem_bytes<128>(), stream,
-                   tk, tv, a);
+    e = pk ? launch_pdl(heal_attn_decode_kernel<128, true>, g, t, (size_t)attn_smem_bytes<128>(), stream, tk, tv, a)
+           : launch_pdl(heal_attn_decode_kernel<128, false>, g, t, (size_t)attn_smem_bytes<128>(), stream, tk, tv, a);
     if (e == cudaSuccess) e = launch_pdl(heal_attn_combine_kernel<128>, dim3(B * Hkv * R), dim3(128), 0, stream, a);
   } else {
-    e = launch_pdl(heal_attn_decode_kernel<64>, dim3(a.grid), dim3(kAttnThreads), (size_t)attn_smem_bytes<64>(), stream,
-                   tk, tv, a);
+    e = pk ? launch_pdl(heal_attn_decode_kernel<64, true>, g, t, (size_t)attn_smem_bytes<64>(), stream, tk, tv, a)
+           : launch_pdl(heal_attn_decode_kernel<64, false>, g, t, (size_t)attn_smem_bytes<64>(), stream, tk, tv, a);
     if (e == cudaSuccess) e = launch_pdl(heal_attn_combine_kernel<64>, dim3(B * Hkv * R), dim3(64), 0, stream, a);
   }
   if (e != cudaSuccess) return HEAL_ERR_CUDA;

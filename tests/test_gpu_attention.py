@@ -116,6 +116,15 @@ def test_multi_query_causal():
     check(q, qs, kq, kss, vq, vss, [192, 130], 128 ** -0.5, causal=True)
 
 
+@pytest.mark.parametrize("Hq,Hkv,Tq", [(6, 2, 1), (6, 2, 2), (8, 2, 1), (10, 2, 1)])
+def test_decode_row_counts_packed_and_unpacked(Hq, Hkv, Tq):
+    """R = (Hq/Hkv)*Tq query rows per KV head: 3 and 4 take the form whose PV fragments carry
+    P_hi in columns 0-3 and the residual in columns 4-7; 6 takes the four-product form; 5
+    rows run through the same form."""
+    q, qs, kq, kss, vq, vss = make_inputs(B=2, Hq=Hq, Hkv=Hkv, D=128, T=320, Tq=Tq)
+    check(q, qs, kq, kss, vq, vss, [320, 199], 128 ** -0.5, causal=Tq > 1)
+
+
 def test_mha_and_many_blocks():
     q, qs, kq, kss, vq, vss = make_inputs(B=1, Hq=4, Hkv=4, D=128, T=4096)
     check(q, qs, kq, kss, vq, vss, [4001], 128 ** -0.5)
