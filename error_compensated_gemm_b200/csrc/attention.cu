@@ -11,7 +11,8 @@
 // 2^24); the test hook receives their exact int64 combination.  The logit, in log2 units:
 //   x = fp32( fp32(fp32(S_int) * s_k) * fp32(fp32(s_q * softmax_scale) * log2(e)) )
 // with fp32(S_int) = fp32(65536*S_hh + fp32(256*S_x + S_ll)) (S_hh exact in FP32; two
-// roundings), as in the prefill kernel.  FP32 online softmax in base 2.  P is folded with
+// roundings), as in the prefill kernel.  FP32 online softmax in base 2 (2^x by
+// ex2.approx, as in the prefill kernel).  P is folded with
 // the per-token V scale and a per-block power of two 2^E (chosen so the block's largest V
 // scale times 2^E lies in [32, 64)), then split into FP16 P_hi and the FP16 residual
 // r = P - P_hi; the byte-split V
@@ -75,11 +76,6 @@ struct AttnArgs {
 
 // -------- INT16 byte split into FP16 pairs (bit construction, exact) --------
 // Two int16 values packed in x -> (lo0, lo1) and (hi0, hi1) as half2.
-// n (|n| < 2^22) as FP32, exactly: the integer lands in the mantissa of 1.5 * 2^23.
-__device__ __forceinline__ float small_int_to_float(int n) {
-  return __fsub_rn(__int_as_float(0x4B400000 + n), 12582912.0f);
-}
-
 __device__ __forceinline__ uint32_t lo_pair(uint32_t x) {
   // 0x6400 | b is the FP16 value 1024 + b for b in [0, 1023]
   const uint32_t u = (x & 0x00FF00FFu) | 0x64006400u;
@@ -476,9 +472,9 @@ __global__ void __launch_bounds__(kAttnThreads, kMinBlocks) heal_attn_decode_ker
           alpha[e] = 1.0f;
           pv[0][e] = pv[1][e] = 0.0f;
         } else {
-          alpha[e] = (m_run[e] == -INFINITY) ? 0.0f : exp2f(m_run[e] - m_new);
+          alpha[e] = (m_run[e] == -INFINITY) ? 0.0f : fast_exp2(m_run[e] - m_new);
 #pragma unroll
-          for (int th = 0; th < 2; ++th) pv[th][e] = (x[th][e] == -INFINITY) ? 0.0f : exp2f(x[th][e] - m_new);
+          for (int th = 0; th < 2; ++th) pv[th][e] = (x[th][e] == -INFINITY) ? 0.0f : fast_exp2(x[th][e] - m_new);
         }
         l_run[e] = __fadd_rn(__fmul_rn(l_run[e], alpha[e]), __fadd_rn(pv[0][e], pv[1][e]));
         m_run[e] = m_new;

@@ -239,20 +239,6 @@ __global__ void __launch_bounds__(256) heal_attn_planes_kernel(const PlanesArgs 
   }
 }
 
-// n as a float for |n| < 2^22, exactly: the bits of 1.5 * 2^23 + n, minus 1.5 * 2^23.
-__device__ __forceinline__ float small_int_to_float(int n) {
-  return __fsub_rn(__int_as_float(0x4B400000 + n), 12582912.0f);
-}
-
-// 2^x with the hardware approximation (ex2.approx, relative error about 2^-22; results
-// below 2^-126 flush to zero); 2^-inf = 0.
-__device__ __forceinline__ float fast_exp2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-
-
 __device__ __forceinline__ uint64_t kdesc(uint32_t addr) { return smem_desc_sw128(addr, 16, 1024); }
 __device__ __forceinline__ uint64_t vdesc(uint32_t addr) { return smem_desc_sw128(addr, 8192, 1024); }
 

@@ -127,6 +127,19 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // ---------------------------------------------------------------------------------
 // TMA (tensor tile loads, no multicast)
 // ---------------------------------------------------------------------------------
+// n (|n| < 2^22) as FP32, exactly: the integer lands in the mantissa of 1.5 * 2^23.
+__device__ __forceinline__ float small_int_to_float(int n) {
+  return __fsub_rn(__int_as_float(0x4B400000 + n), 12582912.0f);
+}
+
+// 2^x with the hardware approximation (ex2.approx, relative error about 2^-22; results
+// below 2^-126 flush to zero); 2^-inf = 0.
+__device__ __forceinline__ float fast_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
