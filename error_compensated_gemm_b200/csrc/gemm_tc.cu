@@ -114,6 +114,7 @@ struct Cfg {
 // ---------------------------------------------------------------------------------
 struct WorkIter {
   int tile, chunk, u, u_end, ntiles, nc, splitk;
+  int step, dtile, dchunk;   // split K: chunk-major units dealt round-robin
   __device__ WorkIter(const GemmArgs& a) {
     ntiles = a.tiles_m * a.tiles_n;
     nc = a.num_chunks;
@@ -125,27 +126,42 @@ struct WorkIter {
       u_end = t * nc + ((r + 1) * nc) / S;
       tile = t;
       chunk = u - t * nc;
+      step = 0;
+      dtile = dchunk = 0;
     } else if (splitk) {
-      const long long total = (long long)ntiles * nc;
-      u = (int)((total * blockIdx.x) / gridDim.x);
-      u_end = (int)((total * (blockIdx.x + 1)) / gridDim.x);
-      tile = u / nc;
-      chunk = u % nc;
+      // unit u = (chunk u / ntiles, tile u % ntiles); CTA c takes u = c, c + grid, ...: the
+      // CTAs working at the same time cover every tile of the same few chunks, i.e. whole
+      // rows of the weights, a contiguous region of memory
+      u = blockIdx.x;
+      u_end = ntiles * nc;
+      step = gridDim.x;
+      dtile = step % ntiles;
+      dchunk = step / ntiles;
+      tile = u % ntiles;
+      chunk = u / ntiles;
     } else {
       tile = blockIdx.x;
       chunk = 0;
       u = 0;
       u_end = 0;
+      step = dtile = dchunk = 0;
     }
   }
   __device__ bool valid() const { return splitk ? (u < u_end) : (tile < ntiles); }
   __device__ void advance() {
-    if (splitk) {
-      // tile = u / nc, chunk = u % nc, kept incrementally (no division per unit)
+    if (splitk && step == 0) {   // chain mode: consecutive chunks of one tile
       ++u;
       if (++chunk == nc) {
         chunk = 0;
         ++tile;
+      }
+    } else if (splitk) {         // tile = u % ntiles, chunk = u / ntiles, kept incrementally
+      u += step;
+      tile += dtile;
+      chunk += dchunk;
+      if (tile >= ntiles) {
+        tile -= ntiles;
+        ++chunk;
       }
     } else if (++chunk == nc) {
       chunk = 0;
