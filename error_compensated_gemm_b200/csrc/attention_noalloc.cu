@@ -18,9 +18,9 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 void* g_addr[kMaxDevices] = {};
 
-// Device address of g_attn_scratch on the current device, looked up once per device (the
-// first call on a device does this; it must not run during stream capture).  The address is
-// kept for the life of the process: it is not looked up again after cudaDeviceReset.
+// Device address of g_attn_scratch on the current device, looked up once per device (by the
+// first call on that device).  The address is kept for the life of the process: it is not
+// looked up again after cudaDeviceReset.
 heal_status_t scratch_address(void** out) {
   int dev = -1;
   if (cudaGetDevice(&dev) != cudaSuccess) {

@@ -218,9 +218,9 @@ size_t heal_attention_workspace_bytes(int B, int Hq, int Tq, int Tmax);
  * HEAL_ATTN_STATIC_SCRATCH_BYTES bytes in libheal.so's own device memory, which every GPU
  * that loads the library holds until the process exits.  This call allocates and frees
  * nothing.
- *   - The first call on a device looks up that array's device address, with that device
- *     current, and keeps it for the life of the process.  Make this first call before any
- *     stream capture.  The kept address does not survive cudaDeviceReset(): after a reset
+ *   - The first call on a device looks up that array's device address (a runtime query),
+ *     with that device current, and keeps it for the life of the process.  The kept
+ *     address does not survive cudaDeviceReset(): after a reset
  *     of a device, do not call this entry point on that device again in the same process.
  *   - All calls share the one array and it keeps the last call's contents.  Nothing in it
  *     needs to start at zero: every partial result a call reads was written earlier in the
