@@ -146,6 +146,9 @@ class Workload:
             # decode parts (torch's copy kernel, not this library's; context only)
             self.ref_src = torch.zeros(REF_COPY_BYTES // 8, device=dev)
             self.ref_dst = torch.zeros(REF_COPY_BYTES // 8, device=dev)
+            # and a plain read of that many bytes (a one-dimensional sum)
+            self.ref_read = torch.zeros(REF_COPY_BYTES // 4, device=dev)
+            self.ref_acc = torch.zeros(1, device=dev)
             for i, m in enumerate(DECODE_M):
                 Xd, Wd = synthetic.gemm_decode(m, seed_x=0 + so, seed_w=1 + so + 10 * (i + 1))
                 ws = torch.empty(max(1, heal.heal_gemm_workspace_bytes(m, 4096, 4096, heal.TILE_SKINNY_SPLITK) // 4),
@@ -235,6 +238,7 @@ class Workload:
             out.append(("decode1_chain_presplit", lambda: self.run_chain(True)))
             out.append(("decode1_chain_w16", lambda: self.run_chain16()))
             out.append(("ref_copy_67MB", lambda: self.ref_dst.copy_(self.ref_src)))
+            out.append(("ref_read_67MB", lambda: self.torch.sum(self.ref_read, dim=0, out=self.ref_acc[0])))
         return out
 
     def prefill(self):
@@ -611,7 +615,7 @@ def main():
 
     dec_names = ([f"decode{m}" for m in DECODE_M] + [f"decode{m}_presplit" for m in DECODE_M] +
                  [f"decode{m}_w16" for m in DECODE_M] +
-                 ["decode1_chain", "decode1_chain_presplit", "decode1_chain_w16", "ref_copy_67MB"])
+                 ["decode1_chain", "decode1_chain_presplit", "decode1_chain_w16", "ref_copy_67MB", "ref_read_67MB"])
     names = ["prefill"] + dec_names + ["kv_writer", "attention"]
     if args.only:
         keep = {"prefill": ["prefill"], "decode": dec_names,
@@ -681,6 +685,11 @@ def main():
         t = part_ms[f"decode{m}_w16"] / 1e3 / K
         dec[f"M{m}_fp16_weights_two_products"] = {"gbs": u["decode16_bytes"][m] / t / 1e9, "us": 1e6 * t,
                                                   "frac_hbm": u["decode16_bytes"][m] / t / 1e9 / hbm}
+    t = part_ms["ref_read_67MB"] / 1e3 / K
+    dec["streaming_read_reference"] = {
+        "us": 1e6 * t, "gbs": REF_COPY_BYTES / t / 1e9, "frac_hbm": REF_COPY_BYTES / t / 1e9 / hbm,
+        "note": "torch one-dimensional sum over 67 MB (a decode GEMM's weight bytes, read once), timed in the step "
+                "like the decode parts"}
     t = part_ms["ref_copy_67MB"] / 1e3 / K
     dec["streaming_copy_reference"] = {
         "us": 1e6 * t, "gbs": REF_COPY_BYTES / t / 1e9, "frac_hbm": REF_COPY_BYTES / t / 1e9 / hbm,
