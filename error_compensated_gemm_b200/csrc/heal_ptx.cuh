@@ -125,7 +125,7 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 }
 
 // ---------------------------------------------------------------------------------
-// TMA (tensor tile loads, no multicast)
+// FP32 helpers of the attention kernels' logit and softmax arithmetic
 // ---------------------------------------------------------------------------------
 // n (|n| < 2^22) as FP32, exactly: the integer lands in the mantissa of 1.5 * 2^23.
 __device__ __forceinline__ float small_int_to_float(int n) {
@@ -140,6 +140,9 @@ __device__ __forceinline__ float fast_exp2(float x) {
   return y;
 }
 
+// ---------------------------------------------------------------------------------
+// TMA (tensor tile loads, no multicast)
+// ---------------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
