@@ -510,7 +510,8 @@ def arm_config(n):
             "parallelism": f"independent shards x{n}" if n > 1 else "single GPU",
             "l2": "cold: before every part of a step, outside its events, a 256 MB buffer is written "
                   "and another 256 MB read (the part starts with none of its inputs in L2 and no dirty "
-                  "line of another part); part order: KV writer, prefill, attention, decode GEMMs"}
+                  "line of another part); part order: KV writer, prefill, attention, decode GEMMs, then two "
+                  "torch streaming references (a 67 MB copy and a 67 MB read; not this library's kernels)"}
 
 
 def reference_arm(args):
