@@ -119,11 +119,13 @@ class Workload:
         M, K, N = PREFILL
         so = seed_offset
         # L2 cleaning before every part of a step (outside the part's events): a buffer
-        # larger than L2 (126 MB) is written, then a second one is read, so that each part
-        # starts with none of its inputs in L2 and without another part's dirty lines, whose
-        # write-back it would otherwise pay for.
+        # larger than L2 (126 MB) is written, then two others are read, so that each part
+        # starts with none of its inputs in L2, without another part's dirty lines, whose
+        # write-back it would otherwise pay for, and after the write-backs of the flush's
+        # own lines (evicted by the first read) have drained during the second.
         self.l2_w = torch.zeros(L2_CLEAN_BYTES // 4, device=dev)
         self.l2_r = torch.zeros(L2_CLEAN_BYTES // 4, device=dev)
+        self.l2_r2 = torch.zeros(L2_CLEAN_BYTES // 4, device=dev)
         self.l2_acc = torch.zeros(1, device=dev)
         need = lambda part: only is None or only == part or (part == "kv_writer" and only == "attention")
         if need("prefill"):
@@ -274,6 +276,7 @@ class Workload:
     def l2_clean(self):
         self.l2_w.zero_()
         self.torch.sum(self.l2_r, dim=0, out=self.l2_acc[0])
+        self.torch.sum(self.l2_r2, dim=0, out=self.l2_acc[0])
 
     def run_graphs(self, ev=None):
         for name, g in self.graphs:
@@ -509,8 +512,8 @@ def arm_config(n):
                         "(B=8, 32q/8kv heads, D=128, context 8192)",
             "parallelism": f"independent shards x{n}" if n > 1 else "single GPU",
             "l2": "cold: before every part of a step, outside its events, a 256 MB buffer is written "
-                  "and another 256 MB read (the part starts with none of its inputs in L2 and no dirty "
-                  "line of another part); part order: KV writer, prefill, attention, decode GEMMs, then two "
+                  "and two other 256 MB buffers read (the part starts with none of its inputs in L2, no "
+                  "dirty line of another part and the flush's own write-backs drained); part order: KV writer, prefill, attention, decode GEMMs, then two "
                   "torch streaming references (a 67 MB copy and a 67 MB read; not this library's kernels)"}
 
 
